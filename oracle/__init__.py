@@ -1,0 +1,195 @@
+"""fp64 CPU oracle for the sparse-MoE FFN layer and the decode LRU expert cache.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
+CPU-baseline leg of bench.py, never by the product library.  The arithmetic
+lives in moe_oracle.c (plain loops, fp64); this module only builds it with
+gcc and marshals numpy arrays.  Every function cites, in moe_oracle.c, the
+passage of the source pages (or the OCP MX v1.0 spec) it follows.
+
+Parity pins: every function here is pinned by tests/test_oracle_pins.py
+against something other than itself (spec tables, brute force, numpy float64
+matmul, closed forms and invariants); none is "parity unpinned" except the
+pages' claim that the CPU/GPU merge is exact, which prints no number.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c -> liboracle.so (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i32, i64, dbl = ctypes.c_int, ctypes.c_long, ctypes.c_double
+        L.oracle_bf16_to_f64.restype = dbl
+        L.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        L.oracle_e2m1_to_f64.restype = dbl
+        L.oracle_e2m1_to_f64.argtypes = [ctypes.c_uint8]
+        L.oracle_e8m0_to_f64.restype = dbl
+        L.oracle_e8m0_to_f64.argtypes = [ctypes.c_uint8]
+        L.oracle_decode_matrix.argtypes = [i32, P, P, i64, i64, P]
+        L.oracle_router_logits.argtypes = [i32, i32, i32, P, P, P, P, P]
+        L.oracle_topk.argtypes = [i32, i32, i32, P, P, P]
+        L.oracle_permute.argtypes = [i32, i32, i32, i32, P, P, P, P]
+        L.oracle_expert_ffn.argtypes = [i32, i32, i32, P, P, P, P, P, P]
+        L.oracle_moe_layer.restype = i32
+        L.oracle_moe_layer.argtypes = [i32] * 7 + [P, i32, P, P, P] + [P] * 8 + [P, i32]
+        L.oracle_unit_rms.argtypes = [i32, i32, P, dbl, P]
+        L.oracle_lru_sim.restype = i32
+        L.oracle_lru_sim.argtypes = [i32, i32, i32, P, P, P, P, P, P, P]
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+# ---------------------------------------------------------------- decodes
+def bf16_to_f64(bits) -> float:
+    return lib().oracle_bf16_to_f64(int(bits))
+
+
+def e2m1_to_f64(code) -> float:
+    return lib().oracle_e2m1_to_f64(int(code))
+
+
+def e8m0_to_f64(b) -> float:
+    return lib().oracle_e8m0_to_f64(int(b))
+
+
+def decode_matrix(wdtype: int, w, scale, rows: int, cols: int) -> np.ndarray:
+    w = np.ascontiguousarray(w)
+    scale = _c(scale, np.uint8)
+    out = np.empty((rows, cols), dtype=np.float64)
+    lib().oracle_decode_matrix(wdtype, _p(w), _p(scale), rows, cols, _p(out))
+    return out
+
+
+# ---------------------------------------------------------------- steps
+def router_logits(x_bits, w_router, bias=None, with_absdot=False):
+    x = _c(x_bits, np.uint16)
+    w = _c(w_router, np.float32)
+    b = _c(bias, np.float32)
+    T, H = x.shape
+    E = w.shape[0]
+    out = np.empty((T, E), dtype=np.float64)
+    ad = np.empty((T, E), dtype=np.float64) if with_absdot else None
+    lib().oracle_router_logits(T, H, E, _p(x), _p(w), _p(b), _p(out), _p(ad))
+    return (out, ad) if with_absdot else out
+
+
+def topk(logits32, k: int):
+    l32 = _c(logits32, np.float32)
+    T, E = l32.shape
+    idx = np.empty((T, k), dtype=np.int32)
+    g = np.empty((T, k), dtype=np.float64)
+    lib().oracle_topk(T, E, k, _p(l32), _p(idx), _p(g))
+    return idx, g
+
+
+def permute(idx, num_experts: int, num_shared: int = 0):
+    idx = _c(idx, np.int32)
+    T, k = idx.shape
+    G = num_experts + (1 if num_shared else 0)
+    n = T * k + (T if num_shared else 0)
+    offsets = np.empty(G + 1, dtype=np.int32)
+    sf = np.empty(n, dtype=np.int32)
+    inv = np.empty(n, dtype=np.int32)
+    lib().oracle_permute(T, k, num_experts, 1 if num_shared else 0, _p(idx), _p(offsets), _p(sf), _p(inv))
+    return offsets, sf, inv
+
+
+def expert_ffn(wdtype: int, hidden: int, ffn: int, w13, w13_scale, w2, w2_scale, x64) -> np.ndarray:
+    """One token (fp64 vector) through one expert whose weights are passed unstacked."""
+    w13 = np.ascontiguousarray(w13)
+    w2 = np.ascontiguousarray(w2)
+    x = _c(x64, np.float64)
+    o = np.empty(hidden, dtype=np.float64)
+    lib().oracle_expert_ffn(hidden, ffn, wdtype, _p(w13), _p(_c(w13_scale, np.uint8)), _p(w2),
+                            _p(_c(w2_scale, np.uint8)), _p(x), _p(o))
+    return o
+
+
+def moe_layer(shape: dict, x_bits, idx, g, weights: dict, tokens=None, n_threads: int = 0) -> np.ndarray:
+    """y[n, H] in fp64 for the listed tokens (all if None), given routing (idx, g)."""
+    H, F, E, k, S, wd = (shape[n] for n in ("hidden", "ffn", "num_experts", "top_k", "num_shared", "wdtype"))
+    x = _c(x_bits, np.uint16)
+    T = x.shape[0]
+    idx = _c(idx, np.int32)
+    g = _c(g, np.float64)
+    tok = _c(tokens, np.int32)
+    n = T if tok is None else len(tok)
+    y = np.empty((n, H), dtype=np.float64)
+    keep = [np.ascontiguousarray(weights[key]) if weights.get(key) is not None else None
+            for key in ("w13", "w13_scale", "w2", "w2_scale", "shared_w13", "shared_w13_scale", "shared_w2", "shared_w2_scale")]
+    rc = lib().oracle_moe_layer(T, H, F, E, k, S, wd, _p(tok), n, _p(x), _p(idx), _p(g),
+                                *[_p(a) for a in keep], _p(y), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_moe_layer: token index out of range")
+    return y
+
+
+def unit_rms(y64, eps: float = 1e-6) -> np.ndarray:
+    y = _c(y64, np.float64)
+    T, H = y.shape
+    out = np.empty_like(y)
+    lib().oracle_unit_rms(T, H, _p(y), eps, _p(out))
+    return out
+
+
+def lru_sim(num_experts: int, n_slots: int, steps):
+    """steps: list of per-step expert-id lists.  Returns (slot, hit, slot_expert, hits, misses);
+    slot/hit are lists aligned with sorted(set(step))."""
+    uniq = [sorted(set(int(i) for i in s)) for s in steps]
+    counts = np.array([len(u) for u in uniq], dtype=np.int32)
+    ids = np.array([i for u in uniq for i in u], dtype=np.int32)
+    slot = np.empty(len(ids), dtype=np.int32)
+    hit = np.empty(len(ids), dtype=np.uint8)
+    se = np.empty((len(uniq), n_slots), dtype=np.int32)
+    h = ctypes.c_int64()
+    m = ctypes.c_int64()
+    rc = lib().oracle_lru_sim(num_experts, n_slots, len(uniq), _p(counts), _p(ids), _p(slot), _p(hit), _p(se),
+                              ctypes.byref(h), ctypes.byref(m))
+    if rc != 0:
+        raise ValueError("oracle_lru_sim: step larger than the slot count or id out of range")
+    out_slot, out_hit, b = [], [], 0
+    for u in uniq:
+        out_slot.append(slot[b:b + len(u)].tolist())
+        out_hit.append(hit[b:b + len(u)].astype(bool).tolist())
+        b += len(u)
+    return out_slot, out_hit, se, h.value, m.value
+
+
+def full_layer(shape: dict, x_bits, w_router, bias, weights: dict, logits32=None, tokens=None, n_threads: int = 0):
+    """Convenience: logits (fp64) -> top-k on the given fp32 logits (or on the fp64 logits
+    rounded to fp32 when none are given) -> y for the listed tokens."""
+    l64 = router_logits(x_bits, w_router, bias)
+    l32 = l64.astype(np.float32) if logits32 is None else np.asarray(logits32, dtype=np.float32)
+    idx, g = topk(l32, shape["top_k"])
+    y = moe_layer(shape, x_bits, idx, g, weights, tokens, n_threads)
+    return dict(logits64=l64, idx=idx, g=g, y=y)
