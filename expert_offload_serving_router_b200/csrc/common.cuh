@@ -1,0 +1,91 @@
+// Internal helpers shared by the libftmoe kernels and host code (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/ftmoe.h"
+
+namespace ftmoe {
+
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 8;
+constexpr int kGemmBN = 256;        // token rows per grouped-GEMM tile (max MMA N)
+constexpr int kPermChunk = 1024;    // flat pairs per counting-sort chunk
+constexpr int kSmallRoute = 32;     // T <= this: split-expert router + fused permute
+
+// ------------------------------------------------------------------ device scalar helpers
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
+__device__ __forceinline__ uint16_t f2bf(float f) {
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    return uint32_t(f2bf(lo)) | (uint32_t(f2bf(hi)) << 16);
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float silu_mul(float a, float b) { return a / (1.0f + __expf(-a)) * b; }
+
+// ------------------------------------------------------------------ workspace layout
+// One layout serves every entry point: a region is only touched by the steps that need it.
+struct WsLayout {
+    size_t logits, topk_idx, topk_w, offsets, sorted_flat, inv_pos;
+    size_t chunk_cnt, chunk_base, local_rank, sched, err;
+    size_t x_sorted, h, o_sorted;
+    size_t total;
+    int T, P, R, G, C;
+};
+
+__host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// sched region: [0] total GEMM tiles for BN, [1] n_active groups, [2..] ntile_off[G+1], then active[G]
+inline WsLayout make_layout(const ft_moe_shape& s, int T) {
+    WsLayout L{};
+    L.T = T;
+    L.P = T * s.top_k;
+    L.G = s.num_experts + (s.num_shared ? 1 : 0);
+    L.R = L.P + (s.num_shared ? T : 0);
+    L.C = (L.R + kPermChunk - 1) / kPermChunk;
+    if (L.C < 1) L.C = 1;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t r = o; o = align256(o + bytes); return r; };
+    L.err = take(sizeof(uint32_t) * 8);   // first: [0] device error flag, [1] route ticket
+    L.logits = take(sizeof(float) * size_t(T) * s.num_experts);
+    L.topk_idx = take(sizeof(int32_t) * size_t(L.P));
+    L.topk_w = take(sizeof(float) * size_t(L.P));
+    L.offsets = take(sizeof(int32_t) * size_t(L.G + 1));
+    L.sorted_flat = take(sizeof(int32_t) * size_t(L.R));
+    L.inv_pos = take(sizeof(int32_t) * size_t(L.R));
+    L.chunk_cnt = take(sizeof(int32_t) * size_t(L.C) * L.G);
+    L.chunk_base = take(sizeof(int32_t) * size_t(L.C) * L.G);
+    L.local_rank = take(sizeof(int32_t) * size_t(L.R));
+    L.sched = take(sizeof(int32_t) * size_t(2 + 2 * (L.G + 1)));
+    L.x_sorted = take(sizeof(uint16_t) * size_t(L.R) * s.hidden);
+    L.h = take(sizeof(uint16_t) * size_t(L.R) * s.ffn);
+    L.o_sorted = take(sizeof(uint16_t) * size_t(L.R) * s.hidden);
+    L.total = o;
+    return L;
+}
+
+// device error codes written into ws err[0]
+enum : uint32_t { kDevErrNone = 0, kDevErrBadExpert = 1, kDevErrTimeout = 2, kDevErrShape = 3 };
+
+}  // namespace ftmoe

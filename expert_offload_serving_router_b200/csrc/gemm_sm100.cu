@@ -1,0 +1,553 @@
+// Step 3 (prefill) -- grouped expert GEMMs on the 5th-generation tensor cores.
+//
+//   gate/up:  D[128 weight rows, N tokens] = W13_e[rows, H] . Xs[tokens, H]^T, then
+//             h[token, f] = silu(gate) * up  (fused epilogue), h stored bf16 [R, F]
+//   down:     D[128 hidden rows, N tokens] = W2_e[rows, F] . h[tokens, F]^T,
+//             o_sorted[token, hrow] stored bf16 [R, H]
+//
+// "Weights as A": the MMA M dimension (128) walks weight rows and N walks the tokens of
+// one expert group, so an expert with few tokens costs an MMA of N = round_up(n, 16)
+// instead of a padded 128-row tile.  The gate/up A tile interleaves gate and up rows in
+// blocks of 16 (rows 32i..32i+15 = gate f0+16i.., rows 32i+16..32i+31 = up f0+16i..), so
+// each TMEM lane quarter holds gate and up of the same 16 f values: lane l and l^16
+// exchange halves with one shuffle, no shared-memory round trip.
+//
+// Warp roles (one CTA per SM, persistent over a device-side tile list):
+//   warp 0      TMA producer (weights for BF16; activations always)
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2-5   epilogue (tcgen05.ld 32x32b, SwiGLU / bf16 stores)
+//   warps 6-9   MXFP4 only: load E2M1 codes + E8M0 scales with 128-bit loads, dequantise
+//               exactly to bf16 in registers and write the SW128 A tile to shared memory
+// Operands are K-major, 128-byte swizzled; accumulators fp32 in TMEM, double buffered
+// (2 x 256 columns) so the epilogue of tile i overlaps the MMAs of tile i+1.
+// Every wait is bounded: on timeout the kernel records kDevErrTimeout, drains its own
+// copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include "kernels.h"
+
+namespace ftmoe {
+
+constexpr int kStages = 4;
+constexpr int kBK = 64;                       // K per stage (one 128-byte swizzle atom of bf16)
+constexpr int kATileBytes = 128 * kBK * 2;    // 16 KB
+constexpr int kBTileBytes = kGemmBN * kBK * 2;// 32 KB
+constexpr int kAccCols = 256;
+constexpr unsigned long long kWaitNs = 4000000000ull;  // 4 s bound on any wait
+
+struct GemmParams {
+    int mode;               // 0 gate/up, 1 down
+    int K;                  // H or F
+    int m_tiles;            // F/64 (gate/up) or H/128 (down)
+    int G, E, F, H;
+    int has_shared;
+    const int32_t* offsets; // [G+1]
+    const int32_t* sched;   // [0] n-tiles, [2..2+G] ntile_off
+    uint16_t* out;          // h [R,F] or o_sorted [R,H]
+    int out_ld;
+    uint32_t* err;
+    int b_bytes;            // bytes of one activation box (rows x 128 B); rows = min(256, round_up(R, 16))
+    // MXFP4 weights (A operand built by converter warps)
+    const uint8_t* wq;      // routed codes  [E, rows, K/2]
+    const uint8_t* ws;      // routed scales [E, rows, K/32]
+    const uint8_t* swq;     // shared codes  [1, rows, K/2]
+    const uint8_t* sws;     // shared scales
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t su32(const void* p) { return uint32_t(__cvta_generic_to_shared(p)); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t n) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(su32(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t gtimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait.  Gives up when `abort` is raised by another role or after kWaitNs.
+__device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort) {
+    if (mbar_try(b, parity)) return true;
+    const uint64_t t0 = gtimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try(b, parity)) return true;
+        if ((i & 31) == 0) {
+            if (abort && *abort) return false;
+            if (gtimer() - t0 > kWaitNs) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_2d(const CUtensorMap* m, uint64_t* bar, void* dst, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(su32(dst)), "l"(m), "r"(su32(bar)), "r"(c0), "r"(c1) : "memory");
+}
+__device__ __forceinline__ void tma_3d(const CUtensorMap* m, uint64_t* bar, void* dst, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(su32(dst)), "l"(m), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
+__device__ __forceinline__ void tma_4d(const CUtensorMap* m, uint64_t* bar, void* dst, int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(su32(dst)), "l"(m), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// K-major, 128-byte swizzle, canonical 8-row x 128-byte atoms: LBO = 16 B, SBO = 1024 B, version 1.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+    uint64_t d = uint64_t((saddr >> 4) & 0x3FFFu);
+    d |= uint64_t(1) << 16;
+    d |= uint64_t(1024 >> 4) << 32;
+    d |= uint64_t(1) << 46;
+    d |= uint64_t(2) << 61;
+    return d;
+}
+// kind::f16 instruction descriptor: BF16 x BF16 -> F32, both K-major, M x N.
+__device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_bf16(uint32_t dtm, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(dtm), "l"(ad), "l"(bd), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------------ exact MXFP4 -> bf16
+// Eight E2M1 codes (byte i: element 2i in the low nibble, 2i+1 in the high nibble) to four
+// bf16x2 words, scaled by the block's E8M0 scale.  Magnitudes {0,.5,1,1.5,2,3,4,6} are
+// looked up with byte permutes (bf16 high / low bytes), the sign bit is moved in, and the
+// power-of-two scale multiply is exact in bf16.
+__device__ __forceinline__ void e2m1x8_bf16(uint32_t w, uint32_t scale2, uint32_t (&o)[4]) {
+    const uint32_t HB_LO = 0x3F3F3F00u, HB_HI = 0x40404040u;
+    const uint32_t LB_LO = 0xC0800000u, LB_HI = 0xC0804000u;
+    const uint32_t mag = w & 0x77777777u;
+    const uint32_t hb0 = __byte_perm(HB_LO, HB_HI, mag);
+    const uint32_t lb0 = __byte_perm(LB_LO, LB_HI, mag);
+    const uint32_t hb1 = __byte_perm(HB_LO, HB_HI, mag >> 16);
+    const uint32_t lb1 = __byte_perm(LB_LO, LB_HI, mag >> 16);
+    const uint32_t s_lo = (w << 4) & 0x80808080u;
+    const uint32_t s_hi = w & 0x80808080u;
+    uint32_t v[4];
+    v[0] = __byte_perm(lb0, hb0, 0x5140);
+    v[1] = __byte_perm(lb0, hb0, 0x7362);
+    v[2] = __byte_perm(lb1, hb1, 0x5140);
+    v[3] = __byte_perm(lb1, hb1, 0x7362);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t sg = __byte_perm(s_lo, s_hi, 0x4000u + 0x1111u * i) & 0x80008000u;
+        uint32_t x = v[i] | sg;
+        asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o[i]) : "r"(x), "r"(scale2));
+    }
+}
+__device__ __forceinline__ uint32_t e8m0_bf16x2(uint32_t s) {
+    uint32_t b = s == 0 ? 0x0040u : (s == 255 ? 0x7FC0u : (s << 7));
+    return b | (b << 16);
+}
+
+// ------------------------------------------------------------------ tile schedule
+struct Tile { int g, m, row0, nvalid; };
+
+__device__ __forceinline__ Tile decode_tile(int t, const int* ntile_off, int G, const int32_t* offsets, int m_tiles) {
+    Tile r;
+    int u = t / m_tiles;
+    r.m = t - u * m_tiles;
+    int lo = 0, hi = G;   // largest g with ntile_off[g] <= u
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (ntile_off[mid] <= u) lo = mid; else hi = mid;
+    }
+    r.g = lo;
+    int ni = u - ntile_off[lo];
+    r.row0 = offsets[lo] + ni * kGemmBN;
+    r.nvalid = min(kGemmBN, offsets[lo + 1] - r.row0);
+    return r;
+}
+
+template <bool MX>
+__global__ void __launch_bounds__(MX ? 320 : 192, 1)
+moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sw,
+                const __grid_constant__ CUtensorMap tm_act, GemmParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * kATileBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kBTileBytes);
+    uint64_t* empty = full + kStages;
+    uint64_t* tfull = empty + kStages;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* mma_done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* ntile_off = const_cast<int*>(reinterpret_cast<volatile int*>(tmem_slot + 2));
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = p.G;
+    for (int i = tid; i <= G; i += blockDim.x) ntile_off[i] = p.sched[2 + i];
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], MX ? 1 + 4 : 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                     "r"(2 * kAccCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int total = ntile_off[G] * p.m_tiles;
+    const int nk = p.K / kBK;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued[kStages];
+            uint32_t issued_par[kStages];
+            for (int s = 0; s < kStages; ++s) issued[s] = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                Tile tl = decode_tile(t, ntile_off, G, p.offsets, p.m_tiles);
+                const bool shared_grp = p.has_shared && tl.g == p.E;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    uint8_t* a = sA + stage * kATileBytes;
+                    uint8_t* b = sB + stage * kBTileBytes;
+                    const int k0 = kb * kBK;
+                    if (!MX) {
+                        mbar_expect_tx(&full[stage], kATileBytes + p.b_bytes);
+                        if (p.mode == 0) {
+                            const CUtensorMap* m = shared_grp ? &tm_sw : &tm_w;
+                            const int e = shared_grp ? 0 : tl.g;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                tma_4d(m, &full[stage], a + i * 4096, k0, tl.m * 64 + 16 * i, 0, e);
+                        } else {
+                            const CUtensorMap* m = shared_grp ? &tm_sw : &tm_w;
+                            tma_3d(m, &full[stage], a, k0, tl.m * 128, shared_grp ? 0 : tl.g);
+                        }
+                    } else {
+                        mbar_expect_tx(&full[stage], p.b_bytes);
+                    }
+                    tma_2d(&tm_act, &full[stage], b, k0, tl.row0);
+                    issued[stage] = 1;
+                    issued_par[stage] = phase;
+                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+            // drain: every copy this thread issued must have landed before the CTA exits
+            for (int s = 0; s < kStages; ++s)
+                if (issued[s]) mbar_wait(&full[s], issued_par[s], nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                Tile tl = decode_tile(t, ntile_off, G, p.offsets, p.m_tiles);
+                const int N = (tl.nvalid + 15) & ~15;
+                const uint32_t idesc = idesc_bf16(128, N);
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t dtm = tmem_base + uint32_t(acc * kAccCols);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t ad = sdesc_sw128(su32(sA + stage * kATileBytes));
+                    const uint64_t bd = sdesc_sw128(su32(sB + stage * kBTileBytes));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        umma_bf16(dtm, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+                    umma_commit(&empty[stage]);
+                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[acc]);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+            if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+            umma_commit(mma_done);               // tracks completion of every MMA issued above
+            mbar_wait(mma_done, 0, nullptr);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------ epilogue (TMEM -> registers -> global)
+        const int q = warp & 3;                  // TMEM lanes 32q .. 32q+31
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            Tile tl = decode_tile(t, ntile_off, G, p.offsets, p.m_tiles);
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols);
+            const int nch = (tl.nvalid + 31) >> 5;
+            for (int c = 0; c < nch; ++c) {
+                float v[32];
+                tmem_ld32(tbase + uint32_t(c * 32), v);
+                if (p.mode == 0) {
+                    const int f = tl.m * 64 + 16 * q + (lane & 15);
+                    const bool lo = lane < 16;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float send = lo ? v[16 + i] : v[i];
+                        float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+                        float gt = lo ? v[i] : recv;
+                        float up = lo ? recv : v[16 + i];
+                        int n = c * 32 + (lo ? i : 16 + i);
+                        if (n < tl.nvalid)
+                            p.out[size_t(tl.row0 + n) * p.out_ld + f] = f2bf(silu_mul(gt, up));
+                    }
+                } else {
+                    const int hrow = tl.m * 128 + 32 * q + lane;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        int n = c * 32 + j;
+                        if (n < tl.nvalid) p.out[size_t(tl.row0 + n) * p.out_ld + hrow] = f2bf(v[j]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        }
+        if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
+    } else if (MX) {
+        // ------------------------------------------------ MXFP4 converter warps (one A row per thread)
+        const int r = tid - 192;                 // 0..127
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        const int kq = p.K / 2, ks = p.K / 32;   // code / scale bytes per weight row
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            Tile tl = decode_tile(t, ntile_off, G, p.offsets, p.m_tiles);
+            const bool shared_grp = p.has_shared && tl.g == p.E;
+            int wrow;
+            size_t rows_per_expert;
+            if (p.mode == 0) {
+                const int i = r >> 5, j = r & 31;
+                const int f = tl.m * 64 + 16 * i + (j & 15);
+                wrow = j < 16 ? f : p.F + f;
+                rows_per_expert = size_t(2) * p.F;
+            } else {
+                wrow = tl.m * 128 + r;
+                rows_per_expert = size_t(p.H);
+            }
+            const size_t e = shared_grp ? 0 : size_t(tl.g);
+            const uint8_t* qrow = (shared_grp ? p.swq : p.wq) + (e * rows_per_expert + wrow) * kq;
+            const uint8_t* srow = (shared_grp ? p.sws : p.ws) + (e * rows_per_expert + wrow) * ks;
+            uint4 c0 = ldg_nc_v4(qrow), c1 = ldg_nc_v4(qrow + 16);
+            uint32_t sc = *reinterpret_cast<const uint16_t*>(srow);
+            for (int kb = 0; kb < nk; ++kb) {
+                uint4 n0 = c0, n1 = c1;
+                uint32_t nsc = sc;
+                if (kb + 1 < nk) {
+                    n0 = ldg_nc_v4(qrow + (kb + 1) * 32);
+                    n1 = ldg_nc_v4(qrow + (kb + 1) * 32 + 16);
+                    nsc = *reinterpret_cast<const uint16_t*>(srow + (kb + 1) * 2);
+                }
+                if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                uint8_t* arow = sA + stage * kATileBytes + r * 128;
+                const uint32_t s0 = e8m0_bf16x2(sc & 0xFF), s1 = e8m0_bf16x2(sc >> 8);
+                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                for (int cch = 0; cch < 8; ++cch) {      // 16-byte chunk cch = elements 8cch..8cch+7
+                    uint32_t o[4];
+                    e2m1x8_bf16(words[cch], cch < 4 ? s0 : s1, o);
+                    *reinterpret_cast<uint4*>(arow + ((cch ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[stage]);
+                if (++stage == kStages) { stage = 0; phase ^= 1; }
+                c0 = n0; c1 = n1; sc = nsc;
+            }
+        }
+        if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(2 * kAccCols));
+    }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// bf16 tensor map, dims/strides innermost first (strides in bytes, rank-1 entries)
+static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                     const uint32_t* box) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t d[5], s[4];
+    cuuint32_t b[5], es[5];
+    for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; es[i] = 1; }
+    for (int i = 0; i < rank - 1; ++i) s[i] = strides[i];
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cuuint32_t(rank), const_cast<void*>(base), d, s, b, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+static size_t gemm_smem_bytes() { return 1024 + kStages * (kATileBytes + kBTileBytes) + 256 + 4 * 260; }
+
+
+
+// returns 0 ok, 1 tensor-map failure, 2 launch failure
+int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
+    const bool mx = L.wdtype == FT_W_MXFP4;
+    const int K = L.mode == 0 ? L.H : L.F;
+    CUtensorMap tw{}, tsw{}, tact{};
+    if (!mx) {
+        if (L.mode == 0) {
+            uint64_t dims[4] = {uint64_t(L.H), uint64_t(L.F), 2, uint64_t(L.E)};
+            uint64_t str[3] = {uint64_t(L.H) * 2, uint64_t(L.F) * L.H * 2, uint64_t(2) * L.F * L.H * 2};
+            uint32_t box[4] = {kBK, 16, 2, 1};
+            if (!make_map(&tw, L.w, 4, dims, str, box)) return 1;
+            if (L.S) {
+                uint64_t d1[4] = {uint64_t(L.H), uint64_t(L.F), 2, 1};
+                if (!make_map(&tsw, L.sw, 4, d1, str, box)) return 1;
+            } else {
+                tsw = tw;
+            }
+        } else {
+            uint64_t dims[3] = {uint64_t(L.F), uint64_t(L.H), uint64_t(L.E)};
+            uint64_t str[2] = {uint64_t(L.F) * 2, uint64_t(L.H) * L.F * 2};
+            uint32_t box[3] = {kBK, 128, 1};
+            if (!make_map(&tw, L.w, 3, dims, str, box)) return 1;
+            if (L.S) {
+                uint64_t d1[3] = {uint64_t(L.F), uint64_t(L.H), 1};
+                if (!make_map(&tsw, L.sw, 3, d1, str, box)) return 1;
+            } else {
+                tsw = tw;
+            }
+        }
+    }
+    const int box_rows = L.R >= kGemmBN ? kGemmBN : ((L.R + 15) & ~15);
+    {
+        uint64_t dims[2] = {uint64_t(K), uint64_t(L.R)};
+        uint64_t str[1] = {uint64_t(K) * 2};
+        uint32_t box[2] = {kBK, uint32_t(box_rows)};
+        if (!make_map(&tact, L.act, 2, dims, str, box)) return 1;
+    }
+    if (mx) { tw = tact; tsw = tact; }   // unused by the MXFP4 kernel
+    GemmParams p{};
+    p.mode = L.mode;
+    p.K = K;
+    p.m_tiles = L.mode == 0 ? L.F / 64 : L.H / 128;
+    p.G = L.E + (L.S ? 1 : 0);
+    p.E = L.E;
+    p.F = L.F;
+    p.H = L.H;
+    p.has_shared = L.S ? 1 : 0;
+    p.offsets = L.offsets;
+    p.sched = L.sched;
+    p.out = L.out;
+    p.out_ld = L.mode == 0 ? L.F : L.H;
+    p.err = L.err;
+    p.b_bytes = box_rows * kBK * 2;
+    p.wq = static_cast<const uint8_t*>(L.w);
+    p.ws = L.wscale;
+    p.swq = static_cast<const uint8_t*>(L.sw);
+    p.sws = L.swscale;
+    const size_t smem = gemm_smem_bytes();
+    int grid = num_sms();
+    int max_tiles = L.max_tiles * p.m_tiles;
+    if (max_tiles < grid) grid = max_tiles > 0 ? max_tiles : 1;
+    if (mx) {
+        static bool set = false;
+        if (!set) {
+            if (cudaFuncSetAttribute(moe_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 2;
+            set = true;
+        }
+        moe_gemm_kernel<true><<<grid, 320, smem, st>>>(tw, tsw, tact, p);
+    } else {
+        static bool set = false;
+        if (!set) {
+            if (cudaFuncSetAttribute(moe_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 2;
+            set = true;
+        }
+        moe_gemm_kernel<false><<<grid, 192, smem, st>>>(tw, tsw, tact, p);
+    }
+    return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
+
+}  // namespace ftmoe

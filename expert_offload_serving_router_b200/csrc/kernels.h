@@ -1,0 +1,69 @@
+// Internal launcher declarations shared by the kernel files and the C-ABI layer.
+#pragma once
+#include "common.cuh"
+#include "permute_small.cuh"
+
+namespace ftmoe {
+
+struct DecodeArgs {
+    int T, k, E, S, H, F, wdtype;
+    const uint16_t* x;
+    const int32_t* offsets;
+    const int32_t* sorted_flat;
+    const int32_t* sched;       // [1] n_active, active list at [2 + G + 1 ...]
+    const uint8_t* w13;
+    const uint8_t* w13s;
+    const uint8_t* w2;
+    const uint8_t* w2s;
+    const void* const* eptr;    // optional [E][4] {w13, w13s, w2, w2s}
+    const uint8_t* sw13;
+    const uint8_t* sw13s;
+    const uint8_t* sw2;
+    const uint8_t* sw2s;
+    uint16_t* h;                // [R, F]
+    const int32_t* inv_pos;
+    const float* topk_w;
+    uint16_t* y;                // [T, H] or NULL
+    uint16_t* o_sorted;         // [R, H] when y == NULL
+};
+
+struct GemmLaunch {
+    int mode;                 // 0 gate/up, 1 down
+    int wdtype;
+    int H, F, E, S, R;        // R = rows of the activation operand
+    const void* w;            // bf16 weights or MXFP4 codes (routed)
+    const uint8_t* wscale;
+    const void* sw;           // shared expert weights / codes (S=1)
+    const uint8_t* swscale;
+    const void* act;          // x_sorted [R,H] (gate/up) or h [R,F] (down), bf16
+    const int32_t* offsets;
+    const int32_t* sched;
+    uint16_t* out;
+    uint32_t* err;
+    int max_tiles;            // host upper bound on tiles (grid sizing)
+};
+
+template <class T> inline T* ws_at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off); }
+
+// host helpers of the C-ABI layer (api.cu)
+ft_status fail(ft_status s, const char* fmt, ...);
+ft_status check_shape(const ft_moe_shape* s);
+ft_status cuda_ok(cudaError_t e, const char* what);
+ft_status cuda_state();
+DecodeArgs decode_args(const ft_moe_shape* s, int T, const ft_moe_weights* w, const void* x, const WsLayout& L,
+                       void* ws, const int32_t* offsets, const int32_t* sorted_flat, const int32_t* inv_pos,
+                       const float* topk_w, void* y, void* o_sorted);
+
+cudaError_t launch_route(int T, int H, int E, int k, int S, const uint16_t* x, const float* wr, const float* bias,
+                         int32_t* topk_idx, float* topk_w, float* logits, uint32_t* ticket, const PermOut* perm,
+                         cudaStream_t st);
+cudaError_t launch_permute(int T, int k, int E, int S, int H, const int32_t* idx, const uint16_t* x,
+                           uint16_t* x_sorted, int32_t* chunk_cnt, int32_t* chunk_base, int32_t* local_rank,
+                           const PermOut& out, cudaStream_t st);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st);
+cudaError_t launch_combine(int T, int H, int k, int S, int R, const uint16_t* o, const int32_t* inv_pos,
+                           const float* gw, uint16_t* y, cudaStream_t st);
+cudaError_t launch_unit_rms(int T, int H, const uint16_t* in, uint16_t* out, float eps, cudaStream_t st);
+
+}  // namespace ftmoe

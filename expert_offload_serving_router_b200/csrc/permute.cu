@@ -1,0 +1,180 @@
+// Step 2 -- permutation: stable counting sort of the flat pairs p = t*k + j by expert id,
+// the shared expert (S = 1) appended as group E holding tokens in order (flat id P + t).
+//
+// General path (three launches, any R):
+//   perm_count:   one CTA per 1024-pair chunk; per-chunk histogram and each pair's stable
+//                 rank inside its chunk (warp __match_any_sync + per-warp counts).
+//   perm_scan:    one CTA; per-group running sums over chunks (chunk bases), exclusive
+//                 scan over groups (offsets), GEMM tile schedule and active-group list.
+//   perm_scatter: one CTA per chunk; pos = chunk base + local rank; writes sorted_flat,
+//                 inv_pos and (optionally) gathers x rows into x_sorted with 16-byte moves.
+// Small path (R <= 1024): one CTA does all of it (block_permute_small).
+#include "kernels.h"
+#include "permute_small.cuh"
+
+namespace ftmoe {
+
+struct PermArgs {
+    int T, k, E, S, H;
+    const int32_t* idx;
+    const uint16_t* x;
+    uint16_t* x_sorted;
+    int32_t* chunk_cnt;    // [C][G]
+    int32_t* chunk_base;   // [C][G]
+    int32_t* local_rank;   // [R]
+    PermOut out;
+};
+
+__device__ __forceinline__ int pair_group(const PermArgs& a, int i, int P) {
+    if (i >= P) return a.E;
+    int g = a.idx[i];
+    return (g >= 0 && g < a.E) ? g : -1;
+}
+
+__global__ void __launch_bounds__(256) perm_count_kernel(PermArgs a) {
+    __shared__ int run[kMaxExperts + 2];
+    __shared__ int wcnt[8][kMaxExperts + 2];
+    const int P = a.T * a.k, R = P + (a.S ? a.T : 0), G = a.E + (a.S ? 1 : 0);
+    const int c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int g = tid; g < G; g += 256) run[g] = 0;
+    for (int sub = 0; sub < kPermChunk / 256; ++sub) {
+        for (int i = tid; i < 8 * (kMaxExperts + 2); i += 256) (&wcnt[0][0])[i] = 0;
+        __syncthreads();
+        const int i = c * kPermChunk + sub * 256 + tid;
+        int g = i < R ? pair_group(a, i, P) : -2;
+        if (g == -1) atomicExch(a.out.err, kDevErrBadExpert);
+        unsigned peers = __match_any_sync(0xffffffffu, g);
+        int rk = __popc(peers & ((1u << lane) - 1u));
+        if (g >= 0 && rk == 0) wcnt[warp][g] = __popc(peers);
+        __syncthreads();
+        if (g >= 0) {
+            int before = run[g];
+            for (int w = 0; w < warp; ++w) before += wcnt[w][g];
+            a.local_rank[i] = before + rk;
+        }
+        __syncthreads();
+        for (int gg = tid; gg < G; gg += 256) {
+            int s = 0;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) s += wcnt[w][gg];
+            run[gg] += s;
+        }
+    }
+    __syncthreads();
+    for (int g = tid; g < G; g += 256) a.chunk_cnt[size_t(c) * G + g] = run[g];
+}
+
+__global__ void __launch_bounds__(1024) perm_scan_kernel(PermArgs a, int C) {
+    __shared__ int tot[kMaxExperts + 2];
+    __shared__ int flag[kMaxExperts + 2];
+    __shared__ int tmp[33];
+    const int G = a.E + (a.S ? 1 : 0);
+    const int g = threadIdx.x;
+    if (g < G) {
+        int r = 0;
+        for (int c = 0; c < C; ++c) {
+            int v = a.chunk_cnt[size_t(c) * G + g];
+            a.chunk_base[size_t(c) * G + g] = r;
+            r += v;
+        }
+        tot[g] = r;
+        flag[g] = r > 0 ? 1 : 0;
+    }
+    __syncthreads();
+    int n_active = block_exclusive_scan(flag, G, tmp);
+    if (g < G) {
+        if (tot[g] > 0) a.out.sched[2 + (G + 1) + flag[g]] = g;
+    }
+    __syncthreads();
+    if (g < G) flag[g] = (tot[g] + kGemmBN - 1) / kGemmBN;
+    __syncthreads();
+    int ntiles = block_exclusive_scan(flag, G, tmp);
+    if (g < G) a.out.sched[2 + g] = flag[g];
+    if (g == 0) {
+        a.out.sched[0] = ntiles;
+        a.out.sched[1] = n_active;
+        a.out.sched[2 + G] = ntiles;
+    }
+    int total = block_exclusive_scan(tot, G, tmp);
+    if (g < G) {
+        a.out.offsets[g] = tot[g];
+        for (int c = 0; c < C; ++c) a.chunk_base[size_t(c) * G + g] += tot[g];
+    }
+    if (g == 0) a.out.offsets[G] = total;
+}
+
+__global__ void __launch_bounds__(256) perm_scatter_kernel(PermArgs a) {
+    __shared__ int spos[kPermChunk];
+    __shared__ int stok[kPermChunk];
+    const int P = a.T * a.k, R = P + (a.S ? a.T : 0), G = a.E + (a.S ? 1 : 0);
+    const int c = blockIdx.x, tid = threadIdx.x;
+    const int i0 = c * kPermChunk;
+    const int n = min(kPermChunk, R - i0);
+    for (int q = tid; q < n; q += 256) {
+        int i = i0 + q;
+        int g = pair_group(a, i, P);
+        int pos = -1;
+        if (g >= 0) {
+            pos = a.chunk_base[size_t(c) * G + g] + a.local_rank[i];
+            a.out.sorted_flat[pos] = i;
+            a.out.inv_pos[i] = pos;
+        }
+        spos[q] = pos;
+        stok[q] = i < P ? i / a.k : i - P;
+    }
+    if (!a.x_sorted) return;
+    __syncthreads();
+    // gather: one warp per row, 16-byte vectors
+    const int lane = tid & 31, warp = tid >> 5;
+    const int nv = a.H / 8;
+    for (int q = warp; q < n; q += 8) {
+        int pos = spos[q];
+        if (pos < 0) continue;
+        const uint4* src = reinterpret_cast<const uint4*>(a.x + size_t(stok[q]) * a.H);
+        uint4* dst = reinterpret_cast<uint4*>(a.x_sorted + size_t(pos) * a.H);
+        for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+    }
+}
+
+__global__ void __launch_bounds__(256) perm_small_kernel(const int32_t* idx, int T, int k, int E, int S, PermOut out,
+                                                         const uint16_t* x, uint16_t* x_sorted, int H) {
+    __shared__ int32_t sidx[1024];
+    __shared__ int grp[1024];
+    __shared__ int cnt[kMaxExperts + 2];
+    __shared__ int flag[kMaxExperts + 2];
+    __shared__ int tmp[33];
+    const int P = T * k, R = P + (S ? T : 0);
+    for (int i = threadIdx.x; i < P; i += blockDim.x) sidx[i] = idx[i];
+    __syncthreads();
+    block_permute_small(sidx, T, k, E, S, grp, cnt, flag, tmp, out);
+    if (!x_sorted) return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nv = H / 8;
+    for (int i = warp; i < R; i += blockDim.x / 32) {
+        if (grp[i] < 0) continue;
+        int pos = out.inv_pos[i];
+        int t = i < P ? i / k : i - P;
+        const uint4* src = reinterpret_cast<const uint4*>(x + size_t(t) * H);
+        uint4* dst = reinterpret_cast<uint4*>(x_sorted + size_t(pos) * H);
+        for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+    }
+}
+
+cudaError_t launch_permute(int T, int k, int E, int S, int H, const int32_t* idx, const uint16_t* x,
+                           uint16_t* x_sorted, int32_t* chunk_cnt, int32_t* chunk_base, int32_t* local_rank,
+                           const PermOut& out, cudaStream_t st) {
+    if (T <= 0) return cudaSuccess;
+    const int P = T * k, R = P + (S ? T : 0);
+    if (R <= 1024) {
+        perm_small_kernel<<<1, 256, 0, st>>>(idx, T, k, E, S, out, x, x_sorted, H);
+        return cudaGetLastError();
+    }
+    const int C = (R + kPermChunk - 1) / kPermChunk;
+    PermArgs a{T, k, E, S, H, idx, x, x_sorted, chunk_cnt, chunk_base, local_rank, out};
+    perm_count_kernel<<<C, 256, 0, st>>>(a);
+    perm_scan_kernel<<<1, 1024, 0, st>>>(a, C);
+    perm_scatter_kernel<<<C, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace ftmoe

@@ -1,0 +1,158 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+symbol include/ftmoe.h declares, sizes workspaces, rejects bad arguments before any
+CUDA call, and its host LRU policy matches the oracle's simulator."""
+import ctypes
+import random
+
+import numpy as np
+import pytest
+
+import oracle
+from expert_offload_serving_router_b200 import build as ftbuild
+from expert_offload_serving_router_b200 import ftmoe as F
+from expert_offload_serving_router_b200 import inputs
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    ftbuild.build()
+
+
+def test_exports_every_header_symbol():
+    names = F.header_functions()
+    assert len(names) >= 20
+    L = ctypes.CDLL(F.LIB_PATH)
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    assert set(F._SIGS) == set(names)
+
+
+def test_version_and_threshold():
+    assert "sm_100a" in F.ft_version()
+    prev = F.ft_set_decode_max_tokens(7)
+    assert F.ft_get_decode_max_tokens() == 7
+    assert F.ft_set_decode_max_tokens(1000) == 7 and F.ft_get_decode_max_tokens() == 32
+    assert F.ft_set_decode_max_tokens(-1) == -1
+    F.ft_set_decode_max_tokens(prev)
+
+
+def _shape(name):
+    c = inputs.CONFIGS[name]
+    return F.make_shape(c.hidden, c.ffn, c.num_experts, c.top_k, c.num_shared, c.wdtype)
+
+
+def test_workspace_bytes_grow_with_tokens():
+    s = _shape("qwen3_a3b")
+    a, b = F.ft_moe_workspace_bytes(s, 16), F.ft_moe_workspace_bytes(s, 4096)
+    assert 0 < a < b
+    # x_sorted + h + o_sorted dominate: R*(2H + F)*2 bytes
+    R = 4096 * 8
+    assert b >= R * (2 * 2048 + 768) * 2
+    assert F.ft_moe_workspace_bytes(F.make_shape(100, 512, 8, 2), 4) == 0     # H % 128 != 0
+    assert F.ft_moe_workspace_bytes(s, -1) == 0
+
+
+FAKE = 1 << 20   # 16-byte aligned non-null address; never dereferenced (validation fails first)
+
+
+@pytest.mark.parametrize("shape,code", [
+    (F.make_shape(100, 512, 8, 2), F.FT_ERR_UNSUPPORTED),
+    (F.make_shape(256, 500, 8, 2), F.FT_ERR_UNSUPPORTED),
+    (F.make_shape(256, 512, 300, 2), F.FT_ERR_UNSUPPORTED),
+    (F.make_shape(256, 512, 8, 9), F.FT_ERR_UNSUPPORTED),
+    (F.make_shape(256, 512, 4, 5), F.FT_ERR_UNSUPPORTED),
+    (F.make_shape(256, 512, 8, 0), F.FT_ERR_INVALID_ARG),
+    (F.make_shape(256, 512, 8, 2, num_shared=2), F.FT_ERR_INVALID_ARG),
+    (F.make_shape(256, 512, 8, 2, wdtype=7), F.FT_ERR_INVALID_ARG),
+])
+def test_bad_shapes_rejected_on_host(shape, code):
+    with pytest.raises(F.FtError) as ei:
+        F.ft_moe_route(shape, 4, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, 1 << 30, stream=0)
+    assert ei.value.status == code
+
+
+def test_bad_pointers_and_workspace_rejected_on_host():
+    s = _shape("tiny")
+    with pytest.raises(F.FtError) as ei:
+        F.ft_moe_route(s, 4, None, FAKE, None, FAKE, FAKE, None, FAKE, 1 << 30, stream=0)
+    assert ei.value.status == F.FT_ERR_INVALID_ARG
+    with pytest.raises(F.FtError) as ei:
+        F.ft_moe_route(s, 4, FAKE + 2, FAKE, None, FAKE, FAKE, None, FAKE, 1 << 30, stream=0)
+    assert ei.value.status == F.FT_ERR_INVALID_ARG and "aligned" in str(ei.value)
+    with pytest.raises(F.FtError) as ei:
+        F.ft_moe_route(s, 4, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, 64, stream=0)
+    assert ei.value.status == F.FT_ERR_WORKSPACE
+    with pytest.raises(F.FtError) as ei:
+        F.ft_moe_route(s, 4, FAKE, FAKE, None, FAKE, FAKE, None, FAKE + 16, 1 << 30, stream=0)
+    assert ei.value.status == F.FT_ERR_INVALID_ARG
+    with pytest.raises(F.FtError) as ei:
+        F.ft_moe_route(s, -1, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, 1 << 30, stream=0)
+    assert ei.value.status == F.FT_ERR_INVALID_ARG
+    # T == 0 is a no-op that needs no pointers at all
+    F.ft_moe_route(s, 0, None, None, None, None, None, None, None, 0, stream=0)
+    F.ft_moe_layer_forward(s, 0, None, None, None, F.make_weights(), None, None, None, None, 0, stream=0)
+    w = F.make_weights()   # NULL weights
+    with pytest.raises(F.FtError) as ei:
+        F.ft_moe_layer_forward(s, 4, FAKE, FAKE, None, w, FAKE, None, None, FAKE, 1 << 30, stream=0)
+    assert ei.value.status == F.FT_ERR_INVALID_ARG
+    # expert_ptrs tables are decode-only
+    wt = F.make_weights(expert_ptrs=FAKE)
+    with pytest.raises(F.FtError) as ei:
+        F.ft_moe_layer_forward(s, 64, FAKE, FAKE, None, wt, FAKE, None, None, FAKE, 1 << 30, stream=0)
+    assert ei.value.status == F.FT_ERR_UNSUPPORTED
+    with pytest.raises(F.FtError) as ei:
+        F.ft_moe_unit_rms(4, 100, FAKE, FAKE, stream=0)
+    assert ei.value.status == F.FT_ERR_INVALID_ARG
+
+
+def test_stream_config_rejected_on_host():
+    s = _shape("dsv4_flash")
+    layers = (F.ft_moe_weights * 2)()
+    cfg = F.ft_stream_cfg(2, 8, s, layers, FAKE * 256, 1 << 20, 1000)
+    assert F.ft_expert_stream_arena_bytes(cfg) > 2 * 256 * 13_000_000
+    with pytest.raises(F.FtError) as ei:          # arena too small
+        F.ft_expert_stream_create(cfg)
+    assert ei.value.status == F.FT_ERR_WORKSPACE
+    cfg.slots_per_layer = 3                       # fewer slots than k = 6
+    with pytest.raises(F.FtError) as ei:
+        F.ft_expert_stream_create(cfg)
+    assert ei.value.status == F.FT_ERR_INVALID_ARG
+    cfg.slots_per_layer = 8
+    cfg.hbm_arena_bytes = F.ft_expert_stream_arena_bytes(cfg)
+    with pytest.raises(F.FtError) as ei:          # NULL host pointers
+        F.ft_expert_stream_create(cfg)
+    assert ei.value.status == F.FT_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_host_lru_policy_matches_oracle(seed):
+    r = random.Random(100 + seed)
+    E, n_slots = r.choice([(8, 3), (64, 8), (256, 32)])
+    steps = []
+    for _ in range(80):
+        kk = r.randint(0, min(6, n_slots))
+        steps.append(sorted(set(min(E - 1, int(r.paretovariate(0.8)) - 1 + r.randint(0, 3)) for _ in range(kk))))
+    oslot, ohit, ose, h, m = oracle.lru_sim(E, n_slots, steps)
+    content = np.full(n_slots, -1, np.int32)
+    stamp = np.full(n_slots, -1, np.int64)
+    where = np.full(E, -1, np.int32)
+    for s, ids in enumerate(steps):
+        ids_a = np.array(ids, np.int32)
+        out_slot = np.empty(len(ids), np.int32)
+        out_hit = np.empty(len(ids), np.uint8)
+        F.ft_lru_step(E, n_slots, content, stamp, where, s, ids_a, out_slot, out_hit)
+        assert out_slot.tolist() == oslot[s]
+        assert out_hit.astype(bool).tolist() == ohit[s]
+        assert content.tolist() == ose[s].tolist()
+
+
+def test_host_lru_rejects_unsorted_or_oversized():
+    content = np.full(2, -1, np.int32)
+    stamp = np.full(2, -1, np.int64)
+    where = np.full(8, -1, np.int32)
+    o = np.empty(3, np.int32)
+    hh = np.empty(3, np.uint8)
+    with pytest.raises(F.FtError):
+        F.ft_lru_step(8, 2, content, stamp, where, 0, np.array([1, 2, 3], np.int32), o, hh)
+    with pytest.raises(F.FtError):
+        F.ft_lru_step(8, 2, content, stamp, where, 0, np.array([2, 1], np.int32), o[:2], hh[:2])

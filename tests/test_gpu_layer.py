@@ -1,0 +1,155 @@
+"""GPU parity of the whole layer (route -> permute -> experts -> combine) against the
+fp64 oracle, through the C ABI.  Routing is bit-exact given the GPU's fp32 logits;
+outputs are within max|y - y64| <= 1e-2 max|y64| (BF16) / 3e-2 max|y64| (MXFP4)."""
+import numpy as np
+import pytest
+
+import oracle
+from expert_offload_serving_router_b200 import ftmoe as F
+from expert_offload_serving_router_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+_LAYERS = {}
+
+
+def layer(name, **kw):
+    from gpu_util import DevLayer, ensure_built
+    ensure_built()
+    key = (name, tuple(sorted(kw.items())))
+    if key not in _LAYERS:
+        cfg = inputs.CONFIGS[name] if name in inputs.CONFIGS else inputs.custom_config(**kw)
+        _LAYERS[key] = DevLayer(cfg, inputs.make_layer(cfg, seed=0))
+    return _LAYERS[key]
+
+
+def full_check(L, x, n_rows=12, seed=0):
+    from gpu_util import check_logits, check_y, oracle_rows, run_layer, sample_rows
+    y, idx, lg = run_layer(L, x)
+    rows = sample_rows(x.shape[0], n_rows, seed)
+    check_logits(x, L, lg, rows)
+    oidx, og, y64 = oracle_rows(L, x, lg, rows)
+    assert np.array_equal(idx, oidx), "routing differs from the oracle's top-k on the GPU logits"
+    rel = check_y(y[rows], y64, L.cfg.wdtype, f"{L.cfg.name} T={x.shape[0]}")
+    return y, idx, lg, rel
+
+
+CASES = [("tiny", 64), ("tiny", 1), ("tiny", 37),
+         ("qwen3_a3b", 1), ("qwen3_a3b", 4), ("qwen3_a3b", 16), ("qwen3_a3b", 4096),
+         ("dsv4_flash", 1), ("dsv4_flash", 8), ("dsv4_flash", 8192),
+         ("gemma4_26b_a4b", 1), ("gemma4_26b_a4b", 2048)]
+
+
+@pytest.mark.parametrize("name,T", CASES)
+def test_layer_matches_oracle(name, T):
+    L = layer(name)
+    x = inputs.make_tokens(L.cfg, T, seed=0)
+    full_check(L, x)
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 5), ("qwen3_a3b", 16), ("dsv4_flash", 8), ("gemma4_26b_a4b", 3),
+                                    ("tiny", 32)])
+def test_decode_and_gemm_paths_agree_at_crossover(name, T):
+    from gpu_util import check_y, oracle_rows, run_layer
+    L = layer(name)
+    x = inputs.make_tokens(L.cfg, T, seed=3)
+    y_dec, idx_dec, lg_dec = run_layer(L, x)
+    prev = F.ft_set_decode_max_tokens(0)      # force the tcgen05 grouped GEMM for tiny T
+    try:
+        y_gem, idx_gem, lg_gem = run_layer(L, x)
+    finally:
+        F.ft_set_decode_max_tokens(prev)
+    assert np.array_equal(idx_dec, idx_gem)
+    rows = np.arange(T, dtype=np.int32)
+    _, _, y64 = oracle_rows(L, x, lg_dec, rows)
+    check_y(y_dec, y64, L.cfg.wdtype, "decode path")
+    check_y(y_gem, y64, L.cfg.wdtype, "grouped GEMM path")
+
+
+def test_just_above_threshold_uses_gemm_and_matches():
+    L = layer("qwen3_a3b")
+    x = inputs.make_tokens(L.cfg, F.ft_get_decode_max_tokens() + 1, seed=4)
+    full_check(L, x, n_rows=33)
+
+
+@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_MXFP4])
+@pytest.mark.parametrize("S", [0, 1])
+@pytest.mark.parametrize("T", [3, 300])
+def test_small_custom_layers(wd, S, T):
+    L = layer("custom", hidden=256, ffn=128, num_experts=8, top_k=2, num_shared=S, wdtype=wd,
+              config_id=80 + 2 * wd + S)
+    x = inputs.make_tokens(L.cfg, T, seed=5)
+    full_check(L, x, n_rows=T)
+
+
+def test_all_experts_selected_k_equals_E():
+    L = layer("custom", hidden=128, ffn=64, num_experts=4, top_k=4, config_id=90)
+    x = inputs.make_tokens(L.cfg, 50, seed=6)
+    full_check(L, x, n_rows=50)
+
+
+@pytest.mark.parametrize("T", [700, 9])
+def test_skewed_routing_multi_tile_and_empty_groups(T):
+    """A bias sends every token to experts 3 and 5: two groups of T rows (several 256-row
+    tiles on the GEMM path), six empty groups."""
+    from gpu_util import DevLayer, ensure_built
+    ensure_built()
+    cfg = inputs.custom_config(hidden=256, ffn=128, num_experts=8, top_k=2, config_id=91)
+    d = inputs.make_layer(cfg, seed=7)
+    d["bias"] = np.zeros(8, np.float32)
+    d["bias"][[3, 5]] = 50.0
+    L = DevLayer(cfg, d)
+    x = inputs.make_tokens(cfg, T, seed=7)
+    y, idx, lg, _ = full_check(L, x, n_rows=24)
+    assert set(np.unique(idx)) == {3, 5}
+
+
+def test_deterministic_and_stepwise_equals_fused():
+    import torch
+    from gpu_util import dev, host, run_layer, workspace
+    L = layer("qwen3_a3b")
+    T = 4096
+    x = inputs.make_tokens(L.cfg, T, seed=8)
+    y1, i1, l1 = run_layer(L, x)
+    y2, i2, l2 = run_layer(L, x)
+    assert np.array_equal(y1, y2) and np.array_equal(i1, i2) and np.array_equal(l1, l2)
+    # step by step through the public entry points
+    cfg, s = L.cfg, L.shape
+    k, H, E, F_ = cfg.top_k, cfg.hidden, cfg.num_experts, cfg.ffn
+    R = T * k
+    ws = workspace(s, T)
+    xd = dev(x)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    sf = torch.empty(R, dtype=torch.int32, device="cuda")
+    inv = torch.empty(R, dtype=torch.int32, device="cuda")
+    xs = torch.empty((R, H), dtype=torch.int16, device="cuda")
+    h = torch.empty((R, F_), dtype=torch.int16, device="cuda")
+    o = torch.empty((R, H), dtype=torch.int16, device="cuda")
+    o2 = torch.empty((R, H), dtype=torch.int16, device="cuda")
+    y = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    F.ft_moe_route(s, T, xd, L.t["w_router"], L.t.get("bias"), idx, gw, None, ws)
+    F.ft_moe_permute(s, T, idx, xd, off, sf, inv, xs, ws)
+    F.ft_moe_experts(s, T, L.weights, xd, xs, off, sf, o, ws)
+    F.ft_moe_experts_gateup(s, T, L.weights, xs, off, h, ws)
+    F.ft_moe_experts_down(s, T, L.weights, h, off, o2, ws)
+    F.ft_moe_combine(s, T, o, inv, gw, y)
+    F.ft_moe_check(ws)
+    assert np.array_equal(host(idx, np.int32), i1)
+    assert np.array_equal(host(o, np.uint16), host(o2, np.uint16))
+    assert np.array_equal(host(y, np.uint16), y1)
+    # permutation outputs are the oracle's counting sort of the GPU ids, bit for bit
+    ooff, osf, oinv = oracle.permute(host(idx, np.int32), E)
+    assert np.array_equal(host(off, np.int32), ooff)
+    assert np.array_equal(host(sf, np.int32), osf)
+    assert np.array_equal(host(inv, np.int32), oinv)
+    assert np.array_equal(host(xs, np.uint16), x[osf // k])
+    # gates: oracle softmax over the GPU's kept logits (fp32 on the GPU vs fp64)
+    _, og = oracle.topk(l1, k)
+    assert np.max(np.abs(host(gw, np.float32) - og)) <= 2e-6
+
+
+def test_empty_batch_is_a_noop():
+    L = layer("tiny")
+    F.ft_moe_layer_forward(L.shape, 0, None, None, None, L.weights, None, None, None, None, 0)
