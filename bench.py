@@ -48,6 +48,27 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def recorded_traffic(summary: str, source: str):
+    """DRAM bytes (read + write) per launch from a committed ncu summary under profiles/,
+    or None when the summary is missing or the kernel source changed since the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", summary)
+    src = os.path.join(ROOT, "expert_offload_serving_router_b200", "csrc", source)
+    if not os.path.exists(p) or not os.path.exists(src):
+        return None
+    fields = {}
+    for line in open(p):
+        if ":" in line and line.strip().startswith(("dram_bytes_per_launch", "kernel_source_sha1")):
+            k_, v_ = line.split(":", 1)
+            fields[k_.strip()] = v_.strip().strip("`")
+    if fields.get("kernel_source_sha1") != hashlib.sha1(open(src, "rb").read()).hexdigest():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 # ------------------------------------------------------------------ clocks during the timed region
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -151,6 +172,40 @@ def run_reference(args, rank):
 
 
 # ------------------------------------------------------------------ GPU arm
+def measure_e2e(args, torch, dist, F, world, shape, weights, Wt, x, x_np, y, ws, ws_bytes, stream, T, H):
+    """Same metric through the public whole-layer call with pinned host buffers: every step
+    copies x host->device, runs ft_moe_layer_forward and copies y device->host."""
+    x_host = torch.from_numpy(x_np.view(np.int16)).pin_memory()
+    y_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
+    xe = torch.empty_like(x)
+
+    def e2e_step():
+        xe.copy_(x_host, non_blocking=True)
+        F.ft_moe_layer_forward(shape, T, xe, Wt["w_router"], Wt.get("bias"), weights, y, None, None, ws, ws_bytes,
+                               stream)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+           "d2h_bytes_per_step": T * H * 2, "ms_per_step": e2e_ms}
+
+    return e2e
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -159,6 +214,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-batch measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -271,40 +327,16 @@ def main():
     dn_flops = 2.0 * R * Fd * H
     gu_tflops = gu_flops / (stage_ms[2] * 1e-3) / 1e12
     dn_tflops = dn_flops / (stage_ms[3] * 1e-3) / 1e12
-    traffic = None
-    tf = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tf):
-        traffic = json.load(open(tf)).get("moe_gemm_gateup_qwen3_a3b_T4096")
+    traffic = recorded_traffic("moe_gemm_gateup_qwen3_a3b_T4096.md", "gemm_sm100.cu")
 
     # ---------------- end to end through the public call, host buffers
-    x_host = torch.from_numpy(x_np.view(np.int16)).pin_memory()
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(args, torch, dist, F, world, shape, weights, Wt, x, x_np, y, ws, ws_bytes, stream, T, H)
+
+    # ---------------- decode batches (rotating weight copies so L2 never holds the experts)
+    decode = None
     y_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
-    xe = torch.empty_like(x)
-
-    def e2e_step():
-        xe.copy_(x_host, non_blocking=True)
-        F.ft_moe_layer_forward(shape, T, xe, Wt["w_router"], Wt.get("bias"), weights, y, None, None, ws, ws_bytes,
-                               stream)
-        y_host.copy_(y, non_blocking=True)
-
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
-           "d2h_bytes_per_step": T * H * 2, "ms_per_step": e2e_ms}
-
     # ---------------- decode batches (rotating weight copies so L2 never holds the experts)
     decode = None
     if not args.no_decode:
