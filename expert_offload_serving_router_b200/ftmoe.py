@@ -59,6 +59,7 @@ _SIGS = {
     "ft_moe_check": (c_i32, [c_vp, c_vp]),
     "ft_moe_route": (c_i32, [ctypes.POINTER(ft_moe_shape), c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "ft_moe_permute": (c_i32, [ctypes.POINTER(ft_moe_shape), c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "ft_moe_permute_noalloc": (c_i32, [ctypes.POINTER(ft_moe_shape), c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "ft_moe_experts": (c_i32, [ctypes.POINTER(ft_moe_shape), c_i32, ctypes.POINTER(ft_moe_weights), c_vp, c_vp, c_vp,
                                c_vp, c_vp, c_vp, c_sz, c_vp]),
     "ft_moe_experts_gateup": (c_i32, [ctypes.POINTER(ft_moe_shape), c_i32, ctypes.POINTER(ft_moe_weights), c_vp, c_vp,
@@ -183,6 +184,12 @@ def ft_moe_route(shape, T, x, w_router, bias, topk_idx, topk_w, logits, ws, ws_b
 def ft_moe_permute(shape, T, topk_idx, x, offsets, sorted_flat, inv_pos, x_sorted, ws, ws_bytes=None, stream=None):
     _check(lib().ft_moe_permute(ctypes.byref(shape), T, _p(topk_idx), _p(x), _p(offsets), _p(sorted_flat),
                                 _p(inv_pos), _p(x_sorted), _p(ws), _nbytes(ws, ws_bytes), _s(stream)))
+
+
+def ft_moe_permute_noalloc(shape, T, topk_idx, x, offsets, sorted_flat, inv_pos, x_sorted, stream=None):
+    """Permutation without a workspace (static device scratch); for callers that cannot allocate."""
+    _check(lib().ft_moe_permute_noalloc(ctypes.byref(shape), T, _p(topk_idx), _p(x), _p(offsets), _p(sorted_flat),
+                                        _p(inv_pos), _p(x_sorted), _s(stream)))
 
 
 def ft_moe_experts(shape, T, weights, x, x_sorted, offsets, sorted_flat, o_sorted, ws, ws_bytes=None, stream=None):

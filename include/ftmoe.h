@@ -155,6 +155,26 @@ ft_status ft_moe_permute(const ft_moe_shape* shape, int32_t T, const int32_t* to
                          int32_t* offsets, int32_t* sorted_flat, int32_t* inv_pos, void* x_sorted,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* Step 2 for callers that cannot allocate device memory (the source pages have
+ * no counterpart to this entry point).  Same arithmetic, outputs and layouts
+ * as ft_moe_permute, but no workspace argument: the scratch lives in one
+ * static device array of the library (about 390 KB, held by every GPU that
+ * loads the library until the process exits).  For callers that may not call
+ * cudaMalloc: engines that reserve nearly all HBM for their own pools at
+ * start-up, plugins handed only their input/output buffers by a framework
+ * that owns the allocator, fixed-budget code that must not grow.
+ * Limit: R = T*k + S*T <= 65536 rows, else FT_ERR_UNSUPPORTED before any
+ * launch.  The first call on each device looks the array's device address up
+ * (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ * capture.  Every call shares the array and it keeps the last call's contents:
+ * calls that overlap on the GPU race.  No allocation of any kind.  An id
+ * outside [0,E) drops its pair (offsets[E+S] < R shows it).  The tile schedule
+ * that ft_moe_permute leaves in its ws for ft_moe_experts is not produced for
+ * the caller here. */
+ft_status ft_moe_permute_noalloc(const ft_moe_shape* shape, int32_t T, const int32_t* topk_idx, const void* x,
+                                 int32_t* offsets, int32_t* sorted_flat, int32_t* inv_pos, void* x_sorted,
+                                 void* stream);
+
 /* Step 3 -- experts.  Computes o_sorted[r] = FFN_{group(r)}(x row of r) for
  * every permuted row r.  x: device [T,H]; x_sorted: device [R,H] as written
  * by ft_moe_permute (required when T > decode threshold, else may be NULL);
