@@ -42,7 +42,17 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-__device__ __forceinline__ float silu_mul(float a, float b) { return a / (1.0f + __expf(-a)) * b; }
+// silu(a) * b, silu(a) = a * sigmoid(a) = h + h * tanh(h) with h = a/2 (tanh.approx: one MUFU op,
+// relative error ~2^-11, below the bf16 rounding of the result)
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float silu_mul(float a, float b) {
+    const float h = 0.5f * a;
+    return fmaf(h, tanh_approx(h), h) * b;
+}
 
 // ------------------------------------------------------------------ workspace layout
 // One layout serves every entry point: a region is only touched by the steps that need it.

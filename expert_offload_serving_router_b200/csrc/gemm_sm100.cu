@@ -5,9 +5,11 @@
 //   down:     D[128 hidden rows, N tokens] = W2_e[rows, F] . h[tokens, F]^T,
 //             o_sorted[token, hrow] stored bf16 [R, H]
 //
-// "Weights as A": the MMA M dimension (128) walks weight rows and N walks the tokens of
-// one expert group, so an expert with few tokens costs an MMA of N = round_up(n, 16)
-// instead of a padded 128-row tile.  The gate/up A tile interleaves gate and up rows in
+// "Weights as A": the MMA M dimension walks weight rows and N walks the tokens of one
+// expert group, so an expert with few tokens costs an MMA of N = round_up(n, 16) instead
+// of a padded 128-row tile, and its activation box shrinks to the next power of two.
+// A CTA tile is 256 weight rows (two M=128 MMAs into two TMEM accumulators) x N tokens,
+// so each activation stage feeds twice the math of a single 128-row MMA.  The gate/up A tile interleaves gate and up rows in
 // blocks of 16 (rows 32i..32i+15 = gate f0+16i.., rows 32i+16..32i+31 = up f0+16i..), so
 // each TMEM lane quarter holds gate and up of the same 16 f values: lane l and l^16
 // exchange halves with one shuffle, no shared-memory round trip.
@@ -15,11 +17,11 @@
 // Warp roles (one CTA per SM, persistent over a device-side tile list):
 //   warp 0      TMA producer (weights for BF16; activations always)
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2-5   epilogue (tcgen05.ld 32x32b, SwiGLU / bf16 stores)
-//   warps 6-9   MXFP4 only: load E2M1 codes + E8M0 scales with 128-bit loads, dequantise
-//               exactly to bf16 in registers and write the SW128 A tile to shared memory
-// Operands are K-major, 128-byte swizzled; accumulators fp32 in TMEM, double buffered
-// (2 x 256 columns) so the epilogue of tile i overlaps the MMAs of tile i+1.
+//   warps 2-9   BF16: epilogue, two warps per TMEM lane quarter (tcgen05.ld 32x32b)
+//   warps 2-5   MXFP4: epilogue;  warps 6-9: load E2M1 codes + E8M0 scales with 128-bit
+//               loads, dequantise exactly to bf16 and write the SW128 A tile to smem
+// Operands are K-major, 128-byte swizzled, 3-stage ring of 64 KB stages; the two fp32
+// accumulators take all 512 TMEM columns.
 // Every wait is bounded: on timeout the kernel records kDevErrTimeout, drains its own
 // copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -27,17 +29,21 @@
 
 namespace ftmoe {
 
-constexpr int kStages = 4;
-constexpr int kBK = 64;                       // K per stage (one 128-byte swizzle atom of bf16)
-constexpr int kATileBytes = 128 * kBK * 2;    // 16 KB
-constexpr int kBTileBytes = kGemmBN * kBK * 2;// 32 KB
-constexpr int kAccCols = 256;
+constexpr int kStages = 3;
+constexpr int kBK = 64;                        // K per stage (one 128-byte swizzle atom of bf16)
+constexpr int kAHalfBytes = 128 * kBK * 2;     // 16 KB: one 128-row MMA operand
+constexpr int kATileBytes = 2 * kAHalfBytes;   // 32 KB: 256 weight rows per tile
+constexpr int kBTileBytes = kGemmBN * kBK * 2; // 32 KB: up to 256 token rows
+constexpr int kAccCols = 256;                  // one accumulator = 128 lanes x 256 fp32 columns
+constexpr int kNumBMaps = 5;                   // activation boxes of 16, 32, 64, 128, 256 rows
+constexpr int kXposeBytes = 2048;              // per epilogue warp: 32 tokens x 32 bf16
 constexpr unsigned long long kWaitNs = 4000000000ull;  // 4 s bound on any wait
 
 struct GemmParams {
     int mode;               // 0 gate/up, 1 down
     int K;                  // H or F
-    int m_tiles;            // F/64 (gate/up) or H/128 (down)
+    int m_tiles;            // ceil(F/128) (gate/up) or ceil(H/256) (down): 256 weight rows per tile
+    int m_rows;             // valid weight-row groups: F/64 (gate/up) or H/128 (down) 128-row halves
     int G, E, F, H;
     int has_shared;
     const int32_t* offsets; // [G+1]
@@ -45,7 +51,7 @@ struct GemmParams {
     uint16_t* out;          // h [R,F] or o_sorted [R,H]
     int out_ld;
     uint32_t* err;
-    int b_bytes;            // bytes of one activation box (rows x 128 B); rows = min(256, round_up(R, 16))
+    int b_rows[kNumBMaps];  // rows of activation box i (16 << i, clamped to round_up(R, 16))
     // MXFP4 weights (A operand built by converter warps)
     const uint8_t* wq;      // routed codes  [E, rows, K/2]
     const uint8_t* ws;      // routed scales [E, rows, K/32]
@@ -131,19 +137,34 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
                  : "memory");
 }
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
+// 32 consecutive TMEM columns of this thread's lane -> v (valid only after tmem_wait_ld)
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float (&v)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
         "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+          "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15]),
+          "=f"(v[16]), "=f"(v[17]), "=f"(v[18]), "=f"(v[19]), "=f"(v[20]), "=f"(v[21]), "=f"(v[22]), "=f"(v[23]),
+          "=f"(v[24]), "=f"(v[25]), "=f"(v[26]), "=f"(v[27]), "=f"(v[28]), "=f"(v[29]), "=f"(v[30]), "=f"(v[31])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// Wait for outstanding TMEM loads; the registers are in/out operands so no use of them can
+// be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_16(float* v) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                   "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15])
+                 :: "memory");
+}
+__device__ __forceinline__ void tmem_fence_regs(float* v) {   // no-op that pins 16 registers after the wait
+    asm volatile("" : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                 "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]));
+}
+__device__ __forceinline__ void tmem_wait_ld(float (&a)[32], float (&b)[32]) {
+    tmem_wait_16(a);
+    tmem_fence_regs(a + 16);
+    tmem_fence_regs(b);
+    tmem_fence_regs(b + 16);
 }
 
 // ------------------------------------------------------------------ exact MXFP4 -> bf16
@@ -179,9 +200,10 @@ __device__ __forceinline__ uint32_t e8m0_bf16x2(uint32_t s) {
 }
 
 // ------------------------------------------------------------------ tile schedule
-struct Tile { int g, m, row0, nvalid; };
+struct Tile { int g, m, row0, nvalid, halves; };
 
-__device__ __forceinline__ Tile decode_tile(int t, const int* ntile_off, int G, const int32_t* offsets, int m_tiles) {
+__device__ __forceinline__ Tile decode_tile(int t, const int* ntile_off, int G, const int* offsets, int m_tiles,
+                                            int m_rows) {
     Tile r;
     int u = t / m_tiles;
     r.m = t - u * m_tiles;
@@ -194,38 +216,51 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* ntile_off, int G, 
     int ni = u - ntile_off[lo];
     r.row0 = offsets[lo] + ni * kGemmBN;
     r.nvalid = min(kGemmBN, offsets[lo + 1] - r.row0);
+    r.halves = min(2, m_rows - 2 * r.m);   // the last weight-row tile may hold one 128-row half
     return r;
 }
 
+__device__ __forceinline__ int bmap_index(int n) {   // smallest box of 16 << i rows holding n rows
+    int i = 0;
+    while (i < kNumBMaps - 1 && (16 << i) < n) ++i;
+    return i;
+}
+
 template <bool MX>
-__global__ void __launch_bounds__(MX ? 320 : 192, 1)
+__global__ void __launch_bounds__(320, 1)
 moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sw,
-                const __grid_constant__ CUtensorMap tm_act, GemmParams p) {
+                const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
+                const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_b3,
+                const __grid_constant__ CUtensorMap tm_b4, GemmParams p) {
+    constexpr int kEpiWarps = MX ? 4 : 8;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStages * kATileBytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kBTileBytes);
+    uint8_t* sX = sB + kStages * kBTileBytes;              // epilogue transpose buffers, 2 KB per warp
+    uint64_t* full = reinterpret_cast<uint64_t*>(sX + 8 * kXposeBytes);
     uint64_t* empty = full + kStages;
     uint64_t* tfull = empty + kStages;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* mma_done = tempty + 2;
+    uint64_t* tempty = tfull + 1;
+    uint64_t* mma_done = tempty + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* ntile_off = const_cast<int*>(reinterpret_cast<volatile int*>(tmem_slot + 2));
+    int* s_off = ntile_off + 260;                           // group row offsets [G+1]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = p.G;
-    for (int i = tid; i <= G; i += blockDim.x) ntile_off[i] = p.sched[2 + i];
+    for (int i = tid; i <= G; i += blockDim.x) {
+        ntile_off[i] = p.sched[2 + i];
+        s_off[i] = p.offsets[i];
+    }
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], MX ? 1 + 4 : 1);
             mbar_init(&empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 4);
-        }
+        mbar_init(tfull, 1);
+        mbar_init(tempty, kEpiWarps);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -246,6 +281,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
+            const CUtensorMap* bm[kNumBMaps] = {&tm_b0, &tm_b1, &tm_b2, &tm_b3, &tm_b4};
             int stage = 0;
             uint32_t phase = 0;
             int issued[kStages];
@@ -253,29 +289,32 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
             for (int s = 0; s < kStages; ++s) issued[s] = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                Tile tl = decode_tile(t, ntile_off, G, p.offsets, p.m_tiles);
+                const Tile tl = decode_tile(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
                 const bool shared_grp = p.has_shared && tl.g == p.E;
+                const int bi = bmap_index(tl.nvalid);
+                const uint32_t bbytes = uint32_t(p.b_rows[bi]) * kBK * 2;
+                const uint32_t abytes = MX ? 0u : uint32_t(tl.halves) * kAHalfBytes;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* a = sA + stage * kATileBytes;
                     uint8_t* b = sB + stage * kBTileBytes;
                     const int k0 = kb * kBK;
+                    mbar_expect_tx(&full[stage], abytes + bbytes);
                     if (!MX) {
-                        mbar_expect_tx(&full[stage], kATileBytes + p.b_bytes);
-                        if (p.mode == 0) {
-                            const CUtensorMap* m = shared_grp ? &tm_sw : &tm_w;
-                            const int e = shared_grp ? 0 : tl.g;
+                        const CUtensorMap* m = shared_grp ? &tm_sw : &tm_w;
+                        const int e = shared_grp ? 0 : tl.g;
+                        for (int h = 0; h < tl.halves; ++h) {
+                            if (p.mode == 0) {
 #pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                tma_4d(m, &full[stage], a + i * 4096, k0, tl.m * 64 + 16 * i, 0, e);
-                        } else {
-                            const CUtensorMap* m = shared_grp ? &tm_sw : &tm_w;
-                            tma_3d(m, &full[stage], a, k0, tl.m * 128, shared_grp ? 0 : tl.g);
+                                for (int i = 0; i < 4; ++i)
+                                    tma_4d(m, &full[stage], a + h * kAHalfBytes + i * 4096, k0,
+                                           tl.m * 128 + h * 64 + 16 * i, 0, e);
+                            } else {
+                                tma_3d(m, &full[stage], a + h * kAHalfBytes, k0, tl.m * 256 + h * 128, e);
+                            }
                         }
-                    } else {
-                        mbar_expect_tx(&full[stage], p.b_bytes);
                     }
-                    tma_2d(&tm_act, &full[stage], b, k0, tl.row0);
+                    tma_2d(bm[bi], &full[stage], b, k0, tl.row0);
                     issued[stage] = 1;
                     issued_par[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
@@ -290,128 +329,177 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             int stage = 0;
-            uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
+            uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                Tile tl = decode_tile(t, ntile_off, G, p.offsets, p.m_tiles);
+                const Tile tl = decode_tile(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
                 const int N = (tl.nvalid + 15) & ~15;
                 const uint32_t idesc = idesc_bf16(128, N);
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(tempty, acc_phase ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t dtm = tmem_base + uint32_t(acc * kAccCols);
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t ad = sdesc_sw128(su32(sA + stage * kATileBytes));
                     const uint64_t bd = sdesc_sw128(su32(sB + stage * kBTileBytes));
+                    for (int h = 0; h < tl.halves; ++h) {
+                        const uint64_t ad = sdesc_sw128(su32(sA + stage * kATileBytes + h * kAHalfBytes));
+                        const uint32_t dtm = tmem_base + uint32_t(h * kAccCols);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        umma_bf16(dtm, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            umma_bf16(dtm, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+                    }
                     umma_commit(&empty[stage]);
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                umma_commit(&tfull[acc]);
-                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+                umma_commit(tfull);
+                acc_phase ^= 1;
             }
             if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
             umma_commit(mma_done);               // tracks completion of every MMA issued above
             mbar_wait(mma_done, 0, nullptr);
         }
-    } else if (warp < 6) {
-        // ------------------------------------------------ epilogue (TMEM -> registers -> global)
+    } else if (warp < 2 + kEpiWarps) {
+        // ------------------------------------------------ epilogue (TMEM -> registers -> smem -> global)
+        // Two 32-column chunks are loaded per tcgen05.wait; each chunk is transposed through a
+        // per-warp shared buffer so the global stores are 16-byte vectors along the token row.
         const int q = warp & 3;                  // TMEM lanes 32q .. 32q+31
-        int acc = 0;
+        const int part = (warp - 2) >> 2;        // which column chunks this warp takes
+        constexpr int kParts = kEpiWarps / 4;
+        uint16_t* xb = reinterpret_cast<uint16_t*>(sX + (warp - 2) * kXposeBytes);
         uint32_t acc_phase = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            Tile tl = decode_tile(t, ntile_off, G, p.offsets, p.m_tiles);
-            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) { ok = false; break; }
+            const Tile tl = decode_tile(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+            if (!mbar_wait(tfull, acc_phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols);
             const int nch = (tl.nvalid + 31) >> 5;
-            for (int c = 0; c < nch; ++c) {
-                float v[32];
-                tmem_ld32(tbase + uint32_t(c * 32), v);
-                if (p.mode == 0) {
-                    const int f = tl.m * 64 + 16 * q + (lane & 15);
-                    const bool lo = lane < 16;
+            const int per_half = (nch - part + kParts - 1) / kParts;   // chunks c = part, part + kParts, ...
+            const int items = tl.halves * per_half;
+            for (int it = 0; it < items; it += 2) {
+                float v[2][32];
+                int hh[2], cc[2];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float send = lo ? v[16 + i] : v[i];
-                        float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-                        float gt = lo ? v[i] : recv;
-                        float up = lo ? recv : v[16 + i];
-                        int n = c * 32 + (lo ? i : 16 + i);
-                        if (n < tl.nvalid)
-                            p.out[size_t(tl.row0 + n) * p.out_ld + f] = f2bf(silu_mul(gt, up));
-                    }
-                } else {
-                    const int hrow = tl.m * 128 + 32 * q + lane;
+                for (int u = 0; u < 2; ++u) {
+                    const int iu = it + u < items ? it + u : it;
+                    hh[u] = iu / per_half;
+                    cc[u] = part + kParts * (iu - hh[u] * per_half);
+                    tmem_ld32_nowait(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(hh[u] * kAccCols + cc[u] * 32), v[u]);
+                }
+                tmem_wait_ld(v[0], v[1]);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        int n = c * 32 + j;
-                        if (n < tl.nvalid) p.out[size_t(tl.row0 + n) * p.out_ld + hrow] = f2bf(v[j]);
+                for (int u = 0; u < 2; ++u) {
+                    if (it + u >= items) break;
+                    const int c = cc[u], h = hh[u];
+                    if (p.mode == 0) {
+                        const int fl = lane & 15;
+                        const bool lo = lane < 16;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float send = lo ? v[u][16 + i] : v[u][i];
+                            const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+                            const float gt = lo ? v[u][i] : recv;
+                            const float up = lo ? recv : v[u][16 + i];
+                            xb[(lo ? i : 16 + i) * 16 + fl] = f2bf(silu_mul(gt, up));
+                        }
+                        __syncwarp();
+                        const int fbase = tl.m * 128 + h * 64 + 16 * q;
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            const int ch = lane + 32 * r, tok = ch >> 1, pp = ch & 1;
+                            const int n = c * 32 + tok;
+                            if (n < tl.nvalid)
+                                *reinterpret_cast<uint4*>(p.out + size_t(tl.row0 + n) * p.out_ld + fbase + 8 * pp) =
+                                    *reinterpret_cast<const uint4*>(xb + tok * 16 + 8 * pp);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) xb[j * 32 + lane] = f2bf(v[u][j]);
+                        __syncwarp();
+                        const int hbase = tl.m * 256 + h * 128 + 32 * q;
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const int ch = lane + 32 * r, tok = ch >> 2, pp = ch & 3;
+                            const int n = c * 32 + tok;
+                            if (n < tl.nvalid)
+                                *reinterpret_cast<uint4*>(p.out + size_t(tl.row0 + n) * p.out_ld + hbase + 8 * pp) =
+                                    *reinterpret_cast<const uint4*>(xb + tok * 32 + 8 * pp);
+                        }
                     }
+                    __syncwarp();
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
-            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            if (lane == 0) mbar_arrive(tempty);
+            acc_phase ^= 1;
         }
         if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
     } else if (MX) {
-        // ------------------------------------------------ MXFP4 converter warps (one A row per thread)
-        const int r = tid - 192;                 // 0..127
+        // ------------------------------------------------ MXFP4 converter warps (two A rows per thread)
+        const int r0 = tid - 64 - 32 * kEpiWarps;   // 0..127: rows r0 (half 0) and r0 (half 1)
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         const int kq = p.K / 2, ks = p.K / 32;   // code / scale bytes per weight row
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            Tile tl = decode_tile(t, ntile_off, G, p.offsets, p.m_tiles);
+            const Tile tl = decode_tile(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
             const bool shared_grp = p.has_shared && tl.g == p.E;
-            int wrow;
-            size_t rows_per_expert;
-            if (p.mode == 0) {
-                const int i = r >> 5, j = r & 31;
-                const int f = tl.m * 64 + 16 * i + (j & 15);
-                wrow = j < 16 ? f : p.F + f;
-                rows_per_expert = size_t(2) * p.F;
-            } else {
-                wrow = tl.m * 128 + r;
-                rows_per_expert = size_t(p.H);
-            }
             const size_t e = shared_grp ? 0 : size_t(tl.g);
-            const uint8_t* qrow = (shared_grp ? p.swq : p.wq) + (e * rows_per_expert + wrow) * kq;
-            const uint8_t* srow = (shared_grp ? p.sws : p.ws) + (e * rows_per_expert + wrow) * ks;
-            uint4 c0 = ldg_nc_v4(qrow), c1 = ldg_nc_v4(qrow + 16);
-            uint32_t sc = *reinterpret_cast<const uint16_t*>(srow);
+            const uint8_t* qrow[2];
+            const uint8_t* srow[2];
+            for (int h = 0; h < 2; ++h) {
+                const int hh = h < tl.halves ? h : 0;     // a missing half re-reads half 0 (unused)
+                int wrow;
+                size_t rows_per_expert;
+                if (p.mode == 0) {
+                    const int i = r0 >> 5, j = r0 & 31;
+                    const int f = tl.m * 128 + hh * 64 + 16 * i + (j & 15);
+                    wrow = j < 16 ? f : p.F + f;
+                    rows_per_expert = size_t(2) * p.F;
+                } else {
+                    wrow = tl.m * 256 + hh * 128 + r0;
+                    rows_per_expert = size_t(p.H);
+                }
+                qrow[h] = (shared_grp ? p.swq : p.wq) + (e * rows_per_expert + wrow) * kq;
+                srow[h] = (shared_grp ? p.sws : p.ws) + (e * rows_per_expert + wrow) * ks;
+            }
+            uint4 c[2][2];
+            uint32_t sc[2];
+            for (int h = 0; h < 2; ++h) {
+                c[h][0] = ldg_nc_v4(qrow[h]);
+                c[h][1] = ldg_nc_v4(qrow[h] + 16);
+                sc[h] = *reinterpret_cast<const uint16_t*>(srow[h]);
+            }
             for (int kb = 0; kb < nk; ++kb) {
-                uint4 n0 = c0, n1 = c1;
-                uint32_t nsc = sc;
-                if (kb + 1 < nk) {
-                    n0 = ldg_nc_v4(qrow + (kb + 1) * 32);
-                    n1 = ldg_nc_v4(qrow + (kb + 1) * 32 + 16);
-                    nsc = *reinterpret_cast<const uint16_t*>(srow + (kb + 1) * 2);
+                uint4 nx[2][2];
+                uint32_t nsc[2];
+                for (int h = 0; h < 2; ++h) {
+                    nx[h][0] = c[h][0]; nx[h][1] = c[h][1]; nsc[h] = sc[h];
+                    if (kb + 1 < nk) {
+                        nx[h][0] = ldg_nc_v4(qrow[h] + (kb + 1) * 32);
+                        nx[h][1] = ldg_nc_v4(qrow[h] + (kb + 1) * 32 + 16);
+                        nsc[h] = *reinterpret_cast<const uint16_t*>(srow[h] + (kb + 1) * 2);
+                    }
                 }
                 if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-                uint8_t* arow = sA + stage * kATileBytes + r * 128;
-                const uint32_t s0 = e8m0_bf16x2(sc & 0xFF), s1 = e8m0_bf16x2(sc >> 8);
-                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                for (int h = 0; h < tl.halves; ++h) {
+                    uint8_t* arow = sA + stage * kATileBytes + h * kAHalfBytes + r0 * 128;
+                    const uint32_t s0 = e8m0_bf16x2(sc[h] & 0xFF), s1 = e8m0_bf16x2(sc[h] >> 8);
+                    const uint32_t words[8] = {c[h][0].x, c[h][0].y, c[h][0].z, c[h][0].w,
+                                               c[h][1].x, c[h][1].y, c[h][1].z, c[h][1].w};
 #pragma unroll
-                for (int cch = 0; cch < 8; ++cch) {      // 16-byte chunk cch = elements 8cch..8cch+7
-                    uint32_t o[4];
-                    e2m1x8_bf16(words[cch], cch < 4 ? s0 : s1, o);
-                    *reinterpret_cast<uint4*>(arow + ((cch ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    for (int cch = 0; cch < 8; ++cch) {  // 16-byte chunk cch = elements 8cch..8cch+7
+                        uint32_t o[4];
+                        e2m1x8_bf16(words[cch], cch < 4 ? s0 : s1, o);
+                        *reinterpret_cast<uint4*>(arow + ((cch ^ (r0 & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[stage]);
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
-                c0 = n0; c1 = n1; sc = nsc;
+                for (int h = 0; h < 2; ++h) { c[h][0] = nx[h][0]; c[h][1] = nx[h][1]; sc[h] = nsc[h]; }
             }
         }
         if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
@@ -467,15 +555,22 @@ static int num_sms() {
     return n;
 }
 
-static size_t gemm_smem_bytes() { return 1024 + kStages * (kATileBytes + kBTileBytes) + 256 + 4 * 260; }
-
-
+static size_t gemm_smem_bytes() { return 1024 + kStages * (kATileBytes + kBTileBytes) + 8 * kXposeBytes + 256 + 8 * 260; }
 
 // returns 0 ok, 1 tensor-map failure, 2 launch failure
 int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
     const bool mx = L.wdtype == FT_W_MXFP4;
     const int K = L.mode == 0 ? L.H : L.F;
-    CUtensorMap tw{}, tsw{}, tact{};
+    CUtensorMap tw{}, tsw{}, tb[kNumBMaps]{};
+    GemmParams p{};
+    const int rR = (L.R + 15) & ~15;
+    for (int i = 0; i < kNumBMaps; ++i) {
+        p.b_rows[i] = (16 << i) < rR ? (16 << i) : rR;
+        uint64_t dims[2] = {uint64_t(K), uint64_t(L.R)};
+        uint64_t str[1] = {uint64_t(K) * 2};
+        uint32_t box[2] = {kBK, uint32_t(p.b_rows[i])};
+        if (!make_map(&tb[i], L.act, 2, dims, str, box)) return 1;
+    }
     if (!mx) {
         if (L.mode == 0) {
             uint64_t dims[4] = {uint64_t(L.H), uint64_t(L.F), 2, uint64_t(L.E)};
@@ -500,19 +595,14 @@ int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
                 tsw = tw;
             }
         }
+    } else {
+        tw = tb[0];   // unused by the MXFP4 kernel (A comes from the converter warps)
+        tsw = tb[0];
     }
-    const int box_rows = L.R >= kGemmBN ? kGemmBN : ((L.R + 15) & ~15);
-    {
-        uint64_t dims[2] = {uint64_t(K), uint64_t(L.R)};
-        uint64_t str[1] = {uint64_t(K) * 2};
-        uint32_t box[2] = {kBK, uint32_t(box_rows)};
-        if (!make_map(&tact, L.act, 2, dims, str, box)) return 1;
-    }
-    if (mx) { tw = tact; tsw = tact; }   // unused by the MXFP4 kernel
-    GemmParams p{};
     p.mode = L.mode;
     p.K = K;
-    p.m_tiles = L.mode == 0 ? L.F / 64 : L.H / 128;
+    p.m_rows = L.mode == 0 ? L.F / 64 : L.H / 128;
+    p.m_tiles = (p.m_rows + 1) / 2;
     p.G = L.E + (L.S ? 1 : 0);
     p.E = L.E;
     p.F = L.F;
@@ -523,14 +613,13 @@ int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
     p.out = L.out;
     p.out_ld = L.mode == 0 ? L.F : L.H;
     p.err = L.err;
-    p.b_bytes = box_rows * kBK * 2;
     p.wq = static_cast<const uint8_t*>(L.w);
     p.ws = L.wscale;
     p.swq = static_cast<const uint8_t*>(L.sw);
     p.sws = L.swscale;
     const size_t smem = gemm_smem_bytes();
     int grid = num_sms();
-    int max_tiles = L.max_tiles * p.m_tiles;
+    const int max_tiles = L.max_tiles * p.m_tiles;
     if (max_tiles < grid) grid = max_tiles > 0 ? max_tiles : 1;
     if (mx) {
         static bool set = false;
@@ -538,14 +627,14 @@ int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
             if (cudaFuncSetAttribute(moe_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 2;
             set = true;
         }
-        moe_gemm_kernel<true><<<grid, 320, smem, st>>>(tw, tsw, tact, p);
+        moe_gemm_kernel<true><<<grid, 320, smem, st>>>(tw, tsw, tb[0], tb[1], tb[2], tb[3], tb[4], p);
     } else {
         static bool set = false;
         if (!set) {
             if (cudaFuncSetAttribute(moe_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 2;
             set = true;
         }
-        moe_gemm_kernel<false><<<grid, 192, smem, st>>>(tw, tsw, tact, p);
+        moe_gemm_kernel<false><<<grid, 320, smem, st>>>(tw, tsw, tb[0], tb[1], tb[2], tb[3], tb[4], p);
     }
     return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }

@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(PermArgs a, int C) {
     const int g = threadIdx.x;
     if (g < G) {
         int r = 0;
+#pragma unroll 8
         for (int c = 0; c < C; ++c) {
             int v = a.chunk_cnt[size_t(c) * G + g];
             a.chunk_base[size_t(c) * G + g] = r;
@@ -103,36 +104,48 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(PermArgs a, int C) {
     if (g == 0) a.out.offsets[G] = total;
 }
 
+// One CTA per 128 pairs (8 warps x 16): scatter the permutation, then gather the x rows.
+constexpr int kScatterItems = 128;
+
 __global__ void __launch_bounds__(256) perm_scatter_kernel(PermArgs a) {
-    __shared__ int spos[kPermChunk];
-    __shared__ int stok[kPermChunk];
+    __shared__ int spos[kScatterItems];
+    __shared__ int stok[kScatterItems];
     const int P = a.T * a.k, R = P + (a.S ? a.T : 0), G = a.E + (a.S ? 1 : 0);
-    const int c = blockIdx.x, tid = threadIdx.x;
-    const int i0 = c * kPermChunk;
-    const int n = min(kPermChunk, R - i0);
-    for (int q = tid; q < n; q += 256) {
-        int i = i0 + q;
-        int g = pair_group(a, i, P);
+    const int tid = threadIdx.x;
+    const int i0 = blockIdx.x * kScatterItems;
+    const int n = min(kScatterItems, R - i0);
+    if (tid < n) {
+        const int i = i0 + tid;
+        const int c = i / kPermChunk;
+        const int g = pair_group(a, i, P);
         int pos = -1;
         if (g >= 0) {
             pos = a.chunk_base[size_t(c) * G + g] + a.local_rank[i];
             a.out.sorted_flat[pos] = i;
             a.out.inv_pos[i] = pos;
         }
-        spos[q] = pos;
-        stok[q] = i < P ? i / a.k : i - P;
+        spos[tid] = pos;
+        stok[tid] = i < P ? i / a.k : i - P;
     }
     if (!a.x_sorted) return;
     __syncthreads();
-    // gather: one warp per row, 16-byte vectors
+    // gather: one warp per row, 16-byte vectors, 4 vectors in flight per lane
     const int lane = tid & 31, warp = tid >> 5;
     const int nv = a.H / 8;
     for (int q = warp; q < n; q += 8) {
-        int pos = spos[q];
+        const int pos = spos[q];
         if (pos < 0) continue;
         const uint4* src = reinterpret_cast<const uint4*>(a.x + size_t(stok[q]) * a.H);
         uint4* dst = reinterpret_cast<uint4*>(a.x_sorted + size_t(pos) * a.H);
-        for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+        for (int v0 = lane; v0 < nv; v0 += 128) {
+            uint4 u[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (v0 + 32 * j < nv) u[j] = __ldg(src + v0 + 32 * j);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (v0 + 32 * j < nv) dst[v0 + 32 * j] = u[j];
+        }
     }
 }
 
@@ -173,7 +186,7 @@ cudaError_t launch_permute(int T, int k, int E, int S, int H, const int32_t* idx
     PermArgs a{T, k, E, S, H, idx, x, x_sorted, chunk_cnt, chunk_base, local_rank, out};
     perm_count_kernel<<<C, 256, 0, st>>>(a);
     perm_scan_kernel<<<1, 1024, 0, st>>>(a, C);
-    perm_scatter_kernel<<<C, 256, 0, st>>>(a);
+    perm_scatter_kernel<<<(R + kScatterItems - 1) / kScatterItems, 256, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -67,83 +67,98 @@ __device__ inline void warp_topk_row(const float* row, int E, int k, int32_t* id
 }
 
 // ------------------------------------------------------------------ T > 32
-constexpr int kRtTok = 32;    // tokens per CTA
-constexpr int kRtBK = 32;     // K slice staged per iteration
-constexpr int kRtLd = kRtBK + 4;
+constexpr int kRtTok = 32;          // tokens per CTA (8 per warp)
+constexpr int kRtBK = 32;           // K slice staged per pipeline stage
+constexpr int kRtLdW = kRtBK + 4;   // floats per staged router row (conflict-free float4 reads)
+constexpr int kRtLdX = kRtBK + 8;   // bf16 per staged token row
 
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(uint32_t(__cvta_generic_to_shared(smem))),
+                 "l"(gmem), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// NE = experts per lane (E <= 32*NE).  Each thread owns 8 tokens x NE experts of the logit
+// tile; K slices of the router rows and token rows are double buffered with cp.async.
+template <int NE>
 __global__ void __launch_bounds__(128)
 route_tile_kernel(int T, int H, int E, int k, const uint16_t* __restrict__ x, const float* __restrict__ wr,
                   const float* __restrict__ bias, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                   float* __restrict__ logits) {
     extern __shared__ float4 smem4[];
-    float* ws = reinterpret_cast<float*>(smem4);            // [256][kRtLd]  (reused as logit tile)
-    float* xs = ws + kMaxExperts * kRtLd;                   // [32][kRtLd]
+    constexpr int kRows = 32 * NE;
+    float* wbuf = reinterpret_cast<float*>(smem4);                                  // [2][kRows][kRtLdW]
+    uint16_t* xbuf = reinterpret_cast<uint16_t*>(wbuf + 2 * kRows * kRtLdW);        // [2][32][kRtLdX]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.x * kRtTok;
-    float acc[8][8];
+    const int nk = H / kRtBK;
+
+    auto stage = [&](int s, int k0) {
+        float* wd = wbuf + s * kRows * kRtLdW;
+        for (int f = tid; f < E * 8; f += 128) {
+            const int e = f >> 3, q = f & 7;
+            cp_async16(wd + e * kRtLdW + q * 4, wr + size_t(e) * H + k0 + q * 4, 16);
+        }
+        const int t = tid >> 2, q = tid & 3;
+        const bool ok = t0 + t < T;
+        cp_async16(xbuf + (s * kRtTok + t) * kRtLdX + q * 8, x + size_t(ok ? t0 + t : 0) * H + k0 + q * 8, ok ? 16 : 0);
+        cp_async_commit();
+    };
+
+    float acc[8][NE];
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+        for (int b = 0; b < NE; ++b) acc[a][b] = 0.f;
 
-    for (int k0 = 0; k0 < H; k0 += kRtBK) {
-        // W slice: E rows x 32 floats, 8 float4 per row, 8 consecutive threads per row
-        for (int f = tid; f < E * 8; f += 128) {
-            int e = f >> 3, q = f & 7;
-            float4 w4 = *reinterpret_cast<const float4*>(wr + size_t(e) * H + k0 + q * 4);
-            *reinterpret_cast<float4*>(ws + e * kRtLd + q * 4) = w4;
-        }
-        // x slice: 32 tokens x 32 bf16 (4 x 16 B per token)
-        {
-            int t = tid >> 2, q = tid & 3;
-            uint4 u = make_uint4(0, 0, 0, 0);
-            if (t0 + t < T) u = *reinterpret_cast<const uint4*>(x + size_t(t0 + t) * H + k0 + q * 8);
-            float* d = xs + t * kRtLd + q * 8;
-            d[0] = bf16lo(u.x); d[1] = bf16hi(u.x); d[2] = bf16lo(u.y); d[3] = bf16hi(u.y);
-            d[4] = bf16lo(u.z); d[5] = bf16hi(u.z); d[6] = bf16lo(u.w); d[7] = bf16hi(u.w);
-        }
+    stage(0, 0);
+    for (int kb = 0; kb < nk; ++kb) {
+        if (kb + 1 < nk) { stage((kb + 1) & 1, (kb + 1) * kRtBK); cp_async_wait<1>(); }
+        else cp_async_wait<0>();
         __syncthreads();
+        const float* wsm = wbuf + (kb & 1) * kRows * kRtLdW;
+        const uint16_t* xsm = xbuf + (kb & 1) * kRtTok * kRtLdX;
 #pragma unroll
         for (int kk = 0; kk < kRtBK; kk += 4) {
-            float4 xv[8], wv[8];
+            float4 wv[NE];
 #pragma unroll
-            for (int a = 0; a < 8; ++a) xv[a] = *reinterpret_cast<const float4*>(xs + (warp * 8 + a) * kRtLd + kk);
+            for (int b = 0; b < NE; ++b) wv[b] = *reinterpret_cast<const float4*>(wsm + (lane + 32 * b) * kRtLdW + kk);
 #pragma unroll
-            for (int b = 0; b < 8; ++b) wv[b] = *reinterpret_cast<const float4*>(ws + (lane + 32 * b) * kRtLd + kk);
+            for (int a = 0; a < 8; ++a) {
+                const uint2 u = *reinterpret_cast<const uint2*>(xsm + (warp * 8 + a) * kRtLdX + kk);
+                const float x0 = bf16lo(u.x), x1 = bf16hi(u.x), x2 = bf16lo(u.y), x3 = bf16hi(u.y);
 #pragma unroll
-            for (int a = 0; a < 8; ++a)
-#pragma unroll
-                for (int b = 0; b < 8; ++b) {
-                    acc[a][b] = fmaf(xv[a].x, wv[b].x, acc[a][b]);
-                    acc[a][b] = fmaf(xv[a].y, wv[b].y, acc[a][b]);
-                    acc[a][b] = fmaf(xv[a].z, wv[b].z, acc[a][b]);
-                    acc[a][b] = fmaf(xv[a].w, wv[b].w, acc[a][b]);
+                for (int b = 0; b < NE; ++b) {
+                    acc[a][b] = fmaf(x0, wv[b].x, acc[a][b]);
+                    acc[a][b] = fmaf(x1, wv[b].y, acc[a][b]);
+                    acc[a][b] = fmaf(x2, wv[b].z, acc[a][b]);
+                    acc[a][b] = fmaf(x3, wv[b].w, acc[a][b]);
                 }
+            }
         }
         __syncthreads();
     }
     // logits -> shared tile [32][E] (+ global when requested)
-    float* lt = ws;
+    float* lt = wbuf;
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
-        int e = lane + 32 * b;
+    for (int b = 0; b < NE; ++b) {
+        const int e = lane + 32 * b;
         if (e >= E) continue;
-        float bb = bias ? bias[e] : 0.f;
+        const float bb = bias ? bias[e] : 0.f;
 #pragma unroll
         for (int a = 0; a < 8; ++a) {
-            int t = warp * 8 + a;
-            float l = acc[a][b] + bb;
-            lt[t * kMaxExperts + e] = l;
+            const int t = warp * 8 + a;
+            const float l = acc[a][b] + bb;
+            lt[t * E + e] = l;
             if (logits && t0 + t < T) logits[size_t(t0 + t) * E + e] = l;
         }
     }
     __syncwarp();
-    // each warp handles its own 8 tokens
-    for (int a = 0; a < 8; ++a) {
-        int t = t0 + warp * 8 + a;
+    for (int a = 0; a < 8; ++a) {     // each warp ranks its own 8 tokens
+        const int t = t0 + warp * 8 + a;
         if (t >= T) break;
-        warp_topk_row(lt + (warp * 8 + a) * kMaxExperts, E, k, topk_idx + size_t(t) * k, topk_w + size_t(t) * k,
-                      nullptr);
+        warp_topk_row(lt + (warp * 8 + a) * E, E, k, topk_idx + size_t(t) * k, topk_w + size_t(t) * k, nullptr);
     }
 }
 
@@ -239,15 +254,24 @@ cudaError_t launch_route(int T, int H, int E, int k, int S, const uint16_t* x, c
         route_small_kernel<<<E, 256, 0, st>>>(a);
         return cudaGetLastError();
     }
-    size_t smem = sizeof(float) * (kMaxExperts * kRtLd + kRtTok * kRtLd);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(route_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    int grid = (T + kRtTok - 1) / kRtTok;
-    route_tile_kernel<<<grid, 128, smem, st>>>(T, H, E, k, x, wr, bias, topk_idx, topk_w, logits);
+    const int grid = (T + kRtTok - 1) / kRtTok;
+    const int ne = (E + 31) / 32;
+#define FT_RT(NEV)                                                                                          \
+    do {                                                                                                    \
+        const size_t smem = sizeof(float) * 2 * 32 * NEV * kRtLdW + sizeof(uint16_t) * 2 * kRtTok * kRtLdX; \
+        static bool set = false;                                                                            \
+        if (!set) {                                                                                         \
+            cudaError_t e = cudaFuncSetAttribute(route_tile_kernel<NEV>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)); \
+            if (e != cudaSuccess) return e;                                                                 \
+            set = true;                                                                                     \
+        }                                                                                                   \
+        route_tile_kernel<NEV><<<grid, 128, smem, st>>>(T, H, E, k, x, wr, bias, topk_idx, topk_w, logits); \
+    } while (0)
+    if (ne <= 1) FT_RT(1);
+    else if (ne <= 2) FT_RT(2);
+    else if (ne <= 4) FT_RT(4);
+    else FT_RT(8);
+#undef FT_RT
     return cudaGetLastError();
 }
 
