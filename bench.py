@@ -36,7 +36,6 @@ from expert_offload_serving_router_b200 import inputs  # noqa: E402
 
 WORKLOAD = "qwen3_a3b"
 PREFILL_T = 4096
-DECODE_TS = (1, 4, 16)
 METRIC = "MoE-layer tokens/s (decode & prefill) and % of HBM / tensor-core roofline"
 
 
@@ -206,6 +205,73 @@ def measure_e2e(args, torch, dist, F, world, shape, weights, Wt, x, x_np, y, ws,
     return e2e
 
 
+def measure_decode(torch, F, cfg, shape, weights, Wt, ws, ws_bytes, stream, rank, hbm_gbs, dev, tokens):
+    """Decode batches through the whole-layer call, rotating over 4 weight copies (4.8 GB) so
+    no batch finds its experts in L2.  Timed as plain launches and as a replayed CUDA graph
+    of 4 calls (one per weight copy)."""
+    H, Fd, E, k = cfg.hidden, cfg.ffn, cfg.num_experts, cfg.top_k
+    nrot = 4
+    rot = [weights]
+    keep = []
+    for _ in range(1, nrot):
+        w13c, w2c = Wt["w13"].clone(), Wt["w2"].clone()
+        keep += [w13c, w2c]
+        rot.append(F.make_weights(w13c, None, w2c, None))
+    out = {}
+    for Td in tokens:
+        xd = dev(inputs.make_tokens(cfg, Td, seed=5, stream=rank))
+        yd = torch.empty((Td, H), dtype=torch.int16, device="cuda")
+        idd = torch.empty((Td, k), dtype=torch.int32, device="cuda")
+
+        def call(i, st):
+            F.ft_moe_layer_forward(shape, Td, xd, Wt["w_router"], Wt.get("bias"), rot[i % nrot], yd, idd, None, ws,
+                                   ws_bytes, st)
+
+        for i in range(8):
+            call(i, stream)
+        torch.cuda.synchronize()
+        n_it = 200
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for i in range(n_it):
+            call(i, stream)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        us_plain = d0.elapsed_time(d1) * 1e3 / n_it
+        # the same calls captured once into a graph and replayed
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream()
+        cs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cs):
+            for i in range(nrot):
+                call(i, cs)
+        cs.synchronize()
+        with torch.cuda.graph(g, stream=cs):
+            for i in range(nrot):
+                call(i, cs)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        reps = n_it // nrot
+        d0.record()
+        for _ in range(reps):
+            g.replay()
+        d1.record()
+        torch.cuda.synchronize()
+        us_graph = d0.elapsed_time(d1) * 1e3 / (reps * nrot)
+        del g
+        n_uniq = len(np.unique(idd.cpu().numpy()))
+        algo_bytes = n_uniq * 3 * H * Fd * 2 + E * H * 4 + 2 * Td * H * 2
+        out[f"T{Td}"] = {"us_graph": us_graph, "us_plain": us_plain, "tokens_per_s": Td / (us_graph * 1e-6),
+                         "experts_touched": n_uniq, "algorithmic_bytes": algo_bytes,
+                         "achieved_gbs": algo_bytes / (us_graph * 1e-6) / 1e9,
+                         "frac_hbm": algo_bytes / (us_graph * 1e-6) / 1e9 / hbm_gbs,
+                         "launches_per_call": 3, "timing": "whole layer call (memset + 3 kernels), CUDA graph replay; "
+                                                          "us_plain = back-to-back plain launches"}
+    F.ft_moe_check(ws)
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -215,7 +281,10 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-batch measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--decode-tokens", default="1,4,16", help="decode batch sizes to time (comma list)")
+    ap.add_argument("--decode-only", action="store_true", help="time only the decode batches (for profiling)")
     args = ap.parse_args()
+    args.decode_tokens = [int(v) for v in args.decode_tokens.split(",") if v]
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
@@ -267,6 +336,13 @@ def main():
     o = torch.empty((R, H), dtype=torch.int16, device="cuda")
     y = torch.empty((T, H), dtype=torch.int16, device="cuda")
     stream = torch.cuda.current_stream()
+    if args.decode_only:
+        hbm_gbs = peaks()[0]
+        decode = measure_decode(torch, F, cfg, shape, weights, Wt, ws, ws_bytes, stream, rank, hbm_gbs, dev,
+                                args.decode_tokens)
+        if rank == 0:
+            print(json.dumps({"mode": "decode-only", "workload": f"{WORKLOAD} decode", "decode": decode}), flush=True)
+        return
     NST = 5
     LAUNCHES_PER_STEP = 1 + 3 + 1 + 1 + 1   # route, permute (count/scan/scatter), gate/up, down, combine
 
@@ -336,44 +412,9 @@ def main():
 
     # ---------------- decode batches (rotating weight copies so L2 never holds the experts)
     decode = None
-    y_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
-    # ---------------- decode batches (rotating weight copies so L2 never holds the experts)
-    decode = None
     if not args.no_decode:
-        decode = {}
-        nrot = 4
-        rot = [weights] + [None] * (nrot - 1)
-        keep = []
-        for r_ in range(1, nrot):
-            w13c, w2c = Wt["w13"].clone(), Wt["w2"].clone()
-            keep += [w13c, w2c]
-            rot[r_] = F.make_weights(w13c, None, w2c, None)
-        for Td in DECODE_TS:
-            xd_np = inputs.make_tokens(cfg, Td, seed=5, stream=rank)
-            xd = dev(xd_np)
-            yd = torch.empty((Td, H), dtype=torch.int16, device="cuda")
-            idd = torch.empty((Td, k), dtype=torch.int32, device="cuda")
-            for i in range(8):
-                F.ft_moe_layer_forward(shape, Td, xd, Wt["w_router"], Wt.get("bias"), rot[i % nrot], yd, idd, None,
-                                       ws, ws_bytes, stream)
-            torch.cuda.synchronize()
-            n_it = 200
-            d0 = torch.cuda.Event(enable_timing=True)
-            d1 = torch.cuda.Event(enable_timing=True)
-            d0.record(stream)
-            for i in range(n_it):
-                F.ft_moe_layer_forward(shape, Td, xd, Wt["w_router"], Wt.get("bias"), rot[i % nrot], yd, idd, None,
-                                       ws, ws_bytes, stream)
-            d1.record(stream)
-            torch.cuda.synchronize()
-            us = d0.elapsed_time(d1) * 1e3 / n_it
-            n_uniq = len(np.unique(idd.cpu().numpy()))
-            algo_bytes = n_uniq * 3 * H * Fd * 2 + E * H * 4 + 2 * Td * H * 2
-            decode[f"T{Td}"] = {"us": us, "tokens_per_s": Td / (us * 1e-6), "experts_touched": n_uniq,
-                                "algorithmic_bytes": algo_bytes, "achieved_gbs": algo_bytes / (us * 1e-6) / 1e9,
-                                "frac_hbm": algo_bytes / (us * 1e-6) / 1e9 / hbm_gbs,
-                                "launches": 3, "timing": "whole layer call, 3 kernels + 1 memset, no CUDA graph"}
-        F.ft_moe_check(ws)
+        decode = measure_decode(torch, F, cfg, shape, weights, Wt, ws, ws_bytes, stream, rank, hbm_gbs, dev,
+                                args.decode_tokens)
 
     if rank != 0:
         if world > 1:

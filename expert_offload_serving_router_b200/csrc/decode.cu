@@ -132,15 +132,15 @@ __global__ void __launch_bounds__(256) decode_gateup_kernel(DecodeArgs a) {
             if (!MX) {
                 const uint4* gr = reinterpret_cast<const uint4*>(w.w13 + size_t(f) * H * 2);
                 const uint4* ur = reinterpret_cast<const uint4*>(w.w13 + size_t(F + f) * H * 2);
-                for (int c0 = lane; c0 < nv; c0 += 32 * 4) {
-                    uint4 wg[4], wu[4];
+                for (int c0 = lane; c0 < nv; c0 += 32 * 8) {
+                    uint4 wg[8], wu[8];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < 8; ++u) {
                         int c = c0 + 32 * u;
                         if (c < nv) { wg[u] = ldg_nc_v4(gr + c); wu[u] = ldg_nc_v4(ur + c); }
                     }
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < 8; ++u) {
                         int c = c0 + 32 * u;
                         if (c >= nv) break;
 #pragma unroll
@@ -198,79 +198,103 @@ __global__ void __launch_bounds__(256) decode_gateup_kernel(DecodeArgs a) {
 constexpr int kRPB = 16;      // hidden rows per CTA
 constexpr int kMaxDecodeRows = 32 * (kMaxTopK + 1);
 
-template <bool MX>
+// Transpose-reduce step: n per-lane values -> n/2, pairing lanes across `off`; lanes with
+// (lane & off) keep the upper half.  After log2(n) steps plus plain butterfly steps each
+// lane holds one complete warp sum (n-1 + 5 - log2 n shuffles instead of 5 n).
+__device__ __forceinline__ void tr_step(float* v, int n, int off, int lane) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+        const float send = up ? v[i] : v[i + n / 2];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, off);
+        v[i] = (up ? v[i + n / 2] : v[i]) + recv;
+    }
+}
+
+template <bool MX, int CPL>
 __global__ void __launch_bounds__(256) decode_down_kernel(DecodeArgs a) {
+    // CPL = weight vectors per lane per row (BF16: 16-byte chunks of 8; MXFP4: 32-element blocks)
+    constexpr int RB = (MX ? 16 : 24) / CPL >= 8 ? 8 : (MX ? 16 : 24) / CPL >= 4 ? 4 : (MX ? 16 : 24) / CPL >= 2 ? 2 : 1;
+    constexpr int NB = kRPB / RB;               // row batches per active group
     __shared__ float prod[kMaxDecodeRows][kRPB + 1];
     const int G = a.E + (a.S ? 1 : 0);
     const int n_active = a.sched[1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H, F = a.F;
     const int hbase = blockIdx.x * kRPB;
-    const int items = n_active * kRPB;
-    for (int it = warp; it < items; it += 8) {
-        const int slot = it / kRPB, j = it - slot * kRPB;
+    const int nvec = MX ? F / 32 : F / 8;      // vectors per row
+    for (int it = warp; it < n_active * NB; it += 8) {
+        const int slot = it / NB, j0 = (it - slot * NB) * RB;
         const int g = a.sched[2 + (G + 1) + slot];
-        const int hrow = hbase + j;
-        if (hrow >= H) continue;
         const int r0 = a.offsets[g], n = a.offsets[g + 1] - r0;
         const EW w = expert_w(a, g);
-        if (!MX) {
-            const int nv = F / 8;
-            const uint4* wr = reinterpret_cast<const uint4*>(w.w2 + size_t(hrow) * F * 2);
-            // weight row into registers (F <= 4096 -> <= 16 vectors per lane)
-            uint4 wv[16];
+        // stream RB weight rows (all loads issued before any use)
+        uint4 wv[RB][CPL];
+        uint32_t ws_[RB][CPL];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                int c = lane + 32 * u;
-                if (c < nv) wv[u] = ldg_nc_v4(wr + c);
-            }
-            for (int r = 0; r < n; ++r) {
-                const uint4* hr = reinterpret_cast<const uint4*>(a.h + size_t(r0 + r) * F);
-                float s0 = 0.f, s1 = 0.f;
+        for (int rr = 0; rr < RB; ++rr) {
+            const int hrow = min(hbase + j0 + rr, H - 1);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    int c = lane + 32 * u;
-                    if (c < nv) {
-                        uint4 hv = __ldg(hr + c);
-                        fma2_bf16(s0, wv[u].x, hv.x); fma2_bf16(s1, wv[u].y, hv.y);
-                        fma2_bf16(s0, wv[u].z, hv.z); fma2_bf16(s1, wv[u].w, hv.w);
+            for (int i = 0; i < CPL; ++i) {
+                const int c = lane + 32 * i;
+                if (c < nvec) {
+                    if (!MX) {
+                        wv[rr][i] = ldg_nc_v4(w.w2 + (size_t(hrow) * F + size_t(c) * 8) * 2);
+                    } else {
+                        wv[rr][i] = ldg_nc_v4(w.w2 + size_t(hrow) * (F / 2) + size_t(c) * 16);
+                        ws_[rr][i] = w.w2s[size_t(hrow) * (F / 32) + c];
                     }
                 }
-                float s = warp_sum(s0 + s1);
-                if (lane == 0) prod[r0 + r][j] = s;
             }
-        } else {
-            const int nblk = F / 32;
-            const uint4* wq = reinterpret_cast<const uint4*>(w.w2 + size_t(hrow) * (F / 2));
-            const uint8_t* wsr = w.w2s + size_t(hrow) * nblk;
-            uint4 cv[4];
-            uint32_t sv[4];
+        }
+        for (int r = 0; r < n; ++r) {
+            const uint4* hr = reinterpret_cast<const uint4*>(a.h + size_t(r0 + r) * F);
+            float s[RB];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {          // F <= 4096 -> <= 4 blocks per lane
-                int b = lane + 32 * u;
-                if (b < nblk) { cv[u] = ldg_nc_v4(wq + b); sv[u] = wsr[b]; }
-            }
-            for (int r = 0; r < n; ++r) {
-                const uint4* hr = reinterpret_cast<const uint4*>(a.h + size_t(r0 + r) * F);
-                float s = 0.f;
+            for (int rr = 0; rr < RB; ++rr) s[rr] = 0.f;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    int b = lane + 32 * u;
-                    if (b < nblk) {
-                        uint4 xv[4];
+            for (int i = 0; i < CPL; ++i) {
+                const int c = lane + 32 * i;
+                if (c >= nvec) break;
+                if (!MX) {
+                    const uint4 hv = __ldg(hr + c);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 hv = __ldg(hr + b * 4 + q);
-                            xv[q] = make_uint4(f32x2_to_f16x2(bf16lo(hv.x), bf16hi(hv.x)),
-                                               f32x2_to_f16x2(bf16lo(hv.y), bf16hi(hv.y)),
-                                               f32x2_to_f16x2(bf16lo(hv.z), bf16hi(hv.z)),
-                                               f32x2_to_f16x2(bf16lo(hv.w), bf16hi(hv.w)));
-                        }
-                        s = fmaf(mx_block_dot(cv[u], xv), e8m0f(sv[u]), s);
+                    for (int rr = 0; rr < RB; ++rr) {
+                        fma2_bf16(s[rr], wv[rr][i].x, hv.x); fma2_bf16(s[rr], wv[rr][i].y, hv.y);
+                        fma2_bf16(s[rr], wv[rr][i].z, hv.z); fma2_bf16(s[rr], wv[rr][i].w, hv.w);
                     }
+                } else {
+                    uint4 xv[4];
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const uint4 hv = __ldg(hr + c * 4 + qq);
+                        xv[qq] = make_uint4(f32x2_to_f16x2(bf16lo(hv.x), bf16hi(hv.x)), f32x2_to_f16x2(bf16lo(hv.y), bf16hi(hv.y)),
+                                            f32x2_to_f16x2(bf16lo(hv.z), bf16hi(hv.z)), f32x2_to_f16x2(bf16lo(hv.w), bf16hi(hv.w)));
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < RB; ++rr) s[rr] = fmaf(mx_block_dot(wv[rr][i], xv), e8m0f(ws_[rr][i]), s[rr]);
                 }
-                s = warp_sum(s);
-                if (lane == 0) prod[r0 + r][j] = s;
+            }
+            // transpose-reduce the RB partial sums across the warp
+            float v[RB];
+#pragma unroll
+            for (int rr = 0; rr < RB; ++rr) v[rr] = s[rr];
+            int nv_ = RB;
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+                if (nv_ > 1) { tr_step(v, nv_, off, lane); nv_ >>= 1; }
+                else v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+            }
+            // lane l holds the sum of value index sel(l): bit (4 - level) of l picks the upper half
+            int sel = 0;
+            {
+                int m = RB, off = 16;
+                while (m > 1) { sel = sel * 2 + ((lane & off) ? 1 : 0); m >>= 1; off >>= 1; }
+            }
+            const int lead = (lane & ~((32 / RB) - 1)) == lane;   // one lane per value index
+            if (lead) {
+                const int j = j0 + sel;
+                if (hbase + j < H) prod[r0 + r][j] = v[0];
             }
         }
     }
@@ -331,8 +355,18 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     dim3 g2((a.H + kRPB - 1) / kRPB);
-    if (mx) decode_down_kernel<true><<<g2, 256, 0, st>>>(a);
-    else decode_down_kernel<false><<<g2, 256, 0, st>>>(a);
+    const int vec = mx ? a.F / 32 : a.F / 8;          // vectors per weight row
+    const int cpl = (vec + 31) / 32;
+#define FT_DN(MXV, C) decode_down_kernel<MXV, C><<<g2, 256, 0, st>>>(a)
+    if (mx) {
+        if (cpl <= 1) FT_DN(true, 1); else if (cpl <= 2) FT_DN(true, 2); else if (cpl <= 4) FT_DN(true, 4);
+        else return cudaErrorInvalidValue;
+    } else {
+        if (cpl <= 1) FT_DN(false, 1); else if (cpl <= 2) FT_DN(false, 2); else if (cpl <= 3) FT_DN(false, 3);
+        else if (cpl <= 4) FT_DN(false, 4); else if (cpl <= 6) FT_DN(false, 6); else if (cpl <= 8) FT_DN(false, 8);
+        else if (cpl <= 12) FT_DN(false, 12); else FT_DN(false, 16);
+    }
+#undef FT_DN
     return cudaGetLastError();
 }
 

@@ -8,8 +8,9 @@
 // "Weights as A": the MMA M dimension walks weight rows and N walks the tokens of one
 // expert group, so an expert with few tokens costs an MMA of N = round_up(n, 16) instead
 // of a padded 128-row tile, and its activation box shrinks to the next power of two.
-// A CTA tile is 256 weight rows (two M=128 MMAs into two TMEM accumulators) x N tokens,
-// so each activation stage feeds twice the math of a single 128-row MMA.  The gate/up A tile interleaves gate and up rows in
+// For long contractions a CTA tile is 256 weight rows (two M=128 MMAs into two TMEM
+// accumulators) x N tokens, so each activation stage feeds twice the math; for short ones
+// it is 128 rows with double-buffered accumulators (see moe_gemm_kernel's HV).  The gate/up A tile interleaves gate and up rows in
 // blocks of 16 (rows 32i..32i+15 = gate f0+16i.., rows 32i+16..32i+31 = up f0+16i..), so
 // each TMEM lane quarter holds gate and up of the same 16 f values: lane l and l^16
 // exchange halves with one shuffle, no shared-memory round trip.
@@ -20,7 +21,7 @@
 //   warps 2-9   BF16: epilogue, two warps per TMEM lane quarter (tcgen05.ld 32x32b)
 //   warps 2-5   MXFP4: epilogue;  warps 6-9: load E2M1 codes + E8M0 scales with 128-bit
 //               loads, dequantise exactly to bf16 and write the SW128 A tile to smem
-// Operands are K-major, 128-byte swizzled, 3-stage ring of 64 KB stages; the two fp32
+// Operands are K-major, 128-byte swizzled (3 x 64 KB or 4 x 48 KB stage ring); the fp32
 // accumulators take all 512 TMEM columns.
 // Every wait is bounded: on timeout the kernel records kDevErrTimeout, drains its own
 // copies and MMAs, frees TMEM and returns.
@@ -29,7 +30,6 @@
 
 namespace ftmoe {
 
-constexpr int kStages = 3;
 constexpr int kBK = 64;                        // K per stage (one 128-byte swizzle atom of bf16)
 constexpr int kAHalfBytes = 128 * kBK * 2;     // 16 KB: one 128-row MMA operand
 constexpr int kATileBytes = 2 * kAHalfBytes;   // 32 KB: 256 weight rows per tile
@@ -42,8 +42,8 @@ constexpr unsigned long long kWaitNs = 4000000000ull;  // 4 s bound on any wait
 struct GemmParams {
     int mode;               // 0 gate/up, 1 down
     int K;                  // H or F
-    int m_tiles;            // ceil(F/128) (gate/up) or ceil(H/256) (down): 256 weight rows per tile
-    int m_rows;             // valid weight-row groups: F/64 (gate/up) or H/128 (down) 128-row halves
+    int m_tiles;            // weight-row tiles: ceil(m_rows / HV)
+    int m_rows;             // 128-row weight groups: F/64 (gate/up, 64 gate + 64 up rows) or H/128 (down)
     int G, E, F, H;
     int has_shared;
     const int32_t* offsets; // [G+1]
@@ -202,6 +202,9 @@ __device__ __forceinline__ uint32_t e8m0_bf16x2(uint32_t s) {
 // ------------------------------------------------------------------ tile schedule
 struct Tile { int g, m, row0, nvalid, halves; };
 
+// HV = 128-row weight halves per tile.  Tile t -> (group g, weight-row tile m, token tile)
+// with m fastest, so the CTAs that share a token tile run together (L2 reuse).
+template <int HV>
 __device__ __forceinline__ Tile decode_tile(int t, const int* ntile_off, int G, const int* offsets, int m_tiles,
                                             int m_rows) {
     Tile r;
@@ -216,7 +219,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* ntile_off, int G, 
     int ni = u - ntile_off[lo];
     r.row0 = offsets[lo] + ni * kGemmBN;
     r.nvalid = min(kGemmBN, offsets[lo + 1] - r.row0);
-    r.halves = min(2, m_rows - 2 * r.m);   // the last weight-row tile may hold one 128-row half
+    r.halves = min(HV, m_rows - HV * r.m);   // the last weight-row tile may hold fewer halves
     return r;
 }
 
@@ -226,27 +229,34 @@ __device__ __forceinline__ int bmap_index(int n) {   // smallest box of 16 << i 
     return i;
 }
 
-template <bool MX>
+// HV = 2: 256 weight rows per tile, both TMEM accumulators belong to one tile (single
+//         buffered), 3 stages of 64 KB -- the least activation traffic per FLOP; for long K.
+// HV = 1: 128 weight rows per tile, accumulators double buffered so the epilogue of tile i
+//         overlaps the MMAs of tile i+1, 4 stages of 48 KB; for short K.
+template <bool MX, int HV>
 __global__ void __launch_bounds__(320, 1)
 moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sw,
                 const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
                 const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_b3,
                 const __grid_constant__ CUtensorMap tm_b4, GemmParams p) {
     constexpr int kEpiWarps = MX ? 4 : 8;
+    constexpr int kSt = HV == 2 ? 3 : 4;                 // pipeline stages
+    constexpr int kATile = HV * kAHalfBytes;             // A bytes per stage
+    constexpr int kNBuf = HV == 2 ? 1 : 2;               // accumulator buffers
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + kStages * kATileBytes;
-    uint8_t* sX = sB + kStages * kBTileBytes;              // epilogue transpose buffers, 2 KB per warp
+    uint8_t* sB = smem + kSt * kATile;
+    uint8_t* sX = sB + kSt * kBTileBytes;                // epilogue transpose buffers, 2 KB per warp
     uint64_t* full = reinterpret_cast<uint64_t*>(sX + 8 * kXposeBytes);
-    uint64_t* empty = full + kStages;
-    uint64_t* tfull = empty + kStages;
-    uint64_t* tempty = tfull + 1;
-    uint64_t* mma_done = tempty + 1;
+    uint64_t* empty = full + kSt;
+    uint64_t* tfull = empty + kSt;
+    uint64_t* tempty = tfull + kNBuf;
+    uint64_t* mma_done = tempty + kNBuf;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* ntile_off = const_cast<int*>(reinterpret_cast<volatile int*>(tmem_slot + 2));
-    int* s_off = ntile_off + 260;                           // group row offsets [G+1]
+    int* s_off = ntile_off + 260;                        // group row offsets [G+1]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = p.G;
@@ -255,12 +265,14 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
         s_off[i] = p.offsets[i];
     }
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kSt; ++s) {
             mbar_init(&full[s], MX ? 1 + 4 : 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(tfull, 1);
-        mbar_init(tempty, kEpiWarps);
+        for (int b = 0; b < kNBuf; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kEpiWarps);
+        }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -284,19 +296,19 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
             const CUtensorMap* bm[kNumBMaps] = {&tm_b0, &tm_b1, &tm_b2, &tm_b3, &tm_b4};
             int stage = 0;
             uint32_t phase = 0;
-            int issued[kStages];
-            uint32_t issued_par[kStages];
-            for (int s = 0; s < kStages; ++s) issued[s] = 0;
+            int issued[kSt];
+            uint32_t issued_par[kSt];
+            for (int s = 0; s < kSt; ++s) issued[s] = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile tl = decode_tile(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+                const Tile tl = decode_tile<HV>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
                 const bool shared_grp = p.has_shared && tl.g == p.E;
                 const int bi = bmap_index(tl.nvalid);
                 const uint32_t bbytes = uint32_t(p.b_rows[bi]) * kBK * 2;
                 const uint32_t abytes = MX ? 0u : uint32_t(tl.halves) * kAHalfBytes;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-                    uint8_t* a = sA + stage * kATileBytes;
+                    uint8_t* a = sA + stage * kATile;
                     uint8_t* b = sB + stage * kBTileBytes;
                     const int k0 = kb * kBK;
                     mbar_expect_tx(&full[stage], abytes + bbytes);
@@ -304,56 +316,56 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
                         const CUtensorMap* m = shared_grp ? &tm_sw : &tm_w;
                         const int e = shared_grp ? 0 : tl.g;
                         for (int h = 0; h < tl.halves; ++h) {
+                            const int rg = tl.m * HV + h;       // 128-row weight group index
                             if (p.mode == 0) {
 #pragma unroll
                                 for (int i = 0; i < 4; ++i)
-                                    tma_4d(m, &full[stage], a + h * kAHalfBytes + i * 4096, k0,
-                                           tl.m * 128 + h * 64 + 16 * i, 0, e);
+                                    tma_4d(m, &full[stage], a + h * kAHalfBytes + i * 4096, k0, rg * 64 + 16 * i, 0, e);
                             } else {
-                                tma_3d(m, &full[stage], a + h * kAHalfBytes, k0, tl.m * 256 + h * 128, e);
+                                tma_3d(m, &full[stage], a + h * kAHalfBytes, k0, rg * 128, e);
                             }
                         }
                     }
                     tma_2d(bm[bi], &full[stage], b, k0, tl.row0);
                     issued[stage] = 1;
                     issued_par[stage] = phase;
-                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                    if (++stage == kSt) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
             // drain: every copy this thread issued must have landed before the CTA exits
-            for (int s = 0; s < kStages; ++s)
+            for (int s = 0; s < kSt; ++s)
                 if (issued[s]) mbar_wait(&full[s], issued_par[s], nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int stage = 0;
+            int stage = 0, buf = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile tl = decode_tile(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+                const Tile tl = decode_tile<HV>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
                 const int N = (tl.nvalid + 15) & ~15;
                 const uint32_t idesc = idesc_bf16(128, N);
-                if (!mbar_wait(tempty, acc_phase ^ 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(&tempty[buf], acc_phase ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t bd = sdesc_sw128(su32(sB + stage * kBTileBytes));
                     for (int h = 0; h < tl.halves; ++h) {
-                        const uint64_t ad = sdesc_sw128(su32(sA + stage * kATileBytes + h * kAHalfBytes));
-                        const uint32_t dtm = tmem_base + uint32_t(h * kAccCols);
+                        const uint64_t ad = sdesc_sw128(su32(sA + stage * kATile + h * kAHalfBytes));
+                        const uint32_t dtm = tmem_base + uint32_t((buf * HV + h) * kAccCols);
 #pragma unroll
                         for (int kk = 0; kk < kBK / 16; ++kk)
                             umma_bf16(dtm, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
                     }
                     umma_commit(&empty[stage]);
-                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                    if (++stage == kSt) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                umma_commit(tfull);
-                acc_phase ^= 1;
+                umma_commit(&tfull[buf]);
+                if (++buf == kNBuf) { buf = 0; acc_phase ^= 1; }
             }
             if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
             umma_commit(mma_done);               // tracks completion of every MMA issued above
@@ -367,11 +379,12 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
         const int part = (warp - 2) >> 2;        // which column chunks this warp takes
         constexpr int kParts = kEpiWarps / 4;
         uint16_t* xb = reinterpret_cast<uint16_t*>(sX + (warp - 2) * kXposeBytes);
+        int buf = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            const Tile tl = decode_tile(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
-            if (!mbar_wait(tfull, acc_phase, abort_flag)) { ok = false; break; }
+            const Tile tl = decode_tile<HV>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+            if (!mbar_wait(&tfull[buf], acc_phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const int nch = (tl.nvalid + 31) >> 5;
             const int per_half = (nch - part + kParts - 1) / kParts;   // chunks c = part, part + kParts, ...
@@ -384,13 +397,14 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
                     const int iu = it + u < items ? it + u : it;
                     hh[u] = iu / per_half;
                     cc[u] = part + kParts * (iu - hh[u] * per_half);
-                    tmem_ld32_nowait(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(hh[u] * kAccCols + cc[u] * 32), v[u]);
+                    tmem_ld32_nowait(tmem_base + (uint32_t(q * 32) << 16) + uint32_t((buf * HV + hh[u]) * kAccCols + cc[u] * 32),
+                                     v[u]);
                 }
                 tmem_wait_ld(v[0], v[1]);
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     if (it + u >= items) break;
-                    const int c = cc[u], h = hh[u];
+                    const int c = cc[u], rg = tl.m * HV + hh[u];
                     if (p.mode == 0) {
                         const int fl = lane & 15;
                         const bool lo = lane < 16;
@@ -403,7 +417,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
                             xb[(lo ? i : 16 + i) * 16 + fl] = f2bf(silu_mul(gt, up));
                         }
                         __syncwarp();
-                        const int fbase = tl.m * 128 + h * 64 + 16 * q;
+                        const int fbase = rg * 64 + 16 * q;
 #pragma unroll
                         for (int r = 0; r < 2; ++r) {
                             const int ch = lane + 32 * r, tok = ch >> 1, pp = ch & 1;
@@ -416,7 +430,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
 #pragma unroll
                         for (int j = 0; j < 32; ++j) xb[j * 32 + lane] = f2bf(v[u][j]);
                         __syncwarp();
-                        const int hbase = tl.m * 256 + h * 128 + 32 * q;
+                        const int hbase = rg * 128 + 32 * q;
 #pragma unroll
                         for (int r = 0; r < 4; ++r) {
                             const int ch = lane + 32 * r, tok = ch >> 2, pp = ch & 3;
@@ -431,50 +445,53 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty);
-            acc_phase ^= 1;
+            if (lane == 0) mbar_arrive(&tempty[buf]);
+            if (++buf == kNBuf) { buf = 0; acc_phase ^= 1; }
         }
         if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
     } else if (MX) {
-        // ------------------------------------------------ MXFP4 converter warps (two A rows per thread)
-        const int r0 = tid - 64 - 32 * kEpiWarps;   // 0..127: rows r0 (half 0) and r0 (half 1)
+        // ------------------------------------------------ MXFP4 converter warps (one A row per half per thread)
+        const int r0 = tid - 64 - 32 * kEpiWarps;   // 0..127: row r0 of each 128-row half
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         const int kq = p.K / 2, ks = p.K / 32;   // code / scale bytes per weight row
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Tile tl = decode_tile(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+            const Tile tl = decode_tile<HV>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
             const bool shared_grp = p.has_shared && tl.g == p.E;
             const size_t e = shared_grp ? 0 : size_t(tl.g);
-            const uint8_t* qrow[2];
-            const uint8_t* srow[2];
-            for (int h = 0; h < 2; ++h) {
-                const int hh = h < tl.halves ? h : 0;     // a missing half re-reads half 0 (unused)
+            const uint8_t* qrow[HV];
+            const uint8_t* srow[HV];
+#pragma unroll
+            for (int h = 0; h < HV; ++h) {
+                const int rg = tl.m * HV + (h < tl.halves ? h : 0);   // a missing half re-reads half 0 (unused)
                 int wrow;
                 size_t rows_per_expert;
                 if (p.mode == 0) {
                     const int i = r0 >> 5, j = r0 & 31;
-                    const int f = tl.m * 128 + hh * 64 + 16 * i + (j & 15);
+                    const int f = rg * 64 + 16 * i + (j & 15);
                     wrow = j < 16 ? f : p.F + f;
                     rows_per_expert = size_t(2) * p.F;
                 } else {
-                    wrow = tl.m * 256 + hh * 128 + r0;
+                    wrow = rg * 128 + r0;
                     rows_per_expert = size_t(p.H);
                 }
                 qrow[h] = (shared_grp ? p.swq : p.wq) + (e * rows_per_expert + wrow) * kq;
                 srow[h] = (shared_grp ? p.sws : p.ws) + (e * rows_per_expert + wrow) * ks;
             }
-            uint4 c[2][2];
-            uint32_t sc[2];
-            for (int h = 0; h < 2; ++h) {
+            uint4 c[HV][2];
+            uint32_t sc[HV];
+#pragma unroll
+            for (int h = 0; h < HV; ++h) {
                 c[h][0] = ldg_nc_v4(qrow[h]);
                 c[h][1] = ldg_nc_v4(qrow[h] + 16);
                 sc[h] = *reinterpret_cast<const uint16_t*>(srow[h]);
             }
             for (int kb = 0; kb < nk; ++kb) {
-                uint4 nx[2][2];
-                uint32_t nsc[2];
-                for (int h = 0; h < 2; ++h) {
+                uint4 nx[HV][2];
+                uint32_t nsc[HV];
+#pragma unroll
+                for (int h = 0; h < HV; ++h) {
                     nx[h][0] = c[h][0]; nx[h][1] = c[h][1]; nsc[h] = sc[h];
                     if (kb + 1 < nk) {
                         nx[h][0] = ldg_nc_v4(qrow[h] + (kb + 1) * 32);
@@ -483,8 +500,10 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
                     }
                 }
                 if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-                for (int h = 0; h < tl.halves; ++h) {
-                    uint8_t* arow = sA + stage * kATileBytes + h * kAHalfBytes + r0 * 128;
+#pragma unroll
+                for (int h = 0; h < HV; ++h) {
+                    if (h >= tl.halves) break;
+                    uint8_t* arow = sA + stage * kATile + h * kAHalfBytes + r0 * 128;
                     const uint32_t s0 = e8m0_bf16x2(sc[h] & 0xFF), s1 = e8m0_bf16x2(sc[h] >> 8);
                     const uint32_t words[8] = {c[h][0].x, c[h][0].y, c[h][0].z, c[h][0].w,
                                                c[h][1].x, c[h][1].y, c[h][1].z, c[h][1].w};
@@ -498,8 +517,9 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[stage]);
-                if (++stage == kStages) { stage = 0; phase ^= 1; }
-                for (int h = 0; h < 2; ++h) { c[h][0] = nx[h][0]; c[h][1] = nx[h][1]; sc[h] = nsc[h]; }
+                if (++stage == kSt) { stage = 0; phase ^= 1; }
+#pragma unroll
+                for (int h = 0; h < HV; ++h) { c[h][0] = nx[h][0]; c[h][1] = nx[h][1]; sc[h] = nsc[h]; }
             }
         }
         if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
@@ -555,7 +575,28 @@ static int num_sms() {
     return n;
 }
 
-static size_t gemm_smem_bytes() { return 1024 + kStages * (kATileBytes + kBTileBytes) + 8 * kXposeBytes + 256 + 8 * 260; }
+static size_t gemm_smem_bytes(int hv) {
+    const int stages = hv == 2 ? 3 : 4;
+    return 1024 + size_t(stages) * (hv * kAHalfBytes + kBTileBytes) + 8 * kXposeBytes + 256 + 8 * 260;
+}
+
+// Tile height: long contractions (K >= 1536) amortise the single-buffered 256-row tile's
+// epilogue; short ones keep 128-row tiles with double-buffered accumulators.
+static int pick_halves(int K) { return K >= 1536 ? 2 : 1; }
+
+template <bool MX, int HV>
+static int launch_variant(int grid, cudaStream_t st, const CUtensorMap& tw, const CUtensorMap& tsw, const CUtensorMap* tb,
+                          const GemmParams& p) {
+    const size_t smem = gemm_smem_bytes(HV);
+    static bool set = false;
+    if (!set) {
+        if (cudaFuncSetAttribute(moe_gemm_kernel<MX, HV>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+            return 2;
+        set = true;
+    }
+    moe_gemm_kernel<MX, HV><<<grid, 320, smem, st>>>(tw, tsw, tb[0], tb[1], tb[2], tb[3], tb[4], p);
+    return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
 
 // returns 0 ok, 1 tensor-map failure, 2 launch failure
 int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
@@ -599,10 +640,11 @@ int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
         tw = tb[0];   // unused by the MXFP4 kernel (A comes from the converter warps)
         tsw = tb[0];
     }
+    const int hv = pick_halves(K);
     p.mode = L.mode;
     p.K = K;
     p.m_rows = L.mode == 0 ? L.F / 64 : L.H / 128;
-    p.m_tiles = (p.m_rows + 1) / 2;
+    p.m_tiles = (p.m_rows + hv - 1) / hv;
     p.G = L.E + (L.S ? 1 : 0);
     p.E = L.E;
     p.F = L.F;
@@ -617,26 +659,11 @@ int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
     p.ws = L.wscale;
     p.swq = static_cast<const uint8_t*>(L.sw);
     p.sws = L.swscale;
-    const size_t smem = gemm_smem_bytes();
     int grid = num_sms();
     const int max_tiles = L.max_tiles * p.m_tiles;
     if (max_tiles < grid) grid = max_tiles > 0 ? max_tiles : 1;
-    if (mx) {
-        static bool set = false;
-        if (!set) {
-            if (cudaFuncSetAttribute(moe_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 2;
-            set = true;
-        }
-        moe_gemm_kernel<true><<<grid, 320, smem, st>>>(tw, tsw, tb[0], tb[1], tb[2], tb[3], tb[4], p);
-    } else {
-        static bool set = false;
-        if (!set) {
-            if (cudaFuncSetAttribute(moe_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 2;
-            set = true;
-        }
-        moe_gemm_kernel<false><<<grid, 320, smem, st>>>(tw, tsw, tb[0], tb[1], tb[2], tb[3], tb[4], p);
-    }
-    return cudaGetLastError() == cudaSuccess ? 0 : 2;
+    if (mx) return hv == 2 ? launch_variant<true, 2>(grid, st, tw, tsw, tb, p) : launch_variant<true, 1>(grid, st, tw, tsw, tb, p);
+    return hv == 2 ? launch_variant<false, 2>(grid, st, tw, tsw, tb, p) : launch_variant<false, 1>(grid, st, tw, tsw, tb, p);
 }
 
 }  // namespace ftmoe

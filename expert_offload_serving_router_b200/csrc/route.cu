@@ -69,6 +69,7 @@ __device__ inline void warp_topk_row(const float* row, int E, int k, int32_t* id
 // ------------------------------------------------------------------ T > 32
 constexpr int kRtTok = 32;          // tokens per CTA (8 per warp)
 constexpr int kRtBK = 32;           // K slice staged per pipeline stage
+constexpr int kRtStages = 4;        // cp.async pipeline depth
 constexpr int kRtLdW = kRtBK + 4;   // floats per staged router row (conflict-free float4 reads)
 constexpr int kRtLdX = kRtBK + 8;   // bf16 per staged token row
 
@@ -79,57 +80,72 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint32_
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// NE = experts per lane (E <= 32*NE).  Each thread owns 8 tokens x NE experts of the logit
-// tile; K slices of the router rows and token rows are double buffered with cp.async.
+// NE = router rows per lane for all E (E <= 32*NE).  256 threads: warp w owns tokens
+// 8*(w&3) .. +7 and expert half w>>2 (NEH = ceil(NE/2) rows per lane), so two warps share
+// each scheduler for latency hiding.  K slices of the router rows and token rows stream
+// through a 4-stage cp.async ring (one barrier per slice).
 template <int NE>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
 route_tile_kernel(int T, int H, int E, int k, const uint16_t* __restrict__ x, const float* __restrict__ wr,
                   const float* __restrict__ bias, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                   float* __restrict__ logits) {
     extern __shared__ float4 smem4[];
     constexpr int kRows = 32 * NE;
-    float* wbuf = reinterpret_cast<float*>(smem4);                                  // [2][kRows][kRtLdW]
-    uint16_t* xbuf = reinterpret_cast<uint16_t*>(wbuf + 2 * kRows * kRtLdW);        // [2][32][kRtLdX]
+    constexpr int NEH = NE >= 2 ? NE / 2 : 1;
+    float* wbuf = reinterpret_cast<float*>(smem4);                                   // [S][kRows][kRtLdW]
+    uint16_t* xbuf = reinterpret_cast<uint16_t*>(wbuf + kRtStages * kRows * kRtLdW); // [S][32][kRtLdX]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tg = warp & 3, eh = warp >> 2;
+    const int ebase = eh * 32 * NEH;
     const int t0 = blockIdx.x * kRtTok;
     const int nk = H / kRtBK;
 
     auto stage = [&](int s, int k0) {
         float* wd = wbuf + s * kRows * kRtLdW;
-        for (int f = tid; f < E * 8; f += 128) {
+        for (int f = tid; f < E * 8; f += 256) {
             const int e = f >> 3, q = f & 7;
             cp_async16(wd + e * kRtLdW + q * 4, wr + size_t(e) * H + k0 + q * 4, 16);
         }
-        const int t = tid >> 2, q = tid & 3;
-        const bool ok = t0 + t < T;
-        cp_async16(xbuf + (s * kRtTok + t) * kRtLdX + q * 8, x + size_t(ok ? t0 + t : 0) * H + k0 + q * 8, ok ? 16 : 0);
+        if (tid < 128) {
+            const int t = tid >> 2, q = tid & 3;
+            const bool ok = t0 + t < T;
+            cp_async16(xbuf + (s * kRtTok + t) * kRtLdX + q * 8, x + size_t(ok ? t0 + t : 0) * H + k0 + q * 8,
+                       ok ? 16 : 0);
+        }
         cp_async_commit();
     };
 
-    float acc[8][NE];
+    float acc[8][NEH];
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < NE; ++b) acc[a][b] = 0.f;
+        for (int b = 0; b < NEH; ++b) acc[a][b] = 0.f;
 
-    stage(0, 0);
+#pragma unroll
+    for (int s = 0; s < kRtStages - 1; ++s) {
+        if (s < nk) stage(s, s * kRtBK);
+        else cp_async_commit();
+    }
     for (int kb = 0; kb < nk; ++kb) {
-        if (kb + 1 < nk) { stage((kb + 1) & 1, (kb + 1) * kRtBK); cp_async_wait<1>(); }
-        else cp_async_wait<0>();
-        __syncthreads();
-        const float* wsm = wbuf + (kb & 1) * kRows * kRtLdW;
-        const uint16_t* xsm = xbuf + (kb & 1) * kRtTok * kRtLdX;
+        cp_async_wait<kRtStages - 2>();     // slice kb has landed (this thread's copies)
+        __syncthreads();                    // ... and everyone's; slice kb-1 is no longer read
+        const int nxt = kb + kRtStages - 1;
+        if (nxt < nk) stage(nxt % kRtStages, nxt * kRtBK);
+        else cp_async_commit();
+        const float* wsm = wbuf + (kb % kRtStages) * kRows * kRtLdW;
+        const uint16_t* xsm = xbuf + (kb % kRtStages) * kRtTok * kRtLdX;
 #pragma unroll
         for (int kk = 0; kk < kRtBK; kk += 4) {
-            float4 wv[NE];
+            float4 wv[NEH];
 #pragma unroll
-            for (int b = 0; b < NE; ++b) wv[b] = *reinterpret_cast<const float4*>(wsm + (lane + 32 * b) * kRtLdW + kk);
+            for (int b = 0; b < NEH; ++b)
+                wv[b] = *reinterpret_cast<const float4*>(wsm + (ebase + lane + 32 * b) * kRtLdW + kk);
 #pragma unroll
             for (int a = 0; a < 8; ++a) {
-                const uint2 u = *reinterpret_cast<const uint2*>(xsm + (warp * 8 + a) * kRtLdX + kk);
+                const uint2 u = *reinterpret_cast<const uint2*>(xsm + (tg * 8 + a) * kRtLdX + kk);
                 const float x0 = bf16lo(u.x), x1 = bf16hi(u.x), x2 = bf16lo(u.y), x3 = bf16hi(u.y);
 #pragma unroll
-                for (int b = 0; b < NE; ++b) {
+                for (int b = 0; b < NEH; ++b) {
                     acc[a][b] = fmaf(x0, wv[b].x, acc[a][b]);
                     acc[a][b] = fmaf(x1, wv[b].y, acc[a][b]);
                     acc[a][b] = fmaf(x2, wv[b].z, acc[a][b]);
@@ -137,28 +153,30 @@ route_tile_kernel(int T, int H, int E, int k, const uint16_t* __restrict__ x, co
                 }
             }
         }
-        __syncthreads();
     }
+    cp_async_wait<0>();
+    __syncthreads();
     // logits -> shared tile [32][E] (+ global when requested)
     float* lt = wbuf;
 #pragma unroll
-    for (int b = 0; b < NE; ++b) {
-        const int e = lane + 32 * b;
+    for (int b = 0; b < NEH; ++b) {
+        const int e = ebase + lane + 32 * b;
         if (e >= E) continue;
         const float bb = bias ? bias[e] : 0.f;
 #pragma unroll
         for (int a = 0; a < 8; ++a) {
-            const int t = warp * 8 + a;
+            const int t = tg * 8 + a;
             const float l = acc[a][b] + bb;
             lt[t * E + e] = l;
             if (logits && t0 + t < T) logits[size_t(t0 + t) * E + e] = l;
         }
     }
-    __syncwarp();
-    for (int a = 0; a < 8; ++a) {     // each warp ranks its own 8 tokens
-        const int t = t0 + warp * 8 + a;
+    __syncthreads();
+    for (int a = 0; a < 4; ++a) {     // warp w ranks tokens 4w .. 4w+3
+        const int tl = warp * 4 + a;
+        const int t = t0 + tl;
         if (t >= T) break;
-        warp_topk_row(lt + (warp * 8 + a) * E, E, k, topk_idx + size_t(t) * k, topk_w + size_t(t) * k, nullptr);
+        warp_topk_row(lt + tl * E, E, k, topk_idx + size_t(t) * k, topk_w + size_t(t) * k, nullptr);
     }
 }
 
@@ -258,14 +276,14 @@ cudaError_t launch_route(int T, int H, int E, int k, int S, const uint16_t* x, c
     const int ne = (E + 31) / 32;
 #define FT_RT(NEV)                                                                                          \
     do {                                                                                                    \
-        const size_t smem = sizeof(float) * 2 * 32 * NEV * kRtLdW + sizeof(uint16_t) * 2 * kRtTok * kRtLdX; \
+        const size_t smem = sizeof(float) * kRtStages * 32 * NEV * kRtLdW + sizeof(uint16_t) * kRtStages * kRtTok * kRtLdX; \
         static bool set = false;                                                                            \
         if (!set) {                                                                                         \
             cudaError_t e = cudaFuncSetAttribute(route_tile_kernel<NEV>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)); \
             if (e != cudaSuccess) return e;                                                                 \
             set = true;                                                                                     \
         }                                                                                                   \
-        route_tile_kernel<NEV><<<grid, 128, smem, st>>>(T, H, E, k, x, wr, bias, topk_idx, topk_w, logits); \
+        route_tile_kernel<NEV><<<grid, 256, smem, st>>>(T, H, E, k, x, wr, bias, topk_idx, topk_w, logits); \
     } while (0)
     if (ne <= 1) FT_RT(1);
     else if (ne <= 2) FT_RT(2);
