@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark: MoE-layer tokens/s on B200 and the roofline fraction of the dominant kernel.
 
-Workload (default): the Qwen3-A3B-shaped MoE layer -- hidden 2048, expert FFN 768
+Workload (headline): the Qwen3-A3B-shaped MoE layer -- hidden 2048, expert FFN 768
 (SwiGLU), 128 experts, top-8 with a Zipf(s=1) rank-scaled router bias, BF16 weights
 N(0, 0.02^2) -- on a 4096-token prefill batch (x ~ N(0,1) bf16).  One step = one pass of
 the whole hot path: route (fp32 logits + top-k + gates), permute (counting sort + row
@@ -9,9 +9,11 @@ gather), grouped gate/up GEMM with fused SwiGLU, grouped down GEMM, combine.  We
 (1.21 GB) and the permuted activations exceed the 126 MB L2, so every step streams
 from HBM without an explicit flush.  Decode batches (1/4/16 tokens) are reported in
 an extra object, timed while rotating over 4 weight copies so that no batch finds its
-experts in L2.
+experts in L2.  --extra adds the other layer shapes (DeepSeek-V4-Flash-shaped MXFP4,
+Gemma-4-26B-A4B-shaped with a shared expert, the tiny layer) and --stack the
+expert-offload stack (8 DSV4-Flash-shaped layers served from pinned host memory).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--extra] [--stack]
 
 Multi-GPU: the layer forward does not shard (one GPU per layer by construction), so
 N > 1 runs N independent replicas, one process per GPU under torchrun; value is the
@@ -37,6 +39,7 @@ from expert_offload_serving_router_b200 import inputs  # noqa: E402
 WORKLOAD = "qwen3_a3b"
 PREFILL_T = 4096
 METRIC = "MoE-layer tokens/s (decode & prefill) and % of HBM / tensor-core roofline"
+LAUNCHES_PER_STEP = 1 + 3 + 1 + 1 + 1   # route, permute (count/scan/scatter), gate/up, down, combine
 
 
 def peaks():
@@ -171,61 +174,137 @@ def run_reference(args, rank):
 
 
 # ------------------------------------------------------------------ GPU arm
-def measure_e2e(args, torch, dist, F, world, shape, weights, Wt, x, x_np, y, ws, ws_bytes, stream, T, H):
-    """Same metric through the public whole-layer call with pinned host buffers: every step
-    copies x host->device, runs ft_moe_layer_forward and copies y device->host."""
-    x_host = torch.from_numpy(x_np.view(np.int16)).pin_memory()
-    y_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
-    xe = torch.empty_like(x)
+class Layer:
+    """One layer's weights resident on the GPU, plus the ABI structs."""
+    KEYS = ("w13", "w13_scale", "w2", "w2_scale", "shared_w13", "shared_w13_scale", "shared_w2", "shared_w2_scale")
 
-    def e2e_step():
-        xe.copy_(x_host, non_blocking=True)
-        F.ft_moe_layer_forward(shape, T, xe, Wt["w_router"], Wt.get("bias"), weights, y, None, None, ws, ws_bytes,
-                               stream)
-        y_host.copy_(y, non_blocking=True)
+    def __init__(self, torch, F, cfg, layer_np):
+        self.cfg = cfg
+        self.np = layer_np
+        self.t = {k: self.dev(torch, v) for k, v in layer_np.items() if v is not None}
+        self.shape = F.make_shape(cfg.hidden, cfg.ffn, cfg.num_experts, cfg.top_k, cfg.num_shared, cfg.wdtype)
+        self.weights = self.struct(F, self.t)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    @staticmethod
+    def dev(torch, a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            a = a.view(np.int16)
+        return torch.from_numpy(a).cuda()
+
+    def struct(self, F, t):
+        return F.make_weights(*[t.get(k) for k in self.KEYS[:4]], None, *[t.get(k) for k in self.KEYS[4:]])
+
+    def copy_weights(self, F):
+        """A second copy of the routed expert weights (for L2-defeating rotation)."""
+        t = dict(self.t)
+        for k in self.KEYS[:4]:
+            if k in t:
+                t[k] = t[k].clone()
+        return self.struct(F, t), t
+
+    def expert_bytes(self):
+        c = self.cfg
+        hf = c.hidden * c.ffn
+        return 3 * hf * 2 if c.wdtype == inputs.WDTYPE_BF16 else 3 * hf // 2 + 3 * hf // 32
+
+
+def measure_prefill(torch, F, L, T, steps, warmup, stream, rank, clock_index=None):
+    """Stepwise prefill through the public stage entry points, CUDA events between stages."""
+    cfg = L.cfg
+    H, Fd, E, k, S = cfg.hidden, cfg.ffn, cfg.num_experts, cfg.top_k, cfg.num_shared
+    R, G = T * k + (T if S else 0), E + (1 if S else 0)
+    x = Layer.dev(torch, inputs.make_tokens(cfg, T, seed=0, stream=rank))
+    ws_bytes = F.ft_moe_workspace_bytes(L.shape, T)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    F.ft_moe_workspace_init(ws)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    off = torch.empty(G + 1, dtype=torch.int32, device="cuda")
+    sf = torch.empty(R, dtype=torch.int32, device="cuda")
+    inv = torch.empty(R, dtype=torch.int32, device="cuda")
+    xs = torch.empty((R, H), dtype=torch.int16, device="cuda")
+    hbuf = torch.empty((R, Fd), dtype=torch.int16, device="cuda")
+    o = torch.empty((R, H), dtype=torch.int16, device="cuda")
+    y = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    nst = 5
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        F.ft_moe_route(L.shape, T, x, L.t["w_router"], L.t.get("bias"), idx, gw, None, ws, ws_bytes, stream)
+        mark(1)
+        F.ft_moe_permute(L.shape, T, idx, x, off, sf, inv, xs, ws, ws_bytes, stream)
+        mark(2)
+        F.ft_moe_experts_gateup(L.shape, T, L.weights, xs, off, hbuf, ws, ws_bytes, stream)
+        mark(3)
+        F.ft_moe_experts_down(L.shape, T, L.weights, hbuf, off, o, ws, ws_bytes, stream)
+        mark(4)
+        F.ft_moe_combine(L.shape, T, o, inv, gw, y, stream)
+        mark(5)
+
+    for _ in range(warmup):
+        step()
+    F.ft_moe_check(ws)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(steps)]
+    clk = ClockSampler(clock_index) if clock_index is not None else None
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    if clk:
+        clk.start()
+        time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(steps):
+        step(evs[s])
+    t1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
-           "d2h_bytes_per_step": T * H * 2, "ms_per_step": e2e_ms}
+    clocks = clk.stop() if clk else None
+    F.ft_moe_check(ws)
+    total_ms = t0.elapsed_time(t1)
+    stage = np.zeros(nst)
+    for s in range(steps):
+        for i in range(nst):
+            stage[i] += evs[s][i].elapsed_time(evs[s][i + 1])
+    stage /= steps
+    n_rows = int(off[G].item())
+    gu_flops = 2.0 * n_rows * (2 * Fd) * H
+    dn_flops = 2.0 * n_rows * Fd * H
+    touched = int((off[1:] - off[:-1] > 0).sum().item())
+    wbytes = touched * L.expert_bytes()
+    names = ["route", "permute", "gateup_gemm", "down_gemm", "combine"]
+    return dict(T=T, ms_step=total_ms / steps, total_ms=total_ms, stage_ms={n: float(v) for n, v in zip(names, stage)},
+                gateup_tflops=gu_flops / (stage[2] * 1e-3) / 1e12, down_tflops=dn_flops / (stage[3] * 1e-3) / 1e12,
+                gateup_flops=gu_flops, down_flops=dn_flops, experts_touched=touched, weight_bytes=wbytes,
+                clocks=clocks, ctx=dict(x=x, ws=ws, ws_bytes=ws_bytes, y=y))
 
-    return e2e
 
-
-def measure_decode(torch, F, cfg, shape, weights, Wt, ws, ws_bytes, stream, rank, hbm_gbs, dev, tokens):
-    """Decode batches through the whole-layer call, rotating over 4 weight copies (4.8 GB) so
-    no batch finds its experts in L2.  Timed as plain launches and as a replayed CUDA graph
+def measure_decode(torch, F, L, tokens, rank, hbm_gbs):
+    """Decode batches through the whole-layer call, rotating over 4 weight copies so no
+    batch finds its experts in L2.  Timed as plain launches and as a replayed CUDA graph
     of 4 calls (one per weight copy)."""
-    H, Fd, E, k = cfg.hidden, cfg.ffn, cfg.num_experts, cfg.top_k
+    cfg = L.cfg
+    H, E, k = cfg.hidden, cfg.num_experts, cfg.top_k
     nrot = 4
-    rot = [weights]
-    keep = []
+    rot, keep = [L.weights], []
     for _ in range(1, nrot):
-        w13c, w2c = Wt["w13"].clone(), Wt["w2"].clone()
-        keep += [w13c, w2c]
-        rot.append(F.make_weights(w13c, None, w2c, None))
+        wstruct, t = L.copy_weights(F)
+        rot.append(wstruct)
+        keep.append(t)
+    stream = torch.cuda.current_stream()
     out = {}
     for Td in tokens:
-        xd = dev(inputs.make_tokens(cfg, Td, seed=5, stream=rank))
+        xd = Layer.dev(torch, inputs.make_tokens(cfg, Td, seed=5, stream=rank))
         yd = torch.empty((Td, H), dtype=torch.int16, device="cuda")
         idd = torch.empty((Td, k), dtype=torch.int32, device="cuda")
+        ws_bytes = F.ft_moe_workspace_bytes(L.shape, Td)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        F.ft_moe_workspace_init(ws)
 
         def call(i, st):
-            F.ft_moe_layer_forward(shape, Td, xd, Wt["w_router"], Wt.get("bias"), rot[i % nrot], yd, idd, None, ws,
-                                   ws_bytes, st)
+            F.ft_moe_layer_forward(L.shape, Td, xd, L.t["w_router"], L.t.get("bias"), rot[i % nrot], yd, idd, None,
+                                   ws, ws_bytes, st)
 
         for i in range(8):
             call(i, stream)
@@ -238,7 +317,6 @@ def measure_decode(torch, F, cfg, shape, weights, Wt, ws, ws_bytes, stream, rank
         d1.record(stream)
         torch.cuda.synchronize()
         us_plain = d0.elapsed_time(d1) * 1e3 / n_it
-        # the same calls captured once into a graph and replayed
         g = torch.cuda.CUDAGraph()
         cs = torch.cuda.Stream()
         cs.wait_stream(torch.cuda.current_stream())
@@ -261,14 +339,156 @@ def measure_decode(torch, F, cfg, shape, weights, Wt, ws, ws_bytes, stream, rank
         us_graph = d0.elapsed_time(d1) * 1e3 / (reps * nrot)
         del g
         n_uniq = len(np.unique(idd.cpu().numpy()))
-        algo_bytes = n_uniq * 3 * H * Fd * 2 + E * H * 4 + 2 * Td * H * 2
+        algo_bytes = (n_uniq + cfg.num_shared) * L.expert_bytes() + E * H * 4 + 2 * Td * H * 2
         out[f"T{Td}"] = {"us_graph": us_graph, "us_plain": us_plain, "tokens_per_s": Td / (us_graph * 1e-6),
                          "experts_touched": n_uniq, "algorithmic_bytes": algo_bytes,
                          "achieved_gbs": algo_bytes / (us_graph * 1e-6) / 1e9,
                          "frac_hbm": algo_bytes / (us_graph * 1e-6) / 1e9 / hbm_gbs,
-                         "launches_per_call": 3, "timing": "whole layer call (memset + 3 kernels), CUDA graph replay; "
+                         "launches_per_call": 3, "timing": "whole layer call (3 kernels), CUDA graph replay; "
                                                           "us_plain = back-to-back plain launches"}
-    F.ft_moe_check(ws)
+        F.ft_moe_check(ws)
+    return out
+
+
+def measure_e2e(torch, dist, F, L, ctx, T, steps, warmup, world):
+    """Same metric through the public whole-layer call with pinned host buffers: every step
+    copies x host->device, runs ft_moe_layer_forward and copies y device->host."""
+    H = L.cfg.hidden
+    stream = torch.cuda.current_stream()
+    x, ws, ws_bytes, y = ctx["x"], ctx["ws"], ctx["ws_bytes"], ctx["y"]
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
+    xe = torch.empty_like(x)
+
+    def e2e_step():
+        xe.copy_(x_host, non_blocking=True)
+        F.ft_moe_layer_forward(L.shape, T, xe, L.t["w_router"], L.t.get("bias"), L.weights, y, None, None, ws,
+                               ws_bytes, stream)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": world * T / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+            "d2h_bytes_per_step": T * H * 2, "ms_per_step": ms}
+
+
+def summarize_prefill(p, hbm_gbs, tc_peak):
+    t_gemm = (p["stage_ms"]["gateup_gemm"] + p["stage_ms"]["down_gemm"]) * 1e-3
+    return {"T": p["T"], "ms_step": p["ms_step"], "tokens_per_s": p["T"] / (p["ms_step"] * 1e-3),
+            "stage_ms": p["stage_ms"], "gateup_tflops": p["gateup_tflops"], "down_tflops": p["down_tflops"],
+            "gateup_frac_tc": p["gateup_tflops"] / tc_peak,
+            "experts_frac_tc": (p["gateup_flops"] + p["down_flops"]) / t_gemm / 1e12 / tc_peak,
+            "experts_frac_hbm": p["weight_bytes"] / t_gemm / 1e9 / hbm_gbs, "experts_touched": p["experts_touched"]}
+
+
+def measure_stack(torch, F, rank, hbm_gbs):
+    """Expert-offload stack: 8 DSV4-Flash-shaped MXFP4 layers in pinned host memory, an
+    8192-token prefill streamed with full-layer double buffering, then 256 single-token
+    decode steps through 32 HBM expert slots per layer (cold start)."""
+    st = inputs.STACK
+    cfg = inputs.CONFIGS[st["layer"]]
+    nl, slots = st["num_layers"], st["slots_per_layer"]
+    H = cfg.hidden
+    shape = F.make_shape(cfg.hidden, cfg.ffn, cfg.num_experts, cfg.top_k, 0, cfg.wdtype)
+    hl = (F.ft_moe_weights * nl)()
+    pinned, routers = [], []
+    t_gen = time.perf_counter()
+    for l in range(nl):
+        d = inputs.make_layer(cfg, seed=0, layer=l, zipf=True, config_id=st["config_id"])
+        ph = {}
+        for key in ("w13", "w13_scale", "w2", "w2_scale"):
+            a = np.ascontiguousarray(d[key])
+            t = torch.empty(a.nbytes, dtype=torch.uint8, pin_memory=True)
+            t.numpy()[:] = a.view(np.uint8).ravel()
+            ph[key] = t
+        pinned.append(ph)
+        hl[l] = F.make_weights(ph["w13"], ph["w13_scale"], ph["w2"], ph["w2_scale"])
+        routers.append((Layer.dev(torch, d["w_router"]), Layer.dev(torch, d["bias"])))
+        del d
+    t_gen = time.perf_counter() - t_gen
+    cfgs = F.ft_stream_cfg(nl, slots, shape, hl, None, 0, 20000)
+    n = F.ft_expert_stream_arena_bytes(cfgs)
+    arena = torch.empty(n, dtype=torch.uint8, device="cuda")
+    cfgs.hbm_arena, cfgs.hbm_arena_bytes = arena.data_ptr(), n
+    handle = F.ft_expert_stream_create(cfgs)
+    copy_stream = torch.cuda.Stream()
+    out = {"host_bytes": int(sum(v.numel() for ph in pinned for v in ph.values())), "arena_bytes": n,
+           "input_generation_s": t_gen}
+    try:
+        # pinned host -> device bandwidth probe (one 1 GiB copy, best of 3)
+        probe_h = pinned[0]["w13"][: 1 << 30]
+        probe_d = torch.empty(probe_h.numel(), dtype=torch.uint8, device="cuda")
+        best = 0.0
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            probe_d.copy_(probe_h, non_blocking=True)
+            e1.record()
+            torch.cuda.synchronize()
+            best = max(best, probe_h.numel() / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+        out["h2d_probe_gbs"] = best
+        del probe_d
+        # prefill: all layers, double buffered
+        Tp = st["prefill_tokens"]
+        x = Layer.dev(torch, inputs.make_tokens(cfg, Tp, seed=0, stream=500))
+        wsb = F.ft_moe_workspace_bytes(shape, Tp)
+        ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+        F.ft_moe_workspace_init(ws)
+        yl = torch.empty((nl, Tp, H), dtype=torch.int16, device="cuda")
+        xl = torch.empty((nl, Tp, H), dtype=torch.int16, device="cuda")
+        wr = [r[0] for r in routers]
+        bs = [r[1] for r in routers]
+        F.ft_expert_stream_prefill(handle, Tp, x, wr, bs, yl, xl, ws, copy_stream=copy_stream)   # warm-up
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        F.ft_expert_stream_prefill(handle, Tp, x, wr, bs, yl, xl, ws, copy_stream=copy_stream)
+        e1.record()
+        torch.cuda.synchronize()
+        pf_ms = e0.elapsed_time(e1)
+        layer_bytes = out["host_bytes"] / nl
+        out["prefill"] = {"T": Tp, "ms": pf_ms, "tokens_per_s": Tp / (pf_ms * 1e-3),
+                          "h2d_gbs": out["host_bytes"] / (pf_ms * 1e-3) / 1e9,
+                          "frac_of_h2d_probe": out["host_bytes"] / (pf_ms * 1e-3) / 1e9 / best,
+                          "layer_copy_ms_at_probe": layer_bytes / (best * 1e9) * 1e3}
+        del ws, yl, xl
+        # decode: cold cache, 256 single-token steps
+        F.ft_expert_stream_reset_cache(handle)
+        steps = st["decode_steps"]
+        wsb = F.ft_moe_workspace_bytes(shape, 1)
+        ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+        F.ft_moe_workspace_init(ws)
+        yl = torch.empty((nl, 1, H), dtype=torch.int16, device="cuda")
+        xl = torch.empty((nl, 1, H), dtype=torch.int16, device="cuda")
+        xs = [Layer.dev(torch, inputs.make_tokens(cfg, 1, seed=1, stream=600 + s)) for s in range(steps)]
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for s in range(steps):
+            F.ft_expert_stream_decode_step(handle, 1, xs[s], wr, bs, yl, xl, ws, copy_stream=copy_stream)
+        torch.cuda.synchronize()
+        dec_s = time.perf_counter() - t0
+        st_all = F.ft_expert_stream_stats(handle, -1)
+        hits, misses = st_all[0], st_all[1]
+        out["decode"] = {"steps": steps, "layers": nl, "slots_per_layer": slots, "s_total": dec_s,
+                         "steps_per_s": steps / dec_s, "ms_per_step": 1e3 * dec_s / steps,
+                         "hits": hits, "misses": misses, "miss_rate": misses / max(1, hits + misses),
+                         "h2d_bytes": st_all[2], "wait_us_total": st_all[5],
+                         "timing": "host wall clock around the 256 steps (each step waits for its routed ids)"}
+        F.ft_moe_check(ws)
+    finally:
+        F.ft_expert_stream_destroy(handle)
     return out
 
 
@@ -282,7 +502,10 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--decode-tokens", default="1,4,16", help="decode batch sizes to time (comma list)")
-    ap.add_argument("--decode-only", action="store_true", help="time only the decode batches (for profiling)")
+    ap.add_argument("--decode-only", default=None, metavar="CONFIG",
+                    help="time only decode batches of this layer shape (for profiling)")
+    ap.add_argument("--extra", action="store_true", help="also measure the other layer shapes")
+    ap.add_argument("--stack", action="store_true", help="also measure the expert-offload stack")
     args = ap.parse_args()
     args.decode_tokens = [int(v) for v in args.decode_tokens.split(",") if v]
     rank = int(os.environ.get("RANK", 0))
@@ -305,116 +528,47 @@ def main():
     if not os.path.exists(F.LIB_PATH):
         ftbuild.build()
     F.lib()
+    hbm_gbs, tc_burst, tc_sus, peak_src = peaks()
+
+    if args.decode_only:
+        cfg = inputs.CONFIGS[args.decode_only]
+        L = Layer(torch, F, cfg, inputs.make_layer(cfg, seed=0))
+        dec = measure_decode(torch, F, L, args.decode_tokens, rank, hbm_gbs)
+        if rank == 0:
+            print(json.dumps({"mode": "decode-only", "workload": f"{cfg.name} decode", "decode": dec}), flush=True)
+        return
 
     cfg = inputs.CONFIGS[WORKLOAD]
-    T = PREFILL_T
-    H, Fd, E, k = cfg.hidden, cfg.ffn, cfg.num_experts, cfg.top_k
-    R = T * k
     layer_np = inputs.make_layer(cfg, seed=0)
-
-    def dev(a):
-        a = np.ascontiguousarray(a)
-        if a.dtype == np.uint16:
-            a = a.view(np.int16)
-        return torch.from_numpy(a).cuda()
-
-    Wt = {kk: dev(v) for kk, v in layer_np.items() if v is not None}
-    shape = F.make_shape(H, Fd, E, k, cfg.num_shared, cfg.wdtype)
-    weights = F.make_weights(Wt["w13"], None, Wt["w2"], None)
-    x_np = inputs.make_tokens(cfg, T, seed=0, stream=rank)
-    x = dev(x_np)
-    ws_bytes = F.ft_moe_workspace_bytes(shape, T)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
-    F.ft_moe_workspace_init(ws)
-    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
-    gw = torch.empty((T, k), dtype=torch.float32, device="cuda")
-    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
-    sf = torch.empty(R, dtype=torch.int32, device="cuda")
-    inv = torch.empty(R, dtype=torch.int32, device="cuda")
-    xs = torch.empty((R, H), dtype=torch.int16, device="cuda")
-    hbuf = torch.empty((R, Fd), dtype=torch.int16, device="cuda")
-    o = torch.empty((R, H), dtype=torch.int16, device="cuda")
-    y = torch.empty((T, H), dtype=torch.int16, device="cuda")
-    stream = torch.cuda.current_stream()
-    if args.decode_only:
-        hbm_gbs = peaks()[0]
-        decode = measure_decode(torch, F, cfg, shape, weights, Wt, ws, ws_bytes, stream, rank, hbm_gbs, dev,
-                                args.decode_tokens)
-        if rank == 0:
-            print(json.dumps({"mode": "decode-only", "workload": f"{WORKLOAD} decode", "decode": decode}), flush=True)
-        return
-    NST = 5
-    LAUNCHES_PER_STEP = 1 + 3 + 1 + 1 + 1   # route, permute (count/scan/scatter), gate/up, down, combine
-
-    def step(ev=None):
-        def mark(i):
-            if ev is not None:
-                ev[i].record(stream)
-        mark(0)
-        F.ft_moe_route(shape, T, x, Wt["w_router"], Wt.get("bias"), idx, gw, None, ws, ws_bytes, stream)
-        mark(1)
-        F.ft_moe_permute(shape, T, idx, x, off, sf, inv, xs, ws, ws_bytes, stream)
-        mark(2)
-        F.ft_moe_experts_gateup(shape, T, weights, xs, off, hbuf, ws, ws_bytes, stream)
-        mark(3)
-        F.ft_moe_experts_down(shape, T, weights, hbuf, off, o, ws, ws_bytes, stream)
-        mark(4)
-        F.ft_moe_combine(shape, T, o, inv, gw, y, stream)
-        mark(5)
-
-    for _ in range(args.warmup):
-        step()
-    F.ft_moe_check(ws)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NST + 1)] for _ in range(args.steps)]
-    clk = ClockSampler(local)
+    L = Layer(torch, F, cfg, layer_np)
+    T = PREFILL_T
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
-    clk.start()
-    time.sleep(0.3)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for s in range(args.steps):
-        step(evs[s])
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = clk.stop()
-    F.ft_moe_check(ws)
-    total_ms = t_start.elapsed_time(t_end)
-    stage_ms = np.zeros(NST)
-    for s in range(args.steps):
-        for i in range(NST):
-            stage_ms[i] += evs[s][i].elapsed_time(evs[s][i + 1])
-    stage_ms /= args.steps
-    ms_step = total_ms / args.steps
+    pre = measure_prefill(torch, F, L, T, args.steps, args.warmup, torch.cuda.current_stream(), rank, local)
+    ms_step = pre["ms_step"]
     if world > 1:
         t = torch.tensor([ms_step], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step = float(t.item())
+        dist.barrier()
     value = world * T / (ms_step * 1e-3)
-
-    hbm_gbs, tc_burst, tc_sus, peak_src = peaks()
-    timed_s = total_ms * 1e-3
-    tc_peak = tc_sus if timed_s > 1.0 else tc_burst
-    gu_flops = 2.0 * R * (2 * Fd) * H          # algorithmic FLOPs of one gate/up launch
-    dn_flops = 2.0 * R * Fd * H
-    gu_tflops = gu_flops / (stage_ms[2] * 1e-3) / 1e12
-    dn_tflops = dn_flops / (stage_ms[3] * 1e-3) / 1e12
+    tc_peak = tc_sus if pre["total_ms"] > 1000.0 else tc_burst
     traffic = recorded_traffic("moe_gemm_gateup_qwen3_a3b_T4096.md", "gemm_sm100.cu")
-
-    # ---------------- end to end through the public call, host buffers
-    e2e = None
-    if not args.no_e2e:
-        e2e = measure_e2e(args, torch, dist, F, world, shape, weights, Wt, x, x_np, y, ws, ws_bytes, stream, T, H)
-
-    # ---------------- decode batches (rotating weight copies so L2 never holds the experts)
-    decode = None
-    if not args.no_decode:
-        decode = measure_decode(torch, F, cfg, shape, weights, Wt, ws, ws_bytes, stream, rank, hbm_gbs, dev,
-                                args.decode_tokens)
+    e2e = None if args.no_e2e else measure_e2e(torch, dist, F, L, pre["ctx"], T, args.steps, args.warmup, world)
+    decode = None if args.no_decode else measure_decode(torch, F, L, args.decode_tokens, rank, hbm_gbs)
+    extra = None
+    if args.extra:
+        extra = {}
+        for name, Tp, Tds in [("dsv4_flash", 8192, [1, 8]), ("gemma4_26b_a4b", 2048, [1]), ("tiny", 64, [])]:
+            c = inputs.CONFIGS[name]
+            Lx = Layer(torch, F, c, inputs.make_layer(c, seed=0))
+            px = measure_prefill(torch, F, Lx, Tp, 10, 3, torch.cuda.current_stream(), rank)
+            extra[name] = {"prefill": summarize_prefill(px, hbm_gbs, tc_burst)}
+            if Tds:
+                extra[name]["decode"] = measure_decode(torch, F, Lx, Tds, rank, hbm_gbs)
+            del Lx, px
+            torch.cuda.empty_cache()
+    stack = measure_stack(torch, F, rank, hbm_gbs) if args.stack else None
 
     if rank != 0:
         if world > 1:
@@ -423,24 +577,25 @@ def main():
     cpu = None
     if world == 1 and not args.no_cpu:
         cpu = cpu_baseline(cfg, layer_np)
+    sp = summarize_prefill(pre, hbm_gbs, tc_peak)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded numpy: N(0,0.02^2) bf16 weights, "
                                                        "N(0,1) bf16 tokens, Zipf(1) router bias)",
-        "config": {"workload": f"{WORKLOAD} MoE layer prefill, T={T}", "hidden": H, "ffn": Fd, "experts": E,
-                   "top_k": k, "tokens": T, "weights": "bf16", "parallelism": f"replicas x{world}",
+        "config": {"workload": f"{WORKLOAD} MoE layer prefill, T={T}", "hidden": cfg.hidden, "ffn": cfg.ffn,
+                   "experts": cfg.num_experts, "top_k": cfg.top_k, "tokens": T, "weights": "bf16",
+                   "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (1.21 GB weights + 134 MB permuted rows per step), no flush"},
         "roofline": {"bound": "tensor", "kernel": "moe_gemm_kernel<bf16> gate/up + SwiGLU",
-                     "achieved": gu_tflops, "peak": tc_peak, "unit": "TFLOP/s", "frac": gu_tflops / tc_peak,
+                     "achieved": pre["gateup_tflops"], "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": pre["gateup_tflops"] / tc_peak,
                      "peak_source": f"{peak_src} bf16 {'sustained' if tc_peak == tc_sus else 'burst'}",
-                     "algorithmic_flops_per_launch": gu_flops, "traffic": traffic},
-        "stages_ms": {"route": stage_ms[0], "permute": stage_ms[1], "gateup_gemm": stage_ms[2],
-                      "down_gemm": stage_ms[3], "combine": stage_ms[4]},
-        "down_gemm_tflops": dn_tflops,
-        "experts_frac_of_peak": (gu_flops + dn_flops) / ((stage_ms[2] + stage_ms[3]) * 1e-3) / 1e12 / tc_peak,
-        "e2e": e2e, "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks,
-        "cpu_baseline": cpu, "decode": decode,
+                     "algorithmic_flops_per_launch": pre["gateup_flops"], "traffic": traffic},
+        "stages_ms": sp["stage_ms"], "down_gemm_tflops": pre["down_tflops"],
+        "experts_frac_of_peak": sp["experts_frac_tc"], "experts_frac_of_hbm": sp["experts_frac_hbm"],
+        "e2e": e2e, "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": pre["clocks"],
+        "cpu_baseline": cpu, "decode": decode, "other_workloads": extra, "offload_stack": stack,
     }
     print(json.dumps(line), flush=True)
     if world > 1:

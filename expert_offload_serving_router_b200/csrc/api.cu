@@ -211,8 +211,7 @@ ft_status ft_moe_route(const ft_moe_shape* shape, int32_t T, const void* x, cons
     if ((s = check_ws(shape, T, ws, ws_bytes, &L))) return s;
     if ((s = cuda_state())) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint32_t* err = ws_at<uint32_t>(ws, L.err);
-    if ((s = cuda_ok(cudaMemsetAsync(err + 1, 0, sizeof(uint32_t), st), "reset route ticket"))) return s;
+    uint32_t* err = ws_at<uint32_t>(ws, L.err);   // err[1]: decode-router ticket, zero between calls
     float* lg = logits ? logits : ws_at<float>(ws, L.logits);
     return cuda_ok(launch_route(T, shape->hidden, shape->num_experts, shape->top_k, shape->num_shared,
                                 static_cast<const uint16_t*>(x), w_router, bias, topk_idx, topk_w, lg, err + 1,
@@ -335,7 +334,6 @@ ft_status ft_moe_layer_forward(const ft_moe_shape* shape, int32_t T, const void*
     int32_t* inv_pos = ws_at<int32_t>(ws, L.inv_pos);
     PermOut po{offsets, sorted_flat, inv_pos, ws_at<int32_t>(ws, L.sched), err};
     const uint16_t* xb = static_cast<const uint16_t*>(x);
-    if ((s = cuda_ok(cudaMemsetAsync(err + 1, 0, sizeof(uint32_t), st), "reset route ticket"))) return s;
     if (decode) {
         // route + top-k + permutation in one launch, then two weight-streaming kernels
         if ((s = cuda_ok(launch_route(T, H, E, k, S, xb, w_router, bias, idx, gw, lg, err + 1, &po, st), "route launch")))

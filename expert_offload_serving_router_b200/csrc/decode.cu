@@ -22,6 +22,12 @@ namespace ftmoe {
 
 struct EW { const uint8_t *w13, *w13s, *w2, *w2s; };
 
+// Programmatic dependent launch: a kernel launched with the programmatic-serialization
+// attribute may start while its predecessor finishes; griddepcontrol.wait blocks until the
+// predecessor grid has completed and its memory is visible (a no-op for plain launches).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ EW expert_w(const DecodeArgs& a, int g) {
     EW r;
     if (g >= a.E) { r.w13 = a.sw13; r.w13s = a.sw13s; r.w2 = a.sw2; r.w2s = a.sw2s; return r; }
@@ -88,43 +94,65 @@ __device__ __forceinline__ float mx_block_dot(const uint4& c, const uint4* xv) {
 }
 
 // ------------------------------------------------------------------ gate/up + SwiGLU
-constexpr int kFPB = 16;      // f values per CTA (2 per warp)
+constexpr int kFPB = 8;       // f values per CTA (one per warp)
 
-template <int TB, bool MX>
+template <int TB, bool MX, bool FULLX>
 __global__ void __launch_bounds__(256) decode_gateup_kernel(DecodeArgs a) {
-    extern __shared__ uint4 xs4[];                   // [TB][H] bf16 (BF16) or f16 (MXFP4)
+    // FULLX: every token row [T][H] staged once (bf16, or f16 for MXFP4) before the
+    // programmatic dependency wait -- the layer input is complete before the router ran --
+    // so the routing-dependent part starts straight with the weight stream.
+    // Otherwise: the group's rows are staged per batch of TB after the wait.
+    extern __shared__ uint4 xs4[];
+    __shared__ int stok[TB];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = a.H, F = a.F;
+    const int nv = H / 8;                            // 16-byte activation vectors per row
+    auto stage_row = [&](int t, int dst_row) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.x + size_t(t) * H);
+        uint4* dst = xs4 + size_t(dst_row) * nv;
+        for (int v = lane; v < nv; v += 32) {
+            uint4 u = __ldg(src + v);
+            if (MX) {
+                u = make_uint4(f32x2_to_f16x2(bf16lo(u.x), bf16hi(u.x)), f32x2_to_f16x2(bf16lo(u.y), bf16hi(u.y)),
+                               f32x2_to_f16x2(bf16lo(u.z), bf16hi(u.z)), f32x2_to_f16x2(bf16lo(u.w), bf16hi(u.w)));
+            }
+            dst[v] = u;
+        }
+    };
+    if (FULLX)
+        for (int t = warp; t < a.T; t += 8) stage_row(t, t);
+    pdl_wait();
+    pdl_trigger();
     const int G = a.E + (a.S ? 1 : 0);
+    const int P = a.T * a.k;
+    const int nfb = (F + kFPB - 1) / kFPB;
     const int n_active = a.sched[1];
-    const int slot = blockIdx.x;
-    if (slot >= n_active) return;
+    // grid-stride over (active group, f-block) items; f-block fastest so a CTA's items
+    // mostly share their group (and its staged rows)
+    for (int item = blockIdx.x; item < n_active * nfb; item += gridDim.x) {
+    const int slot = item / nfb, fblk = item - slot * nfb;
     const int g = a.sched[2 + (G + 1) + slot];
     const int r0 = a.offsets[g];
     const int n = a.offsets[g + 1] - r0;
-    const int P = a.T * a.k;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const EW w = expert_w(a, g);
-    const int H = a.H, F = a.F;
-    const int nv = H / 8;                            // 16-byte activation vectors per row
     for (int tb = 0; tb < n; tb += TB) {
         const int nb = min(TB, n - tb);
         __syncthreads();
-        for (int i = warp; i < nb; i += 8) {
-            int p = a.sorted_flat[r0 + tb + i];
-            int t = p < P ? p / a.k : p - P;
-            const uint4* src = reinterpret_cast<const uint4*>(a.x + size_t(t) * H);
-            uint4* dst = xs4 + size_t(i) * nv;
-            for (int v = lane; v < nv; v += 32) {
-                uint4 u = __ldg(src + v);
-                if (MX) {
-                    u = make_uint4(f32x2_to_f16x2(bf16lo(u.x), bf16hi(u.x)), f32x2_to_f16x2(bf16lo(u.y), bf16hi(u.y)),
-                                   f32x2_to_f16x2(bf16lo(u.z), bf16hi(u.z)), f32x2_to_f16x2(bf16lo(u.w), bf16hi(u.w)));
-                }
-                dst[v] = u;
+        if (FULLX) {
+            if (tid < nb) {
+                const int p = a.sorted_flat[r0 + tb + tid];
+                stok[tid] = p < P ? p / a.k : p - P;
             }
+        } else {
+            for (int i = warp; i < nb; i += 8) {
+                const int p = a.sorted_flat[r0 + tb + i];
+                stage_row(p < P ? p / a.k : p - P, i);
+            }
+            if (tid < nb) stok[tid] = tid;
         }
         __syncthreads();
         for (int fi = 0; fi < kFPB / 8; ++fi) {
-            const int f = blockIdx.y * kFPB + warp * (kFPB / 8) + fi;
+            const int f = fblk * kFPB + warp * (kFPB / 8) + fi;
             if (f >= F) break;
             float ag[TB], au[TB];
 #pragma unroll
@@ -146,7 +174,7 @@ __global__ void __launch_bounds__(256) decode_gateup_kernel(DecodeArgs a) {
 #pragma unroll
                         for (int i = 0; i < TB; ++i) {
                             if (i >= nb) break;
-                            uint4 xv = xs4[size_t(i) * nv + c];
+                            uint4 xv = xs4[size_t(stok[i]) * nv + c];
                             fma2_bf16(ag[i], wg[u].x, xv.x); fma2_bf16(ag[i], wg[u].y, xv.y);
                             fma2_bf16(ag[i], wg[u].z, xv.z); fma2_bf16(ag[i], wg[u].w, xv.w);
                             fma2_bf16(au[i], wu[u].x, xv.x); fma2_bf16(au[i], wu[u].y, xv.y);
@@ -176,7 +204,7 @@ __global__ void __launch_bounds__(256) decode_gateup_kernel(DecodeArgs a) {
 #pragma unroll
                         for (int i = 0; i < TB; ++i) {
                             if (i >= nb) break;
-                            const uint4* xv = xs4 + size_t(i) * nv + b * 4;
+                            const uint4* xv = xs4 + size_t(stok[i]) * nv + b * 4;
                             ag[i] = fmaf(mx_block_dot(cg[u], xv), scg, ag[i]);
                             au[i] = fmaf(mx_block_dot(cu[u], xv), scu, au[i]);
                         }
@@ -192,10 +220,11 @@ __global__ void __launch_bounds__(256) decode_gateup_kernel(DecodeArgs a) {
             }
         }
     }
+    }
 }
 
 // ------------------------------------------------------------------ down + combine
-constexpr int kRPB = 16;      // hidden rows per CTA
+constexpr int kRPB = 8;       // hidden rows per CTA
 constexpr int kMaxDecodeRows = 32 * (kMaxTopK + 1);
 
 // Transpose-reduce step: n per-lane values -> n/2, pairing lanes across `off`; lanes with
@@ -217,6 +246,7 @@ __global__ void __launch_bounds__(256) decode_down_kernel(DecodeArgs a) {
     constexpr int RB = (MX ? 16 : 24) / CPL >= 8 ? 8 : (MX ? 16 : 24) / CPL >= 4 ? 4 : (MX ? 16 : 24) / CPL >= 2 ? 2 : 1;
     constexpr int NB = kRPB / RB;               // row batches per active group
     __shared__ float prod[kMaxDecodeRows][kRPB + 1];
+    pdl_wait();
     const int G = a.E + (a.S ? 1 : 0);
     const int n_active = a.sched[1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -324,6 +354,21 @@ __global__ void __launch_bounds__(256) decode_down_kernel(DecodeArgs a) {
 }
 
 // ------------------------------------------------------------------ host launch
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
     const int P = a.T * a.k, R = P + (a.S ? a.T : 0);
@@ -332,32 +377,48 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     const bool mx = a.wdtype == FT_W_MXFP4;
     int TB = 1;
     while (TB < a.T && TB < 8) TB <<= 1;
-    // keep the staged token rows within 64 KB of shared memory
-    while (TB > 1 && size_t(TB) * a.H * 2 > 65536) TB >>= 1;
-    const size_t smem = size_t(TB) * a.H * 2;
-    dim3 g1(na_max, (a.F + kFPB - 1) / kFPB);
-#define FT_GU(TBV)                                                                                         \
-    do {                                                                                                   \
-        auto kern = mx ? decode_gateup_kernel<TBV, true> : decode_gateup_kernel<TBV, false>;              \
-        if (smem > 48 * 1024) {                                                                            \
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)); \
-            if (e != cudaSuccess) return e;                                                                \
-        }                                                                                                  \
-        kern<<<g1, 256, smem, st>>>(a);                                                                    \
+    // small batches stage all token rows once per CTA (before the dependency wait); larger
+    // ones stage each group's rows per batch of TB
+    const bool fullx = size_t(a.T) * a.H * 2 <= 16 * 1024;
+    while (!fullx && TB > 1 && size_t(TB) * a.H * 2 > 65536) TB >>= 1;
+    const size_t smem = size_t(fullx ? a.T : TB) * a.H * 2;
+    int items = na_max * ((a.F + kFPB - 1) / kFPB);   // upper bound; the kernel strides over the real count
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    dim3 g1(items < 2 * sms ? items : 2 * sms);     // two resident CTAs per SM: one wave
+    cudaError_t e = cudaSuccess;
+#define FT_GU(TBV, MXV, FX)                                                                                   \
+    do {                                                                                                      \
+        auto kern = decode_gateup_kernel<TBV, MXV, FX>;                                                       \
+        if (smem > 48 * 1024) {                                                                               \
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));            \
+            if (e != cudaSuccess) return e;                                                                   \
+        }                                                                                                     \
+        e = launch_pdl(kern, g1, dim3(256), smem, st, a);                                                    \
+    } while (0)
+#define FT_GU2(TBV)                                                                                           \
+    do {                                                                                                      \
+        if (mx) { if (fullx) FT_GU(TBV, true, true); else FT_GU(TBV, true, false); }                         \
+        else { if (fullx) FT_GU(TBV, false, true); else FT_GU(TBV, false, false); }                           \
     } while (0)
     switch (TB) {
-        case 1: FT_GU(1); break;
-        case 2: FT_GU(2); break;
-        case 4: FT_GU(4); break;
-        default: FT_GU(8); break;
+        case 1: FT_GU2(1); break;
+        case 2: FT_GU2(2); break;
+        case 4: FT_GU2(4); break;
+        default: FT_GU2(8); break;
     }
+#undef FT_GU2
 #undef FT_GU
-    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     dim3 g2((a.H + kRPB - 1) / kRPB);
     const int vec = mx ? a.F / 32 : a.F / 8;          // vectors per weight row
     const int cpl = (vec + 31) / 32;
-#define FT_DN(MXV, C) decode_down_kernel<MXV, C><<<g2, 256, 0, st>>>(a)
+#define FT_DN(MXV, C) e = launch_pdl(decode_down_kernel<MXV, C>, g2, dim3(256), 0, st, a)
     if (mx) {
         if (cpl <= 1) FT_DN(true, 1); else if (cpl <= 2) FT_DN(true, 2); else if (cpl <= 4) FT_DN(true, 4);
         else return cudaErrorInvalidValue;
@@ -367,6 +428,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
         else if (cpl <= 12) FT_DN(false, 12); else FT_DN(false, 16);
     }
 #undef FT_DN
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -8,7 +8,7 @@
 //                 scan over groups (offsets), GEMM tile schedule and active-group list.
 //   perm_scatter: one CTA per chunk; pos = chunk base + local rank; writes sorted_flat,
 //                 inv_pos and (optionally) gathers x rows into x_sorted with 16-byte moves.
-// Small path (R <= 1024): one CTA does all of it (block_permute_small).
+// Small path (R <= 1024): one warp sorts (warp_permute_small), the CTA gathers.
 #include "kernels.h"
 #include "permute_small.cuh"
 
@@ -152,21 +152,20 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(PermArgs a) {
 __global__ void __launch_bounds__(256) perm_small_kernel(const int32_t* idx, int T, int k, int E, int S, PermOut out,
                                                          const uint16_t* x, uint16_t* x_sorted, int H) {
     __shared__ int32_t sidx[1024];
-    __shared__ int grp[1024];
     __shared__ int cnt[kMaxExperts + 2];
-    __shared__ int flag[kMaxExperts + 2];
-    __shared__ int tmp[33];
     const int P = T * k, R = P + (S ? T : 0);
     for (int i = threadIdx.x; i < P; i += blockDim.x) sidx[i] = idx[i];
     __syncthreads();
-    block_permute_small(sidx, T, k, E, S, grp, cnt, flag, tmp, out);
+    if (threadIdx.x < 32) warp_permute_small(sidx, T, k, E, S, cnt, out);
     if (!x_sorted) return;
+    __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nv = H / 8;
     for (int i = warp; i < R; i += blockDim.x / 32) {
-        if (grp[i] < 0) continue;
-        int pos = out.inv_pos[i];
-        int t = i < P ? i / k : i - P;
+        const int g = i < P ? sidx[i] : E;
+        if (g < 0 || g >= E + (i >= P ? 1 : 0)) continue;
+        const int pos = out.inv_pos[i];
+        const int t = i < P ? i / k : i - P;
         const uint4* src = reinterpret_cast<const uint4*>(x + size_t(t) * H);
         uint4* dst = reinterpret_cast<uint4*>(x_sorted + size_t(pos) * H);
         for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);

@@ -1,5 +1,5 @@
-// Single-CTA counting sort used for decode-sized batches (R = T*k + S*T <= a few hundred
-// pairs).  Shared by the fused route+permute kernel and the standalone small permute.
+// Counting-sort building blocks shared by the fused decode route+permute kernel, the
+// standalone small permute and the chunked permute's scan.
 #pragma once
 #include "common.cuh"
 
@@ -57,58 +57,81 @@ struct PermOut {
     uint32_t* err;         // device error flag
 };
 
-// Scratch in shared memory: grp[R], cnt[G+1], flag[G+1], tmp[33].
-// `idx_smem` holds the [T,k] routed ids.  Whole block participates.
-__device__ inline void block_permute_small(const int32_t* idx_smem, int T, int k, int E, int S,
-                                           int* grp, int* cnt, int* flag, int* tmp, PermOut out) {
+// Single-warp counting sort for decode-sized batches (R <= a few hundred pairs): no block
+// barriers.  Called by one full warp; `idx_smem` holds the [T,k] routed ids, `cnt` is
+// shared scratch of G+1 ints.  Same outputs as the chunked path: offsets, stable positions
+// (ascending flat index within a group), active-group list and GEMM tile schedule.
+__device__ inline void warp_permute_small(const int32_t* idx_smem, int T, int k, int E, int S, int* cnt, PermOut out) {
+    const int lane = threadIdx.x & 31;
     const int P = T * k;
     const int R = P + (S ? T : 0);
     const int G = E + (S ? 1 : 0);
-    for (int g = threadIdx.x; g <= G; g += blockDim.x) cnt[g] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < R; i += blockDim.x) {
-        int g = (i < P) ? idx_smem[i] : E;
-        if (g < 0 || g >= E + (i >= P ? 1 : 0)) {  // out-of-range id: flag it, count nowhere
-            atomicExch(out.err, kDevErrBadExpert);
-            g = -1;
-        } else {
-            atomicAdd(&cnt[g], 1);
+    for (int g = lane; g <= G; g += 32) cnt[g] = 0;
+    __syncwarp();
+    for (int i = lane; i < R; i += 32) {
+        const int g = i < P ? idx_smem[i] : E;
+        if (g < 0 || g >= E + (i >= P ? 1 : 0)) atomicExch(out.err, kDevErrBadExpert);
+        else atomicAdd(&cnt[g], 1);
+    }
+    __syncwarp();
+    // one pass over the groups: lane owns the contiguous block [g0, g1); exclusive scans of
+    // counts (offsets), active flags (active-list rank) and 256-row tiles (tile schedule)
+    const int per = (G + 31) / 32;
+    const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+    int sc = 0, sa = 0, st = 0;
+    for (int g = g0; g < g1; ++g) {
+        const int c = cnt[g];
+        sc += c;
+        sa += c > 0;
+        st += (c + kGemmBN - 1) / kGemmBN;
+    }
+    int ic = sc, ia = sa, it = st;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int uc = __shfl_up_sync(0xffffffffu, ic, o);
+        const int ua = __shfl_up_sync(0xffffffffu, ia, o);
+        const int ut = __shfl_up_sync(0xffffffffu, it, o);
+        if (lane >= o) { ic += uc; ia += ua; it += ut; }
+    }
+    int oc = ic - sc, oa = ia - sa, ot = it - st;       // exclusive prefixes at g0
+    for (int g = g0; g < g1; ++g) {
+        const int c = cnt[g];
+        out.offsets[g] = oc;
+        out.sched[2 + g] = ot;
+        if (c > 0) out.sched[2 + (G + 1) + oa] = g;
+        cnt[g] = oc;                                     // becomes the scatter cursor
+        oc += c;
+        oa += c > 0;
+        ot += (c + kGemmBN - 1) / kGemmBN;
+    }
+    if (lane == 31) {
+        out.offsets[G] = ic;
+        out.sched[0] = it;
+        out.sched[1] = ia;
+        out.sched[2 + G] = it;
+    }
+    __syncwarp();
+    // stable scatter, 32 pairs at a time in flat order: rank inside the chunk from
+    // __match_any_sync, base from the group cursor, the lowest peer advances the cursor
+    for (int base = 0; base < R; base += 32) {
+        const int i = base + lane;
+        int g = -1;
+        if (i < R) {
+            g = i < P ? idx_smem[i] : E;
+            if (g < 0 || g >= E + (i >= P ? 1 : 0)) g = -1;
         }
-        grp[i] = g;
+        const unsigned peers = __match_any_sync(0xffffffffu, g);
+        const int rk = __popc(peers & ((1u << lane) - 1u));
+        int pos = 0;
+        if (g >= 0) pos = cnt[g] + rk;
+        __syncwarp();
+        if (g >= 0 && rk == 0) cnt[g] += __popc(peers);
+        __syncwarp();
+        if (g >= 0) {
+            out.sorted_flat[pos] = i;
+            out.inv_pos[i] = pos;
+        }
     }
-    __syncthreads();
-    // active flags and tiles per group (scan inputs) before the counts are overwritten
-    for (int g = threadIdx.x; g < G; g += blockDim.x) flag[g] = cnt[g] > 0 ? 1 : 0;
-    __syncthreads();
-    int n_active = block_exclusive_scan(flag, G, tmp);  // flag[g] = rank among active groups
-    // active list; ntile counts go into the sched array directly
-    for (int g = threadIdx.x; g < G; g += blockDim.x) {
-        int c = cnt[g];
-        if (c > 0) out.sched[2 + (G + 1) + flag[g]] = g;
-        flag[g] = (c + kGemmBN - 1) / kGemmBN;
-    }
-    __syncthreads();
-    int ntiles = block_exclusive_scan(flag, G, tmp);
-    for (int g = threadIdx.x; g < G; g += blockDim.x) out.sched[2 + g] = flag[g];
-    if (threadIdx.x == 0) {
-        out.sched[0] = ntiles;
-        out.sched[1] = n_active;
-        out.sched[2 + G] = ntiles;
-    }
-    int total = block_exclusive_scan(cnt, G, tmp);   // cnt[g] = offsets[g]
-    for (int g = threadIdx.x; g < G; g += blockDim.x) out.offsets[g] = cnt[g];
-    if (threadIdx.x == 0) out.offsets[G] = total;
-    // stable scatter: rank of pair i = number of earlier pairs in the same group
-    for (int i = threadIdx.x; i < R; i += blockDim.x) {
-        int g = grp[i];
-        if (g < 0) continue;
-        int r = 0;
-        for (int j = 0; j < i; ++j) r += (grp[j] == g);
-        int pos = cnt[g] + r;
-        out.sorted_flat[pos] = i;
-        out.inv_pos[i] = pos;
-    }
-    __syncthreads();
 }
 
 }  // namespace ftmoe

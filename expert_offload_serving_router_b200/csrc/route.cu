@@ -14,40 +14,48 @@
 
 namespace ftmoe {
 
+// Order-preserving 32-bit key of an fp32 logit (larger logit -> larger key); -0 is folded
+// onto +0 first so that they compare equal, as floats do.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+    uint32_t u = __float_as_uint(v);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // Warp-wide top-k over the E logits of one token held in `row` (shared memory).
-// Lane l owns experts l, l+32, ...  Ties resolve to the lower index; -0 == +0 as floats.
+// Lane l owns experts l, l+32, ...; each round: the lane's best (largest key, lowest index)
+// candidate, a warp max of the key and a warp min of the index among the lanes holding that
+// key (two redux.sync).  Ties therefore resolve to the lower expert index.
 __device__ inline void warp_topk_row(const float* row, int E, int k, int32_t* idx_out, float* w_out,
                                      int32_t* idx_smem) {
     const int lane = threadIdx.x & 31;
-    float v[kMaxExperts / 32];
-    uint32_t taken = 0;
+    constexpr int NV = kMaxExperts / 32;
+    uint32_t key[NV];
 #pragma unroll
-    for (int i = 0; i < kMaxExperts / 32; ++i) {
-        int e = lane + 32 * i;
-        v[i] = e < E ? row[e] : -INFINITY;
+    for (int i = 0; i < NV; ++i) {
+        const int e = lane + 32 * i;
+        key[i] = e < E ? logit_key(row[e]) : 0u;   // key 0 sorts below every finite logit
     }
+    uint32_t taken = 0;
     float sel_v[kMaxTopK];
     int sel_e[kMaxTopK];
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
         if (j >= k) break;
-        float bv = -INFINITY;
-        int be = 0x7fffffff;
+        uint32_t bk = 0u;
+        int bi = 0;
+        bool have = false;
 #pragma unroll
-        for (int i = 0; i < kMaxExperts / 32; ++i) {
-            int e = lane + 32 * i;
-            bool ok = e < E && !((taken >> i) & 1u);
-            if (ok && (v[i] > bv || (v[i] == bv && e < be))) { bv = v[i]; be = e; }
+        for (int i = 0; i < NV; ++i) {
+            const bool ok = (lane + 32 * i) < E && !((taken >> i) & 1u);
+            if (ok && (!have || key[i] > bk)) { bk = key[i]; bi = i; have = true; }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-        }
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        sel_v[j] = bv;
-        sel_e[j] = be;
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, have ? bk : 0u);
+        const uint32_t cand = (have && bk == kmax) ? uint32_t(lane + 32 * bi) : 0xffffffffu;
+        const uint32_t e = __reduce_min_sync(0xffffffffu, cand);
+        if (int(e & 31) == lane) taken |= 1u << (e >> 5);
+        sel_e[j] = int(e);
+        sel_v[j] = row[e];
     }
     // gates: softmax over the kept logits, fp32, summed in slot order
     float den = 0.f;
@@ -71,7 +79,7 @@ constexpr int kRtTok = 32;          // tokens per CTA (8 per warp)
 constexpr int kRtBK = 32;           // K slice staged per pipeline stage
 constexpr int kRtStages = 4;        // cp.async pipeline depth
 constexpr int kRtLdW = kRtBK + 4;   // floats per staged router row (conflict-free float4 reads)
-constexpr int kRtLdX = kRtBK + 8;   // bf16 per staged token row
+constexpr int kRtLdX = kRtBK + 4;   // floats per staged token row (fp32, converted once per slice)
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(uint32_t(__cvta_generic_to_shared(smem))),
@@ -93,26 +101,35 @@ route_tile_kernel(int T, int H, int E, int k, const uint16_t* __restrict__ x, co
     constexpr int kRows = 32 * NE;
     constexpr int NEH = NE >= 2 ? NE / 2 : 1;
     float* wbuf = reinterpret_cast<float*>(smem4);                                   // [S][kRows][kRtLdW]
-    uint16_t* xbuf = reinterpret_cast<uint16_t*>(wbuf + kRtStages * kRows * kRtLdW); // [S][32][kRtLdX]
+    float* xbuf = wbuf + kRtStages * kRows * kRtLdW;                                  // [2][32][kRtLdX] fp32
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tg = warp & 3, eh = warp >> 2;
     const int ebase = eh * 32 * NEH;
     const int t0 = blockIdx.x * kRtTok;
     const int nk = H / kRtBK;
 
-    auto stage = [&](int s, int k0) {
+    auto stage = [&](int s, int k0) {        // router rows of one K slice: cp.async
         float* wd = wbuf + s * kRows * kRtLdW;
         for (int f = tid; f < E * 8; f += 256) {
             const int e = f >> 3, q = f & 7;
             cp_async16(wd + e * kRtLdW + q * 4, wr + size_t(e) * H + k0 + q * 4, 16);
         }
-        if (tid < 128) {
-            const int t = tid >> 2, q = tid & 3;
-            const bool ok = t0 + t < T;
-            cp_async16(xbuf + (s * kRtTok + t) * kRtLdX + q * 8, x + size_t(ok ? t0 + t : 0) * H + k0 + q * 8,
-                       ok ? 16 : 0);
-        }
         cp_async_commit();
+    };
+    // token rows of one K slice go through registers and are stored as fp32, so the inner
+    // loop does no bf16 unpacking: thread tid < 128 owns token tid/4, 8 values at (tid%4)*8
+    const int xt = tid >> 2, xq = tid & 3;
+    uint4 xr = make_uint4(0, 0, 0, 0);
+    auto xload = [&](int k0) {
+        xr = make_uint4(0, 0, 0, 0);
+        if (tid < 128 && t0 + xt < T) xr = __ldg(reinterpret_cast<const uint4*>(x + size_t(t0 + xt) * H + k0 + xq * 8));
+    };
+    auto xstore = [&](int b) {
+        if (tid < 128) {
+            float* d = xbuf + (b * kRtTok + xt) * kRtLdX + xq * 8;
+            *reinterpret_cast<float4*>(d) = make_float4(bf16lo(xr.x), bf16hi(xr.x), bf16lo(xr.y), bf16hi(xr.y));
+            *reinterpret_cast<float4*>(d + 4) = make_float4(bf16lo(xr.z), bf16hi(xr.z), bf16lo(xr.w), bf16hi(xr.w));
+        }
     };
 
     float acc[8][NEH];
@@ -126,14 +143,19 @@ route_tile_kernel(int T, int H, int E, int k, const uint16_t* __restrict__ x, co
         if (s < nk) stage(s, s * kRtBK);
         else cp_async_commit();
     }
+    xload(0);
+    xstore(0);
+    if (nk > 1) xload(kRtBK);
     for (int kb = 0; kb < nk; ++kb) {
         cp_async_wait<kRtStages - 2>();     // slice kb has landed (this thread's copies)
         __syncthreads();                    // ... and everyone's; slice kb-1 is no longer read
         const int nxt = kb + kRtStages - 1;
         if (nxt < nk) stage(nxt % kRtStages, nxt * kRtBK);
         else cp_async_commit();
+        if (kb + 1 < nk) xstore((kb + 1) & 1);   // buffer of slice kb-1, free after the barrier
+        if (kb + 2 < nk) xload((kb + 2) * kRtBK);
         const float* wsm = wbuf + (kb % kRtStages) * kRows * kRtLdW;
-        const uint16_t* xsm = xbuf + (kb % kRtStages) * kRtTok * kRtLdX;
+        const float* xsm = xbuf + (kb & 1) * kRtTok * kRtLdX;
 #pragma unroll
         for (int kk = 0; kk < kRtBK; kk += 4) {
             float4 wv[NEH];
@@ -142,8 +164,8 @@ route_tile_kernel(int T, int H, int E, int k, const uint16_t* __restrict__ x, co
                 wv[b] = *reinterpret_cast<const float4*>(wsm + (ebase + lane + 32 * b) * kRtLdW + kk);
 #pragma unroll
             for (int a = 0; a < 8; ++a) {
-                const uint2 u = *reinterpret_cast<const uint2*>(xsm + (tg * 8 + a) * kRtLdX + kk);
-                const float x0 = bf16lo(u.x), x1 = bf16hi(u.x), x2 = bf16lo(u.y), x3 = bf16hi(u.y);
+                const float4 xv = *reinterpret_cast<const float4*>(xsm + (tg * 8 + a) * kRtLdX + kk);
+                const float x0 = xv.x, x1 = xv.y, x2 = xv.z, x3 = xv.w;
 #pragma unroll
                 for (int b = 0; b < NEH; ++b) {
                     acc[a][b] = fmaf(x0, wv[b].x, acc[a][b]);
@@ -197,6 +219,9 @@ struct SmallRouteArgs {
 __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteArgs a) {
     __shared__ float red[kSmallRoute][8];
     __shared__ int last;
+    // the expert kernels that follow are launched as programmatic dependents: let them be
+    // scheduled (and stage their token rows) while this grid runs
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nq = a.H >> 2;      // float4s per row
     const float* wrow = a.wr + size_t(e) * a.H;
@@ -254,11 +279,8 @@ __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteArgs a) {
     if (tid == 0) *a.ticket = 0u;
     __syncthreads();
     if (!a.do_permute) return;
-    __shared__ int grp[kSmallRoute * (kMaxTopK + 1)];
     __shared__ int cnt[kMaxExperts + 2];
-    __shared__ int flag[kMaxExperts + 2];
-    __shared__ int tmp[33];
-    block_permute_small(sidx, a.T, a.k, a.E, a.S, grp, cnt, flag, tmp, a.perm);
+    if (warp == 0) warp_permute_small(sidx, a.T, a.k, a.E, a.S, cnt, a.perm);
 }
 
 // ------------------------------------------------------------------ host launchers
@@ -276,7 +298,7 @@ cudaError_t launch_route(int T, int H, int E, int k, int S, const uint16_t* x, c
     const int ne = (E + 31) / 32;
 #define FT_RT(NEV)                                                                                          \
     do {                                                                                                    \
-        const size_t smem = sizeof(float) * kRtStages * 32 * NEV * kRtLdW + sizeof(uint16_t) * kRtStages * kRtTok * kRtLdX; \
+        const size_t smem = sizeof(float) * (kRtStages * 32 * NEV * kRtLdW + 2 * kRtTok * kRtLdX);             \
         static bool set = false;                                                                            \
         if (!set) {                                                                                         \
             cudaError_t e = cudaFuncSetAttribute(route_tile_kernel<NEV>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)); \

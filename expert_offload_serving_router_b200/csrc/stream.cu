@@ -317,7 +317,6 @@ ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const voi
         LayerCache& c = s->cache[size_t(l)];
         // 1. route + top-k + permutation on the GPU (one launch), read the ids back: the one host wait
         const uint16_t* xcur = xl + size_t(l) * TH;
-        if ((st = cuda_ok(cudaMemsetAsync(err + 1, 0, sizeof(uint32_t), cs), "reset route ticket"))) return st;
         if ((st = cuda_ok(launch_route(T, sh.hidden, E, k, sh.num_shared, xcur, w_router[l], bias ? bias[l] : nullptr,
                                        d_idx, gw, lg, err + 1, &po, cs), "route launch")))
             return st;
