@@ -58,11 +58,12 @@ def recorded_traffic(summary: str, source: str):
     src = os.path.join(ROOT, "expert_offload_serving_router_b200", "csrc", source)
     if not os.path.exists(p) or not os.path.exists(src):
         return None
+    import re
     fields = {}
     for line in open(p):
-        if ":" in line and line.strip().startswith(("dram_bytes_per_launch", "kernel_source_sha1")):
-            k_, v_ = line.split(":", 1)
-            fields[k_.strip()] = v_.strip().strip("`")
+        m = re.match(r"\s*-?\s*(dram_bytes_per_launch|kernel_source_sha1):\s*`?([0-9a-fA-F.]+)`?", line)
+        if m:
+            fields[m.group(1)] = m.group(2)
     if fields.get("kernel_source_sha1") != hashlib.sha1(open(src, "rb").read()).hexdigest():
         return None
     try:
