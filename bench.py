@@ -39,7 +39,7 @@ from expert_offload_serving_router_b200 import inputs  # noqa: E402
 WORKLOAD = "qwen3_a3b"
 PREFILL_T = 4096
 METRIC = "MoE-layer tokens/s (decode & prefill) and % of HBM / tensor-core roofline"
-LAUNCHES_PER_STEP = 1 + 3 + 1 + 1 + 1   # route, permute (count/scan/scatter), gate/up, down, combine
+LAUNCHES_PER_STEP = 3 + 3 + 1 + 1 + 1   # router (plane split, GEMM, top-k), permute (count/scan/scatter), gate/up, down, combine
 
 
 def peaks():

@@ -118,6 +118,7 @@ DecodeArgs decode_args(const ft_moe_shape* s, int T, const ft_moe_weights* w, co
     a.topk_w = topk_w;
     a.y = static_cast<uint16_t*>(y);
     a.o_sorted = static_cast<uint16_t*>(o_sorted);
+    a.err = ws_at<uint32_t>(ws, L.err);
     return a;
 }
 
@@ -175,11 +176,11 @@ size_t ft_moe_workspace_bytes(const ft_moe_shape* shape, int32_t max_tokens) {
 }
 
 ft_status ft_moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
-    if (!ws || ws_bytes < 256) return fail(FT_ERR_INVALID_ARG, "workspace NULL or smaller than 256 bytes");
+    if (!ws || ws_bytes < kWsHeaderBytes) return fail(FT_ERR_INVALID_ARG, "workspace NULL or smaller than its %zu-byte header", kWsHeaderBytes);
     if (!al(ws, 256)) return fail(FT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     ft_status st = cuda_state();
     if (st) return st;
-    return cuda_ok(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)), "cudaMemsetAsync(ws status)");
+    return cuda_ok(cudaMemsetAsync(ws, 0, kWsHeaderBytes, static_cast<cudaStream_t>(stream)), "cudaMemsetAsync(ws header)");
 }
 
 ft_status ft_moe_check(void* ws, void* stream) {
@@ -214,8 +215,8 @@ ft_status ft_moe_route(const ft_moe_shape* shape, int32_t T, const void* x, cons
     uint32_t* err = ws_at<uint32_t>(ws, L.err);   // err[1]: decode-router ticket, zero between calls
     float* lg = logits ? logits : ws_at<float>(ws, L.logits);
     return cuda_ok(launch_route(T, shape->hidden, shape->num_experts, shape->top_k, shape->num_shared,
-                                static_cast<const uint16_t*>(x), w_router, bias, topk_idx, topk_w, lg, err + 1,
-                                nullptr, st),
+                                static_cast<const uint16_t*>(x), w_router, bias, topk_idx, topk_w, lg, err,
+                                ws_at<uint16_t>(ws, L.wr_planes), ws_at<float>(ws, L.route_part), nullptr, st),
                    "route launch");
 }
 
@@ -336,12 +337,12 @@ ft_status ft_moe_layer_forward(const ft_moe_shape* shape, int32_t T, const void*
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     if (decode) {
         // route + top-k + permutation in one launch, then two weight-streaming kernels
-        if ((s = cuda_ok(launch_route(T, H, E, k, S, xb, w_router, bias, idx, gw, lg, err + 1, &po, st), "route launch")))
+        if ((s = cuda_ok(launch_route(T, H, E, k, S, xb, w_router, bias, idx, gw, lg, err, ws_at<uint16_t>(ws, L.wr_planes), ws_at<float>(ws, L.route_part), &po, st), "route launch")))
             return s;
         DecodeArgs a = decode_args(shape, T, weights, x, L, ws, offsets, sorted_flat, inv_pos, gw, y, nullptr);
         return cuda_ok(launch_decode(a, st), "decode experts launch");
     }
-    if ((s = cuda_ok(launch_route(T, H, E, k, S, xb, w_router, bias, idx, gw, lg, err + 1, nullptr, st), "route launch")))
+    if ((s = cuda_ok(launch_route(T, H, E, k, S, xb, w_router, bias, idx, gw, lg, err, ws_at<uint16_t>(ws, L.wr_planes), ws_at<float>(ws, L.route_part), nullptr, st), "route launch")))
         return s;
     uint16_t* xs = ws_at<uint16_t>(ws, L.x_sorted);
     if ((s = cuda_ok(launch_permute(T, k, E, S, H, idx, xb, xs, ws_at<int32_t>(ws, L.chunk_cnt),

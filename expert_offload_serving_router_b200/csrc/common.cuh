@@ -60,11 +60,30 @@ struct WsLayout {
     size_t logits, topk_idx, topk_w, offsets, sorted_flat, inv_pos;
     size_t chunk_cnt, chunk_base, local_rank, sched, err;
     size_t x_sorted, h, o_sorted;
+    size_t wr_planes;   // router weights as three bf16 planes (prefill-sized batches only)
+    size_t route_part;  // partial logits of the prefill router, one slab per K split
     size_t total;
     int T, P, R, G, C;
 };
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Workspace header (cleared by ft_moe_workspace_init): word 0 device error flag, word 1 the
+// decode router's ticket (every launch leaves it at zero).
+constexpr size_t kWsHeaderBytes = 256;
+constexpr int kRouteTok = 128;          // tokens per router CTA
+constexpr int kRouteTargetCtas = 148;   // split K until the router grid covers about one wave
+constexpr int kRouteMaxSplit = 8;
+
+// K splits of the prefill router for T tokens, H hidden (each split keeps >= 1 K stage of 64)
+__host__ __device__ inline int route_splits(int T, int H) {
+    const int tiles = (T + kRouteTok - 1) / kRouteTok;
+    if (tiles <= 0) return 1;
+    int ks = kRouteTargetCtas / tiles;
+    if (ks > kRouteMaxSplit) ks = kRouteMaxSplit;
+    if (ks > H / 64) ks = H / 64;
+    return ks < 1 ? 1 : ks;
+}
 
 // sched region: [0] total GEMM tiles for BN, [1] n_active groups, [2..] ntile_off[G+1], then active[G]
 inline WsLayout make_layout(const ft_moe_shape& s, int T) {
@@ -77,7 +96,7 @@ inline WsLayout make_layout(const ft_moe_shape& s, int T) {
     if (L.C < 1) L.C = 1;
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t r = o; o = align256(o + bytes); return r; };
-    L.err = take(sizeof(uint32_t) * 8);   // first: [0] device error flag, [1] route ticket
+    L.err = take(kWsHeaderBytes);   // first: [0] device error flag, [1] decode-router ticket
     L.logits = take(sizeof(float) * size_t(T) * s.num_experts);
     L.topk_idx = take(sizeof(int32_t) * size_t(L.P));
     L.topk_w = take(sizeof(float) * size_t(L.P));
@@ -91,6 +110,9 @@ inline WsLayout make_layout(const ft_moe_shape& s, int T) {
     L.x_sorted = take(sizeof(uint16_t) * size_t(L.R) * s.hidden);
     L.h = take(sizeof(uint16_t) * size_t(L.R) * s.ffn);
     L.o_sorted = take(sizeof(uint16_t) * size_t(L.R) * s.hidden);
+    L.wr_planes = take(T > kSmallRoute ? size_t(3) * size_t((s.num_experts + 15) & ~15) * s.hidden * 2 : 0);
+    L.route_part = take(T > kSmallRoute ? size_t(route_splits(T, s.hidden)) * ((T + kRouteTok - 1) / kRouteTok) *
+                                              kRouteTok * ((s.num_experts + 15) & ~15) * sizeof(float) : 0);
     L.total = o;
     return L;
 }

@@ -25,6 +25,7 @@ struct DecodeArgs {
     const float* topk_w;
     uint16_t* y;                // [T, H] or NULL
     uint16_t* o_sorted;         // [R, H] when y == NULL
+    uint32_t* err;              // workspace device error flag
 };
 
 struct GemmLaunch {
@@ -54,9 +55,15 @@ DecodeArgs decode_args(const ft_moe_shape* s, int T, const ft_moe_weights* w, co
                        void* ws, const int32_t* offsets, const int32_t* sorted_flat, const int32_t* inv_pos,
                        const float* topk_w, void* y, void* o_sorted);
 
+// err: the workspace's device error word ([0] flag, [1] decode-router ticket); planes: the
+// workspace's router-plane region and part its split-K partials (used when T > kSmallRoute).  `perm` (fused counting
+// sort) is only taken by the decode-sized path.
 cudaError_t launch_route(int T, int H, int E, int k, int S, const uint16_t* x, const float* wr, const float* bias,
-                         int32_t* topk_idx, float* topk_w, float* logits, uint32_t* ticket, const PermOut* perm,
-                         cudaStream_t st);
+                         int32_t* topk_idx, float* topk_w, float* logits, uint32_t* err, uint16_t* planes,
+                         float* part, const PermOut* perm, cudaStream_t st);
+cudaError_t launch_route_tc(int T, int H, int E, int k, const uint16_t* x, const float* wr, const float* bias,
+                            int32_t* topk_idx, float* topk_w, float* logits, uint16_t* planes, float* part,
+                            uint32_t* err, cudaStream_t st);
 cudaError_t launch_permute(int T, int k, int E, int S, int H, const int32_t* idx, const uint16_t* x,
                            uint16_t* x_sorted, int32_t* chunk_cnt, int32_t* chunk_base, int32_t* local_rank,
                            const PermOut& out, cudaStream_t st);

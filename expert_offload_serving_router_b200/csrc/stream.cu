@@ -318,7 +318,7 @@ ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const voi
         // 1. route + top-k + permutation on the GPU (one launch), read the ids back: the one host wait
         const uint16_t* xcur = xl + size_t(l) * TH;
         if ((st = cuda_ok(launch_route(T, sh.hidden, E, k, sh.num_shared, xcur, w_router[l], bias ? bias[l] : nullptr,
-                                       d_idx, gw, lg, err + 1, &po, cs), "route launch")))
+                                       d_idx, gw, lg, err, ws_at<uint16_t>(ws, Lw.wr_planes), ws_at<float>(ws, Lw.route_part), &po, cs), "route launch")))
             return st;
         if ((st = cuda_ok(cudaMemcpyAsync(s->hids, d_idx, sizeof(int32_t) * T * k, cudaMemcpyDeviceToHost, cs), "ids D2H")))
             return st;

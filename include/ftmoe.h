@@ -127,9 +127,9 @@ int32_t ft_get_decode_max_tokens(void);
 size_t ft_moe_workspace_bytes(const ft_moe_shape* shape, int32_t max_tokens);
 
 /* Clears the device status words at the start of a freshly allocated
- * workspace (ws: device, >= 256 bytes): the error flag and the decode
- * router's last-CTA ticket, which every call leaves at zero again.  Call once
- * per workspace before its first use; enqueued on `stream`. */
+ * workspace (ws: device, 256-byte aligned, >= 256 bytes): the error flag and
+ * the decode router's last-CTA ticket, which every call leaves at zero again.
+ * Call once per workspace before its first use; enqueued on `stream`. */
 ft_status ft_moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status word of ws.

@@ -24,8 +24,10 @@ def _route(cfg, x, w_r, bias):
     return host(idx, np.int32), host(gw, np.float32), host(lg, np.float32)
 
 
+# T <= 32: decode router; 32 < T: tensor-core router, split K across CTAs while the grid is
+# under one wave (T = 9700: 76 token tiles, no split), ragged last tile everywhere
 @pytest.mark.parametrize("E,k,T", [(8, 2, 1), (8, 2, 64), (8, 8, 40), (128, 8, 16), (128, 8, 100), (256, 6, 8),
-                                   (256, 6, 333), (96, 3, 50)])
+                                   (256, 6, 333), (96, 3, 50), (8, 2, 9700), (40, 4, 2000)])
 def test_route_matches_oracle_with_ties(E, k, T):
     from gpu_util import logits_bound
     cfg = inputs.custom_config(hidden=512, ffn=64, num_experts=E, top_k=k, config_id=60)
