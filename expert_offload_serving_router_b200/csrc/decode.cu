@@ -15,6 +15,7 @@
 // fma.rn.f32.f16 against f16 activations, then scaled once by the block's E8M0 scale.
 // The f16 activation copy is exact for 2^-17 <= |v| <= 65504 (bf16 has 8 significant bits).
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace ftmoe {
 
@@ -246,6 +247,7 @@ __global__ void __launch_bounds__(256) decode_down_kernel(DecodeArgs a) {
     constexpr int RB = (MX ? 16 : 24) / CPL >= 8 ? 8 : (MX ? 16 : 24) / CPL >= 4 ? 4 : (MX ? 16 : 24) / CPL >= 2 ? 2 : 1;
     constexpr int NB = kRPB / RB;               // row batches per active group
     __shared__ float prod[kMaxDecodeRows][kRPB + 1];
+    pdl_trigger();   // the next layer's router may launch; it waits for this grid before writing
     pdl_wait();
     const int G = a.E + (a.S ? 1 : 0);
     const int n_active = a.sched[1];
@@ -353,6 +355,135 @@ __global__ void __launch_bounds__(256) decode_down_kernel(DecodeArgs a) {
     }
 }
 
+// Single-pass variant for small batches: all routed experts' RPB rows of W2 fit in shared
+// memory together, so each CTA issues every weight copy (one bulk async copy per expert, plus
+// one for its MXFP4 scales) before the programmatic dependency wait -- the routing was final
+// before the gate/up kernel started, only h comes from it -- and the weights stream while
+// the gate/up kernel finishes.  Warp items are (expert, 4 rows), dot products from shared
+// memory, then the same products tile and combine as above.
+struct DownBulkCfg { int RPB, chunk, nbuf, R; };
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(su32(dst)), "l"(src), "r"(bytes), "r"(su32(bar)) : "memory");
+}
+
+template <bool MX>
+__global__ void __launch_bounds__(256, 2) decode_down_bulk_kernel(DecodeArgs a, DownBulkCfg c) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    const int RPB = c.RPB;
+    float* prod = reinterpret_cast<float*>(dsm);                                   // [R][RPB + 1]
+    uint8_t* wbuf = dsm + ((size_t(c.R) * (RPB + 1) * 4 + 127) & ~size_t(127));    // [nbuf][chunk]
+    uint64_t* full = reinterpret_cast<uint64_t*>(wbuf + size_t(c.nbuf) * c.chunk);
+    __shared__ int s_g[kMaxExperts + 1];
+    __shared__ int s_bad;
+    pdl_trigger();   // the next layer's router may launch; it waits for this grid before writing
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = a.H, F = a.F;
+    const int G = a.E + (a.S ? 1 : 0);
+    const int hbase = blockIdx.x * RPB;
+    const size_t wrow = MX ? size_t(F) / 2 : size_t(F) * 2;      // weight bytes per row
+    const size_t srow = MX ? size_t(F) / 32 : 0;                 // scale bytes per row
+    const int n_active = __ldcg(a.sched + 1);
+    for (int i = tid; i < n_active; i += blockDim.x) s_g[i] = __ldcg(a.sched + 2 + (G + 1) + i);
+    if (tid == 0) {
+        s_bad = n_active > c.nbuf;   // more experts than buffers: the host sizing was wrong
+        for (int i = 0; i < c.nbuf; ++i) mbar_init(&full[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (s_bad) {
+        if (tid == 0) atomicExch(a.err, kDevErrShape);
+        pdl_wait();
+        return;
+    }
+    if (tid == 0) {
+        for (int i = 0; i < n_active; ++i) {
+            const EW w = expert_w(a, s_g[i]);
+            uint8_t* dst = wbuf + size_t(i) * c.chunk;
+            const uint32_t wb = uint32_t(RPB * wrow), sb = uint32_t(RPB * srow);
+            mbar_expect_tx(&full[i], wb + sb);
+            bulk_g2s(dst, w.w2 + size_t(hbase) * wrow, wb, &full[i]);
+            if (MX) bulk_g2s(dst + wb, w.w2s + size_t(hbase) * srow, sb, &full[i]);
+        }
+    }
+    pdl_wait();   // h from the gate/up kernel
+    const int gpr = RPB / 4;
+    const int nvec = MX ? F / 32 : F / 8;       // 16-byte weight vectors per row
+    for (int it = warp; it < n_active * gpr; it += 8) {
+        const int slot = it / gpr, j0 = 4 * (it - slot * gpr);
+        if (!mbar_wait(&full[slot], 0, nullptr)) { s_bad = 1; continue; }
+        const int g = s_g[slot];
+        const int r0 = a.offsets[g], n = a.offsets[g + 1] - r0;
+        const uint8_t* wb = wbuf + size_t(slot) * c.chunk;
+        for (int r = 0; r < n; ++r) {
+            const uint4* hr = reinterpret_cast<const uint4*>(a.h + size_t(r0 + r) * F);
+            float v[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int q = lane; q < nvec; q += 32) {
+                if (!MX) {
+                    const uint4 hv = __ldg(hr + q);
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) {
+                        const uint4 wv = *reinterpret_cast<const uint4*>(wb + size_t(j0 + rr) * wrow + size_t(q) * 16);
+                        fma2_bf16(v[rr], wv.x, hv.x); fma2_bf16(v[rr], wv.y, hv.y);
+                        fma2_bf16(v[rr], wv.z, hv.z); fma2_bf16(v[rr], wv.w, hv.w);
+                    }
+                } else {
+                    uint4 xv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint4 hv = __ldg(hr + 4 * q + u);
+                        xv[u] = make_uint4(f32x2_to_f16x2(bf16lo(hv.x), bf16hi(hv.x)), f32x2_to_f16x2(bf16lo(hv.y), bf16hi(hv.y)),
+                                           f32x2_to_f16x2(bf16lo(hv.z), bf16hi(hv.z)), f32x2_to_f16x2(bf16lo(hv.w), bf16hi(hv.w)));
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) {
+                        const uint4 wv = *reinterpret_cast<const uint4*>(wb + size_t(j0 + rr) * wrow + size_t(q) * 16);
+                        const uint32_t sc = wb[size_t(RPB) * wrow + size_t(j0 + rr) * srow + q];
+                        v[rr] = fmaf(mx_block_dot(wv, xv), e8m0f(sc), v[rr]);
+                    }
+                }
+            }
+            tr_step(v, 4, 16, lane);
+            tr_step(v, 2, 8, lane);
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], 4);
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+            if ((lane & 7) == 0) {   // lane l holds row 2*bit4(l) + bit3(l)
+                const int sel = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+                prod[size_t(r0 + r) * (RPB + 1) + j0 + sel] = v[0];
+            }
+        }
+    }
+    __syncthreads();
+    if (s_bad) {
+        if (tid == 0) {
+            atomicExch(a.err, kDevErrTimeout);
+            for (int i = 0; i < n_active; ++i) mbar_wait(&full[i], 0, nullptr);   // let copies land
+        }
+        return;
+    }
+    const int P = a.T * a.k;
+    if (a.y) {
+        for (int q = tid; q < a.T * RPB; q += blockDim.x) {
+            const int t = q / RPB, j = q - t * RPB;
+            float acc = 0.f;
+            for (int jj = 0; jj < a.k; ++jj) {
+                const int pos = a.inv_pos[t * a.k + jj];
+                acc = fmaf(a.topk_w[t * a.k + jj], prod[size_t(pos) * (RPB + 1) + j], acc);
+            }
+            if (a.S) acc += prod[size_t(a.inv_pos[P + t]) * (RPB + 1) + j];
+            a.y[size_t(t) * H + hbase + j] = f2bf(acc);
+        }
+    } else {
+        const int R = a.offsets[G];
+        for (int q = tid; q < R * RPB; q += blockDim.x) {
+            const int r = q / RPB, j = q - r * RPB;
+            a.o_sorted[size_t(r) * H + hbase + j] = f2bf(prod[size_t(r) * (RPB + 1) + j]);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ host launch
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
@@ -415,6 +546,32 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
 #undef FT_GU2
 #undef FT_GU
     if (e != cudaSuccess) return e;
+    // down: the single-pass bulk-copy kernel when every routed expert's row block fits in
+    // shared memory at two CTAs per SM, else the register-streaming kernel
+    {
+        constexpr size_t kBulkSmem = 110 * 1024;
+        const size_t wrow = mx ? size_t(a.F) / 2 + size_t(a.F) / 32 : size_t(a.F) * 2;
+        auto need = [&](int rpb) {
+            return ((size_t(R) * (rpb + 1) * 4 + 127) & ~size_t(127)) + size_t(na_max) * (size_t(rpb) * wrow + 8);
+        };
+        int rpb = 0;
+        if (a.H % 16 == 0 && a.H / 8 > 2 * sms && need(16) <= kBulkSmem) rpb = 16;
+        else if (need(8) <= kBulkSmem) rpb = 8;
+        if (rpb && R <= kMaxDecodeRows) {
+            DownBulkCfg c{rpb, int(size_t(rpb) * wrow), na_max, R};
+            const size_t dsm = need(rpb);
+            static bool attr[2] = {false, false};
+            auto kern = mx ? decode_down_bulk_kernel<true> : decode_down_bulk_kernel<false>;
+            if (!attr[mx]) {
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kBulkSmem));
+                if (e != cudaSuccess) return e;
+                attr[mx] = true;
+            }
+            e = launch_pdl(kern, dim3(a.H / rpb), dim3(256), dsm, st, a, c);
+            if (e != cudaSuccess) return e;
+            return cudaGetLastError();
+        }
+    }
     dim3 g2((a.H + kRPB - 1) / kRPB);
     const int vec = mx ? a.F / 32 : a.F / 8;          // vectors per weight row
     const int cpl = (vec + 31) / 32;

@@ -31,9 +31,6 @@ struct SmallRouteArgs {
 __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteArgs a) {
     __shared__ float red[kSmallRoute][8];
     __shared__ int last;
-    // the expert kernels that follow are launched as programmatic dependents: let them be
-    // scheduled (and stage their token rows) while this grid runs
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nq = a.H >> 2;      // float4s per row
     const float* wrow = a.wr + size_t(e) * a.H;
@@ -45,6 +42,13 @@ __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteArgs a) {
         for (int i = 0; i < 4; ++i) {
             int q = base + tid + 256 * i;
             w[i] = q < nq ? __ldg(reinterpret_cast<const float4*>(wrow) + q) : make_float4(0, 0, 0, 0);
+        }
+        // weights do not depend on the preceding kernel: wait for it only before reading x.
+        // Only then let the expert kernels that follow (programmatic dependents) be scheduled:
+        // they stage x before their own wait, so x must be final by the time they start.
+        if (base == 0) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         }
         for (int t = 0; t < a.T; ++t) {
             const uint2* xr = reinterpret_cast<const uint2*>(a.x + size_t(t) * a.H);
@@ -103,8 +107,18 @@ cudaError_t launch_route(int T, int H, int E, int k, int S, const uint16_t* x, c
     if (T <= kSmallRoute) {
         SmallRouteArgs a{T, H, E, k, S, x, wr, bias, topk_idx, topk_w, logits, err + 1, perm != nullptr, {}};
         if (perm) a.perm = *perm;
-        route_small_kernel<<<E, 256, 0, st>>>(a);
-        return cudaGetLastError();
+        // programmatic dependent launch: the router rows stream while the preceding kernel
+        // (the previous layer's down GEMV) finishes
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(E);
+        cfg.blockDim = dim3(256);
+        cfg.stream = st;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, route_small_kernel, a);
     }
     if (perm) return cudaErrorInvalidValue;   // the fused permutation exists only for decode-sized batches
     return launch_route_tc(T, H, E, k, x, wr, bias, topk_idx, topk_w, logits, planes, part, err, st);

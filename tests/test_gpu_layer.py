@@ -153,3 +153,35 @@ def test_deterministic_and_stepwise_equals_fused():
 def test_empty_batch_is_a_noop():
     L = layer("tiny")
     F.ft_moe_layer_forward(L.shape, 0, None, None, None, L.weights, None, None, None, None, 0)
+
+
+@pytest.mark.parametrize("name,T", [("qwen3_a3b", 1), ("dsv4_flash", 1), ("gemma4_26b_a4b", 1), ("qwen3_a3b", 4),
+                                    ("tiny", 64)])
+def test_chained_layers_without_host_sync(name, T):
+    """Layer calls back to back on one stream, each consuming the previous output: the
+    dependent-launch overlap between calls must never let a kernel read an input before the
+    kernel producing it has finished.  Equal bit for bit to the same chain run one call at a
+    time with a synchronisation in between."""
+    import torch
+    from gpu_util import dev, host, run_layer, workspace
+    L = layer(name)
+    H, E, k = L.cfg.hidden, L.cfg.num_experts, L.cfg.top_k
+    steps = 6
+    x0 = inputs.make_tokens(L.cfg, T, seed=11)
+    # reference: one call at a time
+    ref = []
+    x = x0
+    for _ in range(steps):
+        y, _, _ = run_layer(L, x)
+        ref.append(y)
+        x = y
+    # chained: no synchronisation between the calls
+    ws = workspace(L.shape, T)
+    bufs = [dev(x0)] + [torch.empty((T, H), dtype=torch.int16, device="cuda") for _ in range(steps)]
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    for s in range(steps):
+        F.ft_moe_layer_forward(L.shape, T, bufs[s], L.t["w_router"], L.t.get("bias"), L.weights, bufs[s + 1], idx,
+                               None, ws)
+    F.ft_moe_check(ws)
+    for s in range(steps):
+        assert np.array_equal(host(bufs[s + 1], np.uint16), ref[s]), f"step {s} differs"
