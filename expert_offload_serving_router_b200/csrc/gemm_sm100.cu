@@ -208,9 +208,9 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
                         for (int h = 0; h < tl.halves; ++h) {
                             const int rg = tl.m * HV + h;       // 128-row weight group index
                             if (p.mode == 0) {
-#pragma unroll
-                                for (int i = 0; i < 4; ++i)
-                                    tma_4d(m, &full[stage], a + h * kAHalfBytes + i * 4096, k0, rg * 64 + 16 * i, 0, e);
+                                // (k, row-in-block, gate|up, 16-row block, expert): 4 blocks of 16
+                                // gate + 16 up rows land interleaved, one copy per half
+                                tma_5d(m, &full[stage], a + h * kAHalfBytes, k0, 0, 0, rg * 4, e);
                             } else {
                                 tma_3d(m, &full[stage], a + h * kAHalfBytes, k0, rg * 128, e);
                             }
@@ -462,13 +462,17 @@ int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
     }
     if (!mx) {
         if (L.mode == 0) {
-            uint64_t dims[4] = {uint64_t(L.H), uint64_t(L.F), 2, uint64_t(L.E)};
-            uint64_t str[3] = {uint64_t(L.H) * 2, uint64_t(L.F) * L.H * 2, uint64_t(2) * L.F * L.H * 2};
-            uint32_t box[4] = {kBK, 16, 2, 1};
-            if (!make_map(&tw, L.w, 4, dims, str, box)) return 1;
+            // w13 [E][2][F][H] viewed as (H, 16, 2, F/16, E): a (64, 16, 2, 4, 1) box is 4 blocks
+            // of 16 gate rows each followed by the 16 matching up rows (one copy per 128 rows;
+            // four 4-D copies per half measured 4-5 % slower)
+            uint64_t dims[5] = {uint64_t(L.H), 16, 2, uint64_t(L.F / 16), uint64_t(L.E)};
+            uint64_t str[4] = {uint64_t(L.H) * 2, uint64_t(L.F) * L.H * 2, uint64_t(16) * L.H * 2,
+                               uint64_t(2) * L.F * L.H * 2};
+            uint32_t box[5] = {kBK, 16, 2, 4, 1};
+            if (!make_map(&tw, L.w, 5, dims, str, box)) return 1;
             if (L.S) {
-                uint64_t d1[4] = {uint64_t(L.H), uint64_t(L.F), 2, 1};
-                if (!make_map(&tsw, L.sw, 4, d1, str, box)) return 1;
+                uint64_t d1[5] = {uint64_t(L.H), 16, 2, uint64_t(L.F / 16), 1};
+                if (!make_map(&tsw, L.sw, 5, d1, str, box)) return 1;
             } else {
                 tsw = tw;
             }

@@ -22,7 +22,7 @@ static EncodeTiledFn get_encode() {
 }
 
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank, const uint64_t* dims,
-              const uint64_t* strides, const uint32_t* box) {
+              const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw) {
     EncodeTiledFn enc = get_encode();
     if (!enc || rank < 1 || rank > 5) return false;
     cuuint64_t d[5], s[4];
@@ -30,7 +30,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank
     for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; es[i] = 1; }
     for (int i = 0; i < rank - 1; ++i) s[i] = strides[i];
     CUresult r = enc(m, dt, cuuint32_t(rank), const_cast<void*>(base), d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
