@@ -14,232 +14,31 @@
 // are decoded with cvt.rn.f16x2.e2m1x2 (exact) and accumulated per 32-element block with
 // fma.rn.f32.f16 against f16 activations, then scaled once by the block's E8M0 scale.
 // The f16 activation copy is exact for 2^-17 <= |v| <= 65504 (bf16 has 8 significant bits).
-#include "kernels.h"
-#include "sm100.cuh"
+#include "decode_common.cuh"
 
 namespace ftmoe {
 
 
 
-struct EW { const uint8_t *w13, *w13s, *w2, *w2s; };
-
-// Programmatic dependent launch: a kernel launched with the programmatic-serialization
-// attribute may start while its predecessor finishes; griddepcontrol.wait blocks until the
-// predecessor grid has completed and its memory is visible (a no-op for plain launches).
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-__device__ __forceinline__ EW expert_w(const DecodeArgs& a, int g) {
-    EW r;
-    if (g >= a.E) { r.w13 = a.sw13; r.w13s = a.sw13s; r.w2 = a.sw2; r.w2s = a.sw2s; return r; }
-    if (a.eptr) {
-        r.w13 = static_cast<const uint8_t*>(a.eptr[4 * g + 0]);
-        r.w13s = static_cast<const uint8_t*>(a.eptr[4 * g + 1]);
-        r.w2 = static_cast<const uint8_t*>(a.eptr[4 * g + 2]);
-        r.w2s = static_cast<const uint8_t*>(a.eptr[4 * g + 3]);
-        return r;
-    }
-    const size_t HF = size_t(a.H) * a.F;
-    if (a.wdtype == FT_W_BF16) {
-        r.w13 = a.w13 + size_t(g) * 2 * HF * 2;
-        r.w2 = a.w2 + size_t(g) * HF * 2;
-        r.w13s = r.w2s = nullptr;
-    } else {
-        r.w13 = a.w13 + size_t(g) * 2 * HF / 2;
-        r.w13s = a.w13s + size_t(g) * 2 * HF / 32;
-        r.w2 = a.w2 + size_t(g) * HF / 2;
-        r.w2s = a.w2s + size_t(g) * HF / 32;
-    }
-    return r;
-}
-
-// acc += (w.lo * x.lo) + (w.hi * x.hi), exact products, fp32 accumulate
-__device__ __forceinline__ void fma2_bf16(float& acc, uint32_t w, uint32_t x) {
-    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\tmov.b32 {wl, wh}, %1;\n\tmov.b32 {xl, xh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\tfma.rn.f32.bf16 %0, wh, xh, %0;\n\t}"
-        : "+f"(acc) : "r"(w), "r"(x));
-}
-__device__ __forceinline__ void fma2_f16(float& acc, uint32_t w, uint32_t x) {
-    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\tmov.b32 {wl, wh}, %1;\n\tmov.b32 {xl, xh}, %2;\n\t"
-        "fma.rn.f32.f16 %0, wl, xl, %0;\n\tfma.rn.f32.f16 %0, wh, xh, %0;\n\t}"
-        : "+f"(acc) : "r"(w), "r"(x));
-}
-// two E2M1 codes (one byte) -> f16x2 (low nibble in the low half), exact
-__device__ __forceinline__ uint32_t e2m1x2_f16x2(uint32_t byte) {
-    uint32_t r;
-    asm("{\n\t.reg .b8 t;\n\t.reg .b16 s;\n\tcvt.u16.u32 s, %1;\n\tcvt.u8.u16 t, s;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
-        : "=r"(r) : "r"(byte));
-    return r;
-}
-__device__ __forceinline__ float e8m0f(uint32_t s) { return s == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(s << 23); }
-__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
-    __half2 h = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// dot of one 32-element MXFP4 block (16 code bytes) with 32 f16 activations (4 x uint4)
-__device__ __forceinline__ float mx_block_dot(const uint4& c, const uint4* xv) {
-    float a0 = 0.f, a1 = 0.f;
-    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {            // 4 code bytes per word -> 8 elements
-        const uint4 xx = xv[q];
-        const uint32_t xw[4] = {xx.x, xx.y, xx.z, xx.w};
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            uint32_t wf = e2m1x2_f16x2((cw[q] >> (8 * b)) & 0xFFu);
-            if (b & 1) fma2_f16(a1, wf, xw[b]); else fma2_f16(a0, wf, xw[b]);
-        }
-    }
-    return a0 + a1;
-}
-
 // ------------------------------------------------------------------ gate/up + SwiGLU
-constexpr int kFPB = 8;       // f values per CTA (one per warp)
-
 template <int TB, bool MX, bool FULLX>
 __global__ void __launch_bounds__(256) decode_gateup_kernel(DecodeArgs a) {
     // FULLX: every token row [T][H] staged once (bf16, or f16 for MXFP4) before the
     // programmatic dependency wait -- the layer input is complete before the router ran --
     // so the routing-dependent part starts straight with the weight stream.
-    // Otherwise: the group's rows are staged per batch of TB after the wait.
     extern __shared__ uint4 xs4[];
     __shared__ int stok[TB];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int H = a.H, F = a.F;
-    const int nv = H / 8;                            // 16-byte activation vectors per row
-    auto stage_row = [&](int t, int dst_row) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.x + size_t(t) * H);
-        uint4* dst = xs4 + size_t(dst_row) * nv;
-        for (int v = lane; v < nv; v += 32) {
-            uint4 u = __ldg(src + v);
-            if (MX) {
-                u = make_uint4(f32x2_to_f16x2(bf16lo(u.x), bf16hi(u.x)), f32x2_to_f16x2(bf16lo(u.y), bf16hi(u.y)),
-                               f32x2_to_f16x2(bf16lo(u.z), bf16hi(u.z)), f32x2_to_f16x2(bf16lo(u.w), bf16hi(u.w)));
-            }
-            dst[v] = u;
-        }
-    };
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (FULLX)
-        for (int t = warp; t < a.T; t += 8) stage_row(t, t);
+        for (int t = warp; t < a.T; t += 8) stage_x_row<MX>(a, xs4, t, t, lane);
     pdl_wait();
     pdl_trigger();
-    const int G = a.E + (a.S ? 1 : 0);
-    const int P = a.T * a.k;
-    const int nfb = (F + kFPB - 1) / kFPB;
-    const int n_active = a.sched[1];
-    // grid-stride over (active group, f-block) items; f-block fastest so a CTA's items
-    // mostly share their group (and its staged rows)
-    for (int item = blockIdx.x; item < n_active * nfb; item += gridDim.x) {
-    const int slot = item / nfb, fblk = item - slot * nfb;
-    const int g = a.sched[2 + (G + 1) + slot];
-    const int r0 = a.offsets[g];
-    const int n = a.offsets[g + 1] - r0;
-    const EW w = expert_w(a, g);
-    for (int tb = 0; tb < n; tb += TB) {
-        const int nb = min(TB, n - tb);
-        __syncthreads();
-        if (FULLX) {
-            if (tid < nb) {
-                const int p = a.sorted_flat[r0 + tb + tid];
-                stok[tid] = p < P ? p / a.k : p - P;
-            }
-        } else {
-            for (int i = warp; i < nb; i += 8) {
-                const int p = a.sorted_flat[r0 + tb + i];
-                stage_row(p < P ? p / a.k : p - P, i);
-            }
-            if (tid < nb) stok[tid] = tid;
-        }
-        __syncthreads();
-        for (int fi = 0; fi < kFPB / 8; ++fi) {
-            const int f = fblk * kFPB + warp * (kFPB / 8) + fi;
-            if (f >= F) break;
-            float ag[TB], au[TB];
-#pragma unroll
-            for (int i = 0; i < TB; ++i) { ag[i] = 0.f; au[i] = 0.f; }
-            if (!MX) {
-                const uint4* gr = reinterpret_cast<const uint4*>(w.w13 + size_t(f) * H * 2);
-                const uint4* ur = reinterpret_cast<const uint4*>(w.w13 + size_t(F + f) * H * 2);
-                for (int c0 = lane; c0 < nv; c0 += 32 * 8) {
-                    uint4 wg[8], wu[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        int c = c0 + 32 * u;
-                        if (c < nv) { wg[u] = ldg_nc_v4(gr + c); wu[u] = ldg_nc_v4(ur + c); }
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        int c = c0 + 32 * u;
-                        if (c >= nv) break;
-#pragma unroll
-                        for (int i = 0; i < TB; ++i) {
-                            if (i >= nb) break;
-                            uint4 xv = xs4[size_t(stok[i]) * nv + c];
-                            fma2_bf16(ag[i], wg[u].x, xv.x); fma2_bf16(ag[i], wg[u].y, xv.y);
-                            fma2_bf16(ag[i], wg[u].z, xv.z); fma2_bf16(ag[i], wg[u].w, xv.w);
-                            fma2_bf16(au[i], wu[u].x, xv.x); fma2_bf16(au[i], wu[u].y, xv.y);
-                            fma2_bf16(au[i], wu[u].z, xv.z); fma2_bf16(au[i], wu[u].w, xv.w);
-                        }
-                    }
-                }
-            } else {
-                const int nblk = H / 32;
-                const uint4* gq = reinterpret_cast<const uint4*>(w.w13 + size_t(f) * (H / 2));
-                const uint4* uq = reinterpret_cast<const uint4*>(w.w13 + size_t(F + f) * (H / 2));
-                const uint8_t* gs = w.w13s + size_t(f) * nblk;
-                const uint8_t* us = w.w13s + size_t(F + f) * nblk;
-                for (int b0 = lane; b0 < nblk; b0 += 32 * 4) {
-                    uint4 cg[4], cu[4];
-                    uint32_t sg[4], su[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        int b = b0 + 32 * u;
-                        if (b < nblk) { cg[u] = ldg_nc_v4(gq + b); cu[u] = ldg_nc_v4(uq + b); sg[u] = gs[b]; su[u] = us[b]; }
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        int b = b0 + 32 * u;
-                        if (b >= nblk) break;
-                        const float scg = e8m0f(sg[u]), scu = e8m0f(su[u]);
-#pragma unroll
-                        for (int i = 0; i < TB; ++i) {
-                            if (i >= nb) break;
-                            const uint4* xv = xs4 + size_t(stok[i]) * nv + b * 4;
-                            ag[i] = fmaf(mx_block_dot(cg[u], xv), scg, ag[i]);
-                            au[i] = fmaf(mx_block_dot(cu[u], xv), scu, au[i]);
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < TB; ++i) {
-                if (i >= nb) break;
-                float gs_ = warp_sum(ag[i]);
-                float us_ = warp_sum(au[i]);
-                if (lane == 0) a.h[size_t(r0 + tb + i) * F + f] = f2bf(silu_mul(gs_, us_));
-            }
-        }
-    }
-    }
+    gateup_items<TB, MX, FULLX>(a, xs4, stok, blockIdx.x, gridDim.x);
 }
 
 // ------------------------------------------------------------------ down + combine
 constexpr int kRPB = 8;       // hidden rows per CTA
 constexpr int kMaxDecodeRows = 32 * (kMaxTopK + 1);
-
-// Transpose-reduce step: n per-lane values -> n/2, pairing lanes across `off`; lanes with
-// (lane & off) keep the upper half.  After log2(n) steps plus plain butterfly steps each
-// lane holds one complete warp sum (n-1 + 5 - log2 n shuffles instead of 5 n).
-__device__ __forceinline__ void tr_step(float* v, int n, int off, int lane) {
-    const bool up = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < n / 2; ++i) {
-        const float send = up ? v[i] : v[i + n / 2];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, off);
-        v[i] = (up ? v[i + n / 2] : v[i]) + recv;
-    }
-}
 
 template <bool MX, int CPL>
 __global__ void __launch_bounds__(256) decode_down_kernel(DecodeArgs a) {
@@ -363,11 +162,6 @@ __global__ void __launch_bounds__(256) decode_down_kernel(DecodeArgs a) {
 // memory, then the same products tile and combine as above.
 struct DownBulkCfg { int RPB, chunk, nbuf, R; };
 
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(su32(dst)), "l"(src), "r"(bytes), "r"(su32(bar)) : "memory");
-}
-
 template <bool MX>
 __global__ void __launch_bounds__(256, 2) decode_down_bulk_kernel(DecodeArgs a, DownBulkCfg c) {
     extern __shared__ __align__(128) uint8_t dsm[];
@@ -416,44 +210,7 @@ __global__ void __launch_bounds__(256, 2) decode_down_bulk_kernel(DecodeArgs a, 
         const int g = s_g[slot];
         const int r0 = a.offsets[g], n = a.offsets[g + 1] - r0;
         const uint8_t* wb = wbuf + size_t(slot) * c.chunk;
-        for (int r = 0; r < n; ++r) {
-            const uint4* hr = reinterpret_cast<const uint4*>(a.h + size_t(r0 + r) * F);
-            float v[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int q = lane; q < nvec; q += 32) {
-                if (!MX) {
-                    const uint4 hv = __ldg(hr + q);
-#pragma unroll
-                    for (int rr = 0; rr < 4; ++rr) {
-                        const uint4 wv = *reinterpret_cast<const uint4*>(wb + size_t(j0 + rr) * wrow + size_t(q) * 16);
-                        fma2_bf16(v[rr], wv.x, hv.x); fma2_bf16(v[rr], wv.y, hv.y);
-                        fma2_bf16(v[rr], wv.z, hv.z); fma2_bf16(v[rr], wv.w, hv.w);
-                    }
-                } else {
-                    uint4 xv[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint4 hv = __ldg(hr + 4 * q + u);
-                        xv[u] = make_uint4(f32x2_to_f16x2(bf16lo(hv.x), bf16hi(hv.x)), f32x2_to_f16x2(bf16lo(hv.y), bf16hi(hv.y)),
-                                           f32x2_to_f16x2(bf16lo(hv.z), bf16hi(hv.z)), f32x2_to_f16x2(bf16lo(hv.w), bf16hi(hv.w)));
-                    }
-#pragma unroll
-                    for (int rr = 0; rr < 4; ++rr) {
-                        const uint4 wv = *reinterpret_cast<const uint4*>(wb + size_t(j0 + rr) * wrow + size_t(q) * 16);
-                        const uint32_t sc = wb[size_t(RPB) * wrow + size_t(j0 + rr) * srow + q];
-                        v[rr] = fmaf(mx_block_dot(wv, xv), e8m0f(sc), v[rr]);
-                    }
-                }
-            }
-            tr_step(v, 4, 16, lane);
-            tr_step(v, 2, 8, lane);
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], 4);
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-            if ((lane & 7) == 0) {   // lane l holds row 2*bit4(l) + bit3(l)
-                const int sel = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-                prod[size_t(r0 + r) * (RPB + 1) + j0 + sel] = v[0];
-            }
-        }
+        down_item4<MX, false>(a, wb, wb + size_t(RPB) * wrow, RPB, j0, r0, n, prod, lane);
     }
     __syncthreads();
     if (s_bad) {
