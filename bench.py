@@ -38,6 +38,7 @@ from expert_offload_serving_router_b200 import inputs  # noqa: E402
 
 WORKLOAD = "qwen3_a3b"
 PREFILL_T = 4096
+PREFILL_SIZES = {"qwen3_a3b": 4096, "dsv4_flash": 8192, "gemma4_26b_a4b": 2048, "tiny": 64}
 METRIC = "MoE-layer tokens/s (decode & prefill) and % of HBM / tensor-core roofline"
 LAUNCHES_PER_STEP = 3 + 3 + 1 + 1 + 1   # router (plane split, GEMM, top-k), permute (count/scan/scatter), gate/up, down, combine
 
@@ -505,6 +506,8 @@ def main():
     ap.add_argument("--decode-tokens", default="1,4,16", help="decode batch sizes to time (comma list)")
     ap.add_argument("--decode-only", default=None, metavar="CONFIG",
                     help="time only decode batches of this layer shape (for profiling)")
+    ap.add_argument("--prefill-only", default=None, metavar="CONFIG",
+                    help="time only prefill steps of this layer shape at its prefill size (for profiling)")
     ap.add_argument("--extra", action="store_true", help="also measure the other layer shapes")
     ap.add_argument("--stack", action="store_true", help="also measure the expert-offload stack")
     args = ap.parse_args()
@@ -539,6 +542,16 @@ def main():
             print(json.dumps({"mode": "decode-only", "workload": f"{cfg.name} decode", "decode": dec}), flush=True)
         return
 
+    if args.prefill_only:
+        cfg = inputs.CONFIGS[args.prefill_only]
+        Lp = Layer(torch, F, cfg, inputs.make_layer(cfg, seed=0))
+        Tp = PREFILL_SIZES.get(args.prefill_only, PREFILL_T)
+        px = measure_prefill(torch, F, Lp, Tp, args.steps, args.warmup, torch.cuda.current_stream(), rank)
+        if rank == 0:
+            print(json.dumps({"mode": "prefill-only", "workload": f"{cfg.name} prefill, T={Tp}",
+                              "prefill": summarize_prefill(px, hbm_gbs, tc_burst)}), flush=True)
+        return
+
     cfg = inputs.CONFIGS[WORKLOAD]
     layer_np = inputs.make_layer(cfg, seed=0)
     L = Layer(torch, F, cfg, layer_np)
@@ -560,7 +573,8 @@ def main():
     extra = None
     if args.extra:
         extra = {}
-        for name, Tp, Tds in [("dsv4_flash", 8192, [1, 8]), ("gemma4_26b_a4b", 2048, [1]), ("tiny", 64, [])]:
+        for name, Tds in [("dsv4_flash", [1, 8]), ("gemma4_26b_a4b", [1]), ("tiny", [])]:
+            Tp = PREFILL_SIZES[name]
             c = inputs.CONFIGS[name]
             Lx = Layer(torch, F, c, inputs.make_layer(c, seed=0))
             px = measure_prefill(torch, F, Lx, Tp, 10, 3, torch.cuda.current_stream(), rank)
