@@ -21,8 +21,10 @@ namespace ftmoe {
 
 
 // ------------------------------------------------------------------ gate/up + SwiGLU
-template <int TB, bool MX, bool FULLX>
-__global__ void __launch_bounds__(256) decode_gateup_kernel(DecodeArgs a) {
+// U: 16-byte weight vectors per lane kept in flight per row (BF16); MINB: resident CTAs per SM
+// the register budget is cut for (more warps in flight hide the load latency of small batches).
+template <int TB, bool MX, bool FULLX, int U, int MINB>
+__global__ void __launch_bounds__(256, MINB) decode_gateup_kernel(DecodeArgs a) {
     // FULLX: every token row [T][H] staged once (bf16, or f16 for MXFP4) before the
     // programmatic dependency wait -- the layer input is complete before the router ran --
     // so the routing-dependent part starts straight with the weight stream.
@@ -33,7 +35,7 @@ __global__ void __launch_bounds__(256) decode_gateup_kernel(DecodeArgs a) {
         for (int t = warp; t < a.T; t += 8) stage_x_row<MX>(a, xs4, t, t, lane);
     pdl_wait();
     pdl_trigger();
-    gateup_items<TB, MX, FULLX>(a, xs4, stok, blockIdx.x, gridDim.x);
+    gateup_items<TB, MX, FULLX, U>(a, xs4, stok, blockIdx.x, gridDim.x);
 }
 
 // ------------------------------------------------------------------ down + combine
@@ -278,11 +280,19 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (sms <= 0) sms = 148;
     }
-    dim3 g1(items < 2 * sms ? items : 2 * sms);     // two resident CTAs per SM: one wave
+    // one-token BF16 batches: four resident CTAs per SM with half the vectors in flight per lane
+    const bool wide = !mx && TB == 1;
+    const int per_sm = wide ? 4 : 2;
+    dim3 g1(items < per_sm * sms ? items : per_sm * sms);     // one wave
     cudaError_t e = cudaSuccess;
+    if (wide) {
+        e = fullx ? launch_pdl(decode_gateup_kernel<1, false, true, 4, 4>, g1, dim3(256), smem, st, a)
+                  : launch_pdl(decode_gateup_kernel<1, false, false, 4, 4>, g1, dim3(256), smem, st, a);
+        if (e != cudaSuccess) return e;
+    } else {
 #define FT_GU(TBV, MXV, FX)                                                                                   \
     do {                                                                                                      \
-        auto kern = decode_gateup_kernel<TBV, MXV, FX>;                                                       \
+        auto kern = decode_gateup_kernel<TBV, MXV, FX, 8, 1>;                                                 \
         if (smem > 48 * 1024) {                                                                               \
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));            \
             if (e != cudaSuccess) return e;                                                                   \
@@ -302,6 +312,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     }
 #undef FT_GU2
 #undef FT_GU
+    }
     if (e != cudaSuccess) return e;
     // down: the single-pass bulk-copy kernel when every routed expert's row block fits in
     // shared memory at two CTAs per SM, else the register-streaming kernel

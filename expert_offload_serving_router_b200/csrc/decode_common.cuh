@@ -121,7 +121,7 @@ __device__ __forceinline__ void stage_x_row(const DecodeArgs& a, uint4* xs4, int
 // rows; h = silu(gate) * up.  FULLX: all token rows are already staged in xs4; otherwise the
 // group's rows are staged per batch of TB.  Routing (sched, offsets, sorted_flat) comes
 // through `a`, global or shared.
-template <int TB, bool MX, bool FULLX>
+template <int TB, bool MX, bool FULLX, int U = 8>
 __device__ __forceinline__ void gateup_items(const DecodeArgs& a, uint4* xs4, int* stok, int item0, int stride) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H, F = a.F;
@@ -162,15 +162,15 @@ __device__ __forceinline__ void gateup_items(const DecodeArgs& a, uint4* xs4, in
             if (!MX) {
                 const uint4* gr = reinterpret_cast<const uint4*>(w.w13 + size_t(f) * H * 2);
                 const uint4* ur = reinterpret_cast<const uint4*>(w.w13 + size_t(F + f) * H * 2);
-                for (int c0 = lane; c0 < nv; c0 += 32 * 8) {
-                    uint4 wg[8], wu[8];
+                for (int c0 = lane; c0 < nv; c0 += 32 * U) {
+                    uint4 wg[U], wu[U];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
+                    for (int u = 0; u < U; ++u) {
                         int c = c0 + 32 * u;
                         if (c < nv) { wg[u] = ldg_nc_v4(gr + c); wu[u] = ldg_nc_v4(ur + c); }
                     }
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
+                    for (int u = 0; u < U; ++u) {
                         int c = c0 + 32 * u;
                         if (c >= nv) break;
 #pragma unroll
