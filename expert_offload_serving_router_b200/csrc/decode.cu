@@ -292,7 +292,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     } else {
 #define FT_GU(TBV, MXV, FX)                                                                                   \
     do {                                                                                                      \
-        auto kern = decode_gateup_kernel<TBV, MXV, FX, 8, 1>;                                                 \
+        auto kern = decode_gateup_kernel<TBV, MXV, FX, 8, 2>;                                                 \
         if (smem > 48 * 1024) {                                                                               \
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));            \
             if (e != cudaSuccess) return e;                                                                   \

@@ -100,6 +100,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 
 constexpr int kFPB = 8;       // f values per CTA (one per warp)
 
+// Staged rows are kept with their 16-byte vectors permuted inside aligned groups of eight:
+// vector v sits at xswz(v).  The MXFP4 GEMV reads vectors 4b .. 4b+3 for block b = lane (+32u),
+// i.e. a 64-byte stride across the warp; the permutation spreads each such read over all
+// eight 16-byte bank groups (conflict-free), and it keeps unit-stride reads conflict-free.
+__device__ __forceinline__ int xswz(int v) { return v ^ ((v >> 3) & 3); }
+
 // Stage token row t of x into shared row dst_row (bf16, or f16 for MXFP4); one warp.
 template <bool MX>
 __device__ __forceinline__ void stage_x_row(const DecodeArgs& a, uint4* xs4, int t, int dst_row, int lane) {
@@ -112,7 +118,7 @@ __device__ __forceinline__ void stage_x_row(const DecodeArgs& a, uint4* xs4, int
             u = make_uint4(f32x2_to_f16x2(bf16lo(u.x), bf16hi(u.x)), f32x2_to_f16x2(bf16lo(u.y), bf16hi(u.y)),
                            f32x2_to_f16x2(bf16lo(u.z), bf16hi(u.z)), f32x2_to_f16x2(bf16lo(u.w), bf16hi(u.w)));
         }
-        dst[v] = u;
+        dst[xswz(v)] = u;
     }
 }
 
@@ -176,7 +182,7 @@ __device__ __forceinline__ void gateup_items(const DecodeArgs& a, uint4* xs4, in
 #pragma unroll
                         for (int i = 0; i < TB; ++i) {
                             if (i >= nb) break;
-                            uint4 xv = xs4[size_t(stok[i]) * nv + c];
+                            uint4 xv = xs4[size_t(stok[i]) * nv + xswz(c)];
                             fma2_bf16(ag[i], wg[u].x, xv.x); fma2_bf16(ag[i], wg[u].y, xv.y);
                             fma2_bf16(ag[i], wg[u].z, xv.z); fma2_bf16(ag[i], wg[u].w, xv.w);
                             fma2_bf16(au[i], wu[u].x, xv.x); fma2_bf16(au[i], wu[u].y, xv.y);
@@ -206,7 +212,9 @@ __device__ __forceinline__ void gateup_items(const DecodeArgs& a, uint4* xs4, in
 #pragma unroll
                         for (int i = 0; i < TB; ++i) {
                             if (i >= nb) break;
-                            const uint4* xv = xs4 + size_t(stok[i]) * nv + b * 4;
+                            const uint4* xrow = xs4 + size_t(stok[i]) * nv;
+                            const uint4 xv[4] = {xrow[xswz(4 * b)], xrow[xswz(4 * b + 1)], xrow[xswz(4 * b + 2)],
+                                                 xrow[xswz(4 * b + 3)]};
                             ag[i] = fmaf(mx_block_dot(cg[u], xv), scg, ag[i]);
                             au[i] = fmaf(mx_block_dot(cu[u], xv), scu, au[i]);
                         }
