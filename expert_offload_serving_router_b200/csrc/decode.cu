@@ -280,14 +280,14 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (sms <= 0) sms = 148;
     }
-    // one-token BF16 batches: four resident CTAs per SM with half the vectors in flight per lane
-    const bool wide = !mx && TB == 1;
-    const int per_sm = wide ? 4 : 2;
+    // one-token batches: four (MXFP4: three) resident CTAs per SM, fewer vectors in flight per lane
+    const bool wide = TB == 1 && fullx;
+    const int per_sm = wide ? (mx ? 3 : 4) : 2;
     dim3 g1(items < per_sm * sms ? items : per_sm * sms);     // one wave
     cudaError_t e = cudaSuccess;
     if (wide) {
-        e = fullx ? launch_pdl(decode_gateup_kernel<1, false, true, 4, 4>, g1, dim3(256), smem, st, a)
-                  : launch_pdl(decode_gateup_kernel<1, false, false, 4, 4>, g1, dim3(256), smem, st, a);
+        e = mx ? launch_pdl(decode_gateup_kernel<1, true, true, 4, 3>, g1, dim3(256), smem, st, a)
+               : launch_pdl(decode_gateup_kernel<1, false, true, 4, 4>, g1, dim3(256), smem, st, a);
         if (e != cudaSuccess) return e;
     } else {
 #define FT_GU(TBV, MXV, FX)                                                                                   \
