@@ -42,6 +42,19 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Transpose-reduce step: n per-lane values -> n/2, pairing lanes across `off`; lanes with
+// (lane & off) keep the upper half.  After log2(n) steps plus plain butterfly steps each
+// lane holds one complete warp sum (n-1 + 5 - log2 n shuffles instead of 5 n).
+__device__ __forceinline__ void tr_step(float* v, int n, int off, int lane) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+        const float send = up ? v[i] : v[i + n / 2];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, off);
+        v[i] = (up ? v[i + n / 2] : v[i]) + recv;
+    }
+}
+
 // silu(a) * b, silu(a) = a * sigmoid(a) = h + h * tanh(h) with h = a/2 (tanh.approx: one MUFU op,
 // relative error ~2^-11, below the bf16 rounding of the result)
 __device__ __forceinline__ float tanh_approx(float x) {

@@ -269,7 +269,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     while (TB < a.T && TB < 8) TB <<= 1;
     // small batches stage all token rows once per CTA (before the dependency wait); larger
     // ones stage each group's rows per batch of TB
-    const bool fullx = size_t(a.T) * a.H * 2 <= 16 * 1024;
+    const bool fullx = size_t(a.T) * a.H * 2 <= 64 * 1024;
     while (!fullx && TB > 1 && size_t(TB) * a.H * 2 > 65536) TB >>= 1;
     const size_t smem = size_t(fullx ? a.T : TB) * a.H * 2;
     int items = na_max * ((a.F + kFPB - 1) / kFPB);   // upper bound; the kernel strides over the real count

@@ -63,34 +63,43 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// dot of one 32-element MXFP4 block (16 code bytes) with 32 f16 activations (4 x uint4)
+// One 32-element MXFP4 block (16 code bytes) as 16 f16x2 words: word 4q+b holds elements
+// 8q+2b (low half) and 8q+2b+1, exactly.
+__device__ __forceinline__ void mx_block_cvt(const uint4& c, uint32_t (&wf)[16]) {
+    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) wf[4 * q + b] = e2m1x2_f16x2((cw[q] >> (8 * b)) & 0xFFu);
+}
+// dot of a converted block with 32 f16 activations (4 x uint4): exact products, two fp32 chains
+__device__ __forceinline__ float mx_cvt_dot(const uint32_t (&wf)[16], const uint4* xv) {
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 xx = xv[q];
+        fma2_f16(a0, wf[4 * q + 0], xx.x);
+        fma2_f16(a1, wf[4 * q + 1], xx.y);
+        fma2_f16(a0, wf[4 * q + 2], xx.z);
+        fma2_f16(a1, wf[4 * q + 3], xx.w);
+    }
+    return a0 + a1;
+}
+// the same dot with conversion and products interleaved (fewer live registers)
 __device__ __forceinline__ float mx_block_dot(const uint4& c, const uint4* xv) {
     float a0 = 0.f, a1 = 0.f;
     const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {            // 4 code bytes per word -> 8 elements
+    for (int q = 0; q < 4; ++q) {
         const uint4 xx = xv[q];
         const uint32_t xw[4] = {xx.x, xx.y, xx.z, xx.w};
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-            uint32_t wf = e2m1x2_f16x2((cw[q] >> (8 * b)) & 0xFFu);
+            const uint32_t wf = e2m1x2_f16x2((cw[q] >> (8 * b)) & 0xFFu);
             if (b & 1) fma2_f16(a1, wf, xw[b]); else fma2_f16(a0, wf, xw[b]);
         }
     }
     return a0 + a1;
-}
-
-// Transpose-reduce step: n per-lane values -> n/2, pairing lanes across `off`; lanes with
-// (lane & off) keep the upper half.  After log2(n) steps plus plain butterfly steps each
-// lane holds one complete warp sum (n-1 + 5 - log2 n shuffles instead of 5 n).
-__device__ __forceinline__ void tr_step(float* v, int n, int off, int lane) {
-    const bool up = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < n / 2; ++i) {
-        const float send = up ? v[i] : v[i + n / 2];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, off);
-        v[i] = (up ? v[i + n / 2] : v[i]) + recv;
-    }
 }
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -209,14 +218,30 @@ __device__ __forceinline__ void gateup_items(const DecodeArgs& a, uint4* xs4, in
                         int b = b0 + 32 * u;
                         if (b >= nblk) break;
                         const float scg = e8m0f(sg[u]), scu = e8m0f(su[u]);
+                        if (TB == 1) {
+#pragma unroll
+                            for (int i = 0; i < TB; ++i) {
+                                if (i >= nb) break;
+                                const uint4* xrow = xs4 + size_t(stok[i]) * nv;
+                                const uint4 xv[4] = {xrow[xswz(4 * b)], xrow[xswz(4 * b + 1)], xrow[xswz(4 * b + 2)],
+                                                     xrow[xswz(4 * b + 3)]};
+                                ag[i] = fmaf(mx_block_dot(cg[u], xv), scg, ag[i]);
+                                au[i] = fmaf(mx_block_dot(cu[u], xv), scu, au[i]);
+                            }
+                            continue;
+                        }
+                        // E2M1 -> f16 once per block, shared by every token of the batch
+                        uint32_t fg[16], fu[16];
+                        mx_block_cvt(cg[u], fg);
+                        mx_block_cvt(cu[u], fu);
 #pragma unroll
                         for (int i = 0; i < TB; ++i) {
                             if (i >= nb) break;
                             const uint4* xrow = xs4 + size_t(stok[i]) * nv;
                             const uint4 xv[4] = {xrow[xswz(4 * b)], xrow[xswz(4 * b + 1)], xrow[xswz(4 * b + 2)],
                                                  xrow[xswz(4 * b + 3)]};
-                            ag[i] = fmaf(mx_block_dot(cg[u], xv), scg, ag[i]);
-                            au[i] = fmaf(mx_block_dot(cu[u], xv), scu, au[i]);
+                            ag[i] = fmaf(mx_cvt_dot(fg, xv), scg, ag[i]);
+                            au[i] = fmaf(mx_cvt_dot(fu, xv), scu, au[i]);
                         }
                     }
                 }

@@ -50,22 +50,35 @@ __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteArgs a) {
             asm volatile("griddepcontrol.wait;" ::: "memory");
             asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         }
-        for (int t = 0; t < a.T; ++t) {
-            const uint2* xr = reinterpret_cast<const uint2*>(a.x + size_t(t) * a.H);
-            float s = 0.f;
+        // eight tokens per pass: all their x loads in flight together, then one transpose-
+        // reduce leaves token t0 + 4*bit4(lane) + 2*bit3(lane) + bit2(lane) on lane
+        for (int t0 = 0; t0 < a.T; t0 += 8) {
+            float s[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                int q = base + tid + 256 * i;
-                if (q < nq) {
-                    uint2 u = __ldg(xr + q);
-                    s = fmaf(bf16lo(u.x), w[i].x, s);
-                    s = fmaf(bf16hi(u.x), w[i].y, s);
-                    s = fmaf(bf16lo(u.y), w[i].z, s);
-                    s = fmaf(bf16hi(u.y), w[i].w, s);
+            for (int j = 0; j < 8; ++j) {
+                s[j] = 0.f;
+                if (t0 + j < a.T) {
+                    const uint2* xr = reinterpret_cast<const uint2*>(a.x + size_t(t0 + j) * a.H);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        int q = base + tid + 256 * i;
+                        if (q < nq) {
+                            uint2 u = __ldg(xr + q);
+                            s[j] = fmaf(bf16lo(u.x), w[i].x, s[j]);
+                            s[j] = fmaf(bf16hi(u.x), w[i].y, s[j]);
+                            s[j] = fmaf(bf16lo(u.y), w[i].z, s[j]);
+                            s[j] = fmaf(bf16hi(u.y), w[i].w, s[j]);
+                        }
+                    }
                 }
             }
-            s = warp_sum(s);
-            if (lane == 0) red[t][warp] += s;
+            tr_step(s, 8, 16, lane);
+            tr_step(s, 4, 8, lane);
+            tr_step(s, 2, 4, lane);
+            s[0] += __shfl_xor_sync(0xffffffffu, s[0], 2);
+            s[0] += __shfl_xor_sync(0xffffffffu, s[0], 1);
+            const int t = t0 + ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+            if ((lane & 3) == 0 && t < a.T) red[t][warp] += s[0];
         }
     }
     __syncthreads();
