@@ -466,8 +466,8 @@ def measure_stack(torch, F, rank, hbm_gbs):
                           "frac_of_h2d_probe": out["host_bytes"] / (pf_ms * 1e-3) / 1e9 / best,
                           "layer_copy_ms_at_probe": layer_bytes / (best * 1e9) * 1e3}
         del ws, yl, xl
-        # decode: cold cache, 256 single-token steps
-        F.ft_expert_stream_reset_cache(handle)
+        # decode: cold cache, 256 single-token steps, first with a cache per layer, then with
+        # the same total slot count pooled across layers (global LRU at equal capacity)
         steps = st["decode_steps"]
         wsb = F.ft_moe_workspace_bytes(shape, 1)
         ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
@@ -475,22 +475,35 @@ def measure_stack(torch, F, rank, hbm_gbs):
         yl = torch.empty((nl, 1, H), dtype=torch.int16, device="cuda")
         xl = torch.empty((nl, 1, H), dtype=torch.int16, device="cuda")
         xs = [Layer.dev(torch, inputs.make_tokens(cfg, 1, seed=1, stream=600 + s)) for s in range(steps)]
-        torch.cuda.synchronize()
-        t0 = time.perf_counter()
-        for s in range(steps):
-            F.ft_expert_stream_decode_step(handle, 1, xs[s], wr, bs, yl, xl, ws, copy_stream=copy_stream)
-        torch.cuda.synchronize()
-        dec_s = time.perf_counter() - t0
-        st_all = F.ft_expert_stream_stats(handle, -1)
-        hits, misses = st_all[0], st_all[1]
-        out["decode"] = {"steps": steps, "layers": nl, "slots_per_layer": slots, "s_total": dec_s,
-                         "steps_per_s": steps / dec_s, "ms_per_step": 1e3 * dec_s / steps,
-                         "hits": hits, "misses": misses, "miss_rate": misses / max(1, hits + misses),
-                         "h2d_bytes": st_all[2], "wait_us_total": st_all[5],
-                         "timing": "host wall clock around the 256 steps (each step waits for its routed ids)"}
+
+        def decode_run(h):
+            F.ft_expert_stream_reset_cache(h)
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            for s in range(steps):
+                F.ft_expert_stream_decode_step(h, 1, xs[s], wr, bs, yl, xl, ws, copy_stream=copy_stream)
+            torch.cuda.synchronize()
+            dec_s = time.perf_counter() - t0
+            st_all = F.ft_expert_stream_stats(h, -1)
+            hits, misses = st_all[0], st_all[1]
+            return {"steps": steps, "layers": nl, "s_total": dec_s,
+                    "steps_per_s": steps / dec_s, "ms_per_step": 1e3 * dec_s / steps,
+                    "hits": hits, "misses": misses, "miss_rate": misses / max(1, hits + misses),
+                    "h2d_bytes": st_all[2], "wait_us_total": st_all[5],
+                    "timing": "host wall clock around the 256 steps (each step waits for its routed ids)"}
+
+        out["decode"] = dict(decode_run(handle), slots_per_layer=slots, cache="per layer")
+        F.ft_moe_check(ws)
+        F.ft_expert_stream_destroy(handle)
+        handle = None
+        cfgs.cache_policy = F.FT_CACHE_GLOBAL
+        handle = F.ft_expert_stream_create(cfgs)
+        out["decode_global_cache"] = dict(decode_run(handle), slots_total=nl * slots,
+                                          cache="one LRU over all layers' slots (same capacity)")
         F.ft_moe_check(ws)
     finally:
-        F.ft_expert_stream_destroy(handle)
+        if handle is not None:
+            F.ft_expert_stream_destroy(handle)
     return out
 
 

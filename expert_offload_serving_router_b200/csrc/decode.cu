@@ -43,9 +43,9 @@ constexpr int kRPB = 8;       // hidden rows per CTA
 constexpr int kMaxDecodeRows = 32 * (kMaxTopK + 1);
 
 template <bool MX, int CPL>
-__global__ void __launch_bounds__(256, MX ? 1 : 2) decode_down_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(256, 2) decode_down_kernel(DecodeArgs a) {
     // CPL = weight vectors per lane per row (BF16: 16-byte chunks of 8; MXFP4: 32-element blocks)
-    constexpr int RB = (MX ? 16 : 24) / CPL >= 8 ? 8 : (MX ? 16 : 24) / CPL >= 4 ? 4 : (MX ? 16 : 24) / CPL >= 2 ? 2 : 1;
+    constexpr int RB = (MX ? 8 : 24) / CPL >= 8 ? 8 : (MX ? 8 : 24) / CPL >= 4 ? 4 : (MX ? 8 : 24) / CPL >= 2 ? 2 : 1;
     constexpr int NB = kRPB / RB;               // row batches per active group
     __shared__ float prod[kMaxDecodeRows][kRPB + 1];
     pdl_trigger();   // the next layer's router may launch; it waits for this grid before writing

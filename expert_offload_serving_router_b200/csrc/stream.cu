@@ -11,7 +11,11 @@
 // GPU, the routed ids come back through a pinned buffer (the one host wait, bounded), the
 // host LRU policy (ft_lru_step) assigns slots, missed experts are copied host->HBM into
 // their slots on the copy stream, a per-layer device pointer table is refreshed, and the
-// decode kernels read the experts through the table.
+// decode kernels read the experts through the table.  The cache is either one LRU per
+// layer or one LRU over all layers' slots keyed by (layer, expert) (global LRU at equal
+// capacity: FreeToken article, dothoosh.com, "Benchmarks and real performance").  Any
+// slot may be overwritten safely: the host has just waited for this layer's routed ids,
+// which were produced after every earlier kernel on the compute stream finished reading.
 #include <algorithm>
 #include <chrono>
 #include <cstring>
@@ -67,9 +71,9 @@ extern "C" ft_status ft_lru_step(int32_t E, int32_t n_slots, int32_t* content, i
 }
 
 struct LayerCache {
-    std::vector<int32_t> content;   // [slots] expert id or -1
+    std::vector<int32_t> content;   // [slots] expert id (global pool: layer * E + expert) or -1
     std::vector<int64_t> stamp;     // [slots]
-    std::vector<int32_t> where;     // [E] slot or -1
+    std::vector<int32_t> where;     // [E] (global pool: [L * E]) slot or -1
     uint64_t hits = 0, misses = 0, h2d = 0, steps = 0, prefill_copies = 0, wait_us = 0;
 };
 
@@ -84,7 +88,10 @@ struct ft_expert_stream {
     void** htable;                  // pinned host mirror [L][E][4]
     int32_t* hids;                  // pinned [kSmallRoute * kMaxTopK]
     cudaEvent_t ready[2], freed[2], ids_ev, copy_ev;
-    std::vector<LayerCache> cache;
+    std::vector<LayerCache> cache;  // per-layer counters; per-layer policy: also the slot state
+    bool global = false;            // FT_CACHE_GLOBAL: slot state lives in `pool`
+    LayerCache pool;                // [L * S] slots shared by all layers
+    int64_t policy_steps = 0;       // global policy steps taken (decode step * L + layer)
     int64_t timeout_ms;
     int64_t inject_at = 0;          // 0: off; else fail the n-th expert copy enqueue
     int64_t copy_count = 0;
@@ -106,6 +113,21 @@ static size_t arena_bytes(const ft_stream_cfg* c) {
     const size_t expert = a256(b13) + a256(b13s) + a256(b2) + a256(b2s);
     return 2 * layer + size_t(c->num_layers) * c->slots_per_layer * expert +
            a256(size_t(c->num_layers) * E * 4 * sizeof(void*));
+}
+
+// empty every slot of the active policy's state (counters are left alone)
+static void reset_slots(ft_expert_stream* st) {
+    const size_t L = size_t(st->L), S = size_t(st->S), E = size_t(st->E);
+    st->cache.resize(L);
+    for (auto& c : st->cache) {
+        c.content.assign(st->global ? 0 : S, -1);
+        c.stamp.assign(st->global ? 0 : S, -1);
+        c.where.assign(st->global ? 0 : E, -1);
+    }
+    st->pool.content.assign(st->global ? L * S : 0, -1);
+    st->pool.stamp.assign(st->global ? L * S : 0, -1);
+    st->pool.where.assign(st->global ? L * E : 0, -1);
+    st->policy_steps = 0;
 }
 
 static bool is_pinned(const void* p) {
@@ -131,6 +153,8 @@ ft_status ft_expert_stream_create(const ft_stream_cfg* cfg, ft_expert_stream** o
     if (cfg->num_layers <= 0) return fail(FT_ERR_INVALID_ARG, "num_layers must be > 0");
     if (cfg->slots_per_layer < k || cfg->slots_per_layer > E)
         return fail(FT_ERR_INVALID_ARG, "slots_per_layer %d must be in [k=%d, E=%d]", cfg->slots_per_layer, k, E);
+    if (cfg->cache_policy != FT_CACHE_PER_LAYER && cfg->cache_policy != FT_CACHE_GLOBAL)
+        return fail(FT_ERR_INVALID_ARG, "cache_policy %d is not a ft_cache_policy", cfg->cache_policy);
     if (!cfg->host_layers) return fail(FT_ERR_INVALID_ARG, "host_layers is NULL");
     if (!cfg->hbm_arena || (reinterpret_cast<uintptr_t>(cfg->hbm_arena) & 255))
         return fail(FT_ERR_INVALID_ARG, "hbm_arena NULL or not 256-byte aligned");
@@ -168,12 +192,8 @@ ft_status ft_expert_stream_create(const ft_stream_cfg* cfg, ft_expert_stream** o
     st->slots = base + 2 * st->layer_bytes;
     st->dtable = reinterpret_cast<void**>(st->slots + size_t(st->L) * st->S * st->expert_bytes);
     st->timeout_ms = cfg->host_wait_timeout_ms > 0 ? cfg->host_wait_timeout_ms : 10000;
-    st->cache.resize(size_t(st->L));
-    for (auto& c : st->cache) {
-        c.content.assign(size_t(st->S), -1);
-        c.stamp.assign(size_t(st->S), -1);
-        c.where.assign(size_t(E), -1);
-    }
+    st->global = cfg->cache_policy == FT_CACHE_GLOBAL;
+    reset_slots(st);
     cudaError_t e = cudaHostAlloc(reinterpret_cast<void**>(&st->htable), size_t(st->L) * E * 4 * sizeof(void*), cudaHostAllocDefault);
     if (e == cudaSuccess) e = cudaHostAlloc(reinterpret_cast<void**>(&st->hids), sizeof(int32_t) * kSmallRoute * kMaxTopK, cudaHostAllocDefault);
     for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
@@ -339,14 +359,23 @@ ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const voi
         ids.erase(std::unique(ids.begin(), ids.end()), ids.end());
         for (int32_t v : ids)
             if (v < 0 || v >= E) return fail(FT_ERR_DEVICE_CHECK, "layer %d: routed id %d outside [0, %d)", l, v, E);
-        if (int(ids.size()) > s->S)
-            return fail(FT_ERR_UNSUPPORTED, "layer %d: %zu distinct experts in one step > %d slots", l, ids.size(), s->S);
-        const std::vector<int32_t> bc = c.content, bw = c.where;
-        const std::vector<int64_t> bs = c.stamp;
+        const int cap = s->global ? s->L * s->S : s->S;
+        if (int(ids.size()) > cap)
+            return fail(FT_ERR_UNSUPPORTED, "layer %d: %zu distinct experts in one step > %d slots", l, ids.size(), cap);
+        // the policy's state: this layer's own slots, or the pool keyed by layer * E + expert
+        LayerCache& pc = s->global ? s->pool : c;
+        const int32_t key_base = s->global ? l * E : 0;
+        const int32_t key_count = s->global ? s->L * E : E;
+        const int32_t n_slots = s->global ? s->L * s->S : s->S;
+        const int64_t pstep = s->global ? s->policy_steps : int64_t(c.steps);
+        std::vector<int32_t> keys(ids);
+        for (int32_t& v : keys) v += key_base;
+        const std::vector<int32_t> bc = pc.content, bw = pc.where;
+        const std::vector<int64_t> bs = pc.stamp;
         std::vector<int32_t> slot(ids.size());
         std::vector<uint8_t> hit(ids.size());
-        if ((st = ft_lru_step(E, s->S, c.content.data(), c.stamp.data(), c.where.data(), int64_t(c.steps), ids.data(),
-                              int32_t(ids.size()), slot.data(), hit.data())))
+        if ((st = ft_lru_step(key_count, n_slots, pc.content.data(), pc.stamp.data(), pc.where.data(), pstep,
+                              keys.data(), int32_t(ids.size()), slot.data(), hit.data())))
             return st;
         // 3. copy the misses into their slots (copy stream), refresh the pointer table
         void** ht = s->htable + size_t(l) * E * 4;
@@ -354,7 +383,7 @@ ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const voi
         uint64_t bytes = 0, nmiss = 0;
         for (size_t i = 0; i < ids.size(); ++i) {
             const int u = ids[i];
-            uint8_t* sp = s->slots + (size_t(l) * s->S + slot[i]) * s->expert_bytes;
+            uint8_t* sp = s->slots + ((s->global ? 0 : size_t(l) * s->S) + slot[i]) * s->expert_bytes;
             uint8_t* p13 = sp;
             uint8_t* p13s = sp + a256(s->b13);
             uint8_t* p2 = p13s + a256(s->b13s);
@@ -364,12 +393,12 @@ ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const voi
                 if (s->inject_at > 0 && s->copy_count == s->inject_at) {
                     // injected failure: undo this step's policy update; slots already being
                     // overwritten by enqueued copies no longer hold their old expert
-                    c.content = bc; c.where = bw; c.stamp = bs;
+                    pc.content = bc; pc.where = bw; pc.stamp = bs;
                     for (int d : dirtied) {
-                        int old = c.content[d];
-                        if (old >= 0) c.where[old] = -1;
-                        c.content[d] = -1;
-                        c.stamp[d] = -1;
+                        int old = pc.content[d];
+                        if (old >= 0) pc.where[old] = -1;
+                        pc.content[d] = -1;
+                        pc.stamp[d] = -1;
                     }
                     return fail(FT_ERR_CUDA, "layer %d: injected host->device copy failure (copy %lld)", l,
                                 (long long)s->copy_count);
@@ -398,6 +427,7 @@ ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const voi
         c.misses += nmiss;
         c.h2d += bytes;
         c.steps += 1;
+        if (s->global) s->policy_steps += 1;
         if ((st = cuda_ok(cudaEventRecord(s->copy_ev, ps), "record copies"))) return st;
         if ((st = cuda_ok(cudaStreamWaitEvent(cs, s->copy_ev, 0), "wait copies"))) return st;
         void** dt = s->dtable + size_t(l) * E * 4;
@@ -433,7 +463,13 @@ ft_status ft_expert_stream_stats(const ft_expert_stream* s, int32_t layer, uint6
 }
 
 ft_status ft_expert_stream_slots(const ft_expert_stream* s, int32_t layer, int32_t* out) {
-    if (!s || !out || layer < 0 || layer >= s->L) return fail(FT_ERR_INVALID_ARG, "bad slots arguments");
+    if (!s || !out) return fail(FT_ERR_INVALID_ARG, "bad slots arguments");
+    if (s->global) {
+        if (layer != -1) return fail(FT_ERR_INVALID_ARG, "global cache: slots are read with layer = -1");
+        std::copy(s->pool.content.begin(), s->pool.content.end(), out);
+        return FT_OK;
+    }
+    if (layer < 0 || layer >= s->L) return fail(FT_ERR_INVALID_ARG, "bad slots arguments");
     const LayerCache& c = s->cache[size_t(layer)];
     for (int i = 0; i < s->S; ++i) out[i] = c.content[size_t(i)];
     return FT_OK;
@@ -441,12 +477,8 @@ ft_status ft_expert_stream_slots(const ft_expert_stream* s, int32_t layer, int32
 
 ft_status ft_expert_stream_reset_cache(ft_expert_stream* s) {
     if (!s) return fail(FT_ERR_INVALID_ARG, "stream handle is NULL");
-    for (auto& c : s->cache) {
-        c = LayerCache();
-        c.content.assign(size_t(s->S), -1);
-        c.stamp.assign(size_t(s->S), -1);
-        c.where.assign(size_t(s->E), -1);
-    }
+    for (auto& c : s->cache) c = LayerCache();
+    reset_slots(s);
     s->copy_count = 0;
     return FT_OK;
 }

@@ -20,6 +20,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "ftmoe.h")
 FT_OK, FT_ERR_INVALID_ARG, FT_ERR_UNSUPPORTED, FT_ERR_CUDA, FT_ERR_WORKSPACE, FT_ERR_NOT_PINNED, \
     FT_ERR_TIMEOUT, FT_ERR_DEVICE_CHECK = range(8)
 FT_W_BF16, FT_W_MXFP4 = 0, 1
+FT_CACHE_PER_LAYER, FT_CACHE_GLOBAL = 0, 1
 
 c_i32, c_i64, c_u64, c_sz, c_vp, c_f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t, \
     ctypes.c_void_p, ctypes.c_float
@@ -38,7 +39,7 @@ class ft_moe_weights(ctypes.Structure):
 class ft_stream_cfg(ctypes.Structure):
     _fields_ = [("num_layers", c_i32), ("slots_per_layer", c_i32), ("shape", ft_moe_shape),
                 ("host_layers", ctypes.POINTER(ft_moe_weights)), ("hbm_arena", c_vp), ("hbm_arena_bytes", c_sz),
-                ("host_wait_timeout_ms", c_i64)]
+                ("host_wait_timeout_ms", c_i64), ("cache_policy", c_i32)]
 
 
 class FtError(RuntimeError):

@@ -229,9 +229,20 @@ ft_status ft_moe_unit_rms(int32_t T, int32_t H, const void* in, void* out, float
  *   untouched slot with the oldest use), copies the missed experts host->HBM,
  *   and runs the experts through a device pointer table.  The cache starts
  *   cold.  Stacked layers are chained as x_{l+1} = ft_moe_unit_rms(y_l, 1e-6).
+ *   cache_policy FT_CACHE_GLOBAL instead pools all num_layers * slots_per_layer
+ *   slots into one LRU cache keyed by (layer, expert) -- the cross-layer cache of
+ *   the FreeToken article (dothoosh.com, "Benchmarks and real performance":
+ *   global LRU at equal capacity) -- with the same policy, one policy step per
+ *   (decode step, layer) in execution order; a layer's misses may evict any
+ *   layer's expert not touched in that policy step.
  * Shared experts and router weights are device-resident (caller-owned).
  * ------------------------------------------------------------------------- */
 typedef struct ft_expert_stream ft_expert_stream;
+
+typedef enum {
+    FT_CACHE_PER_LAYER = 0,   /* slots_per_layer slots owned by each layer */
+    FT_CACHE_GLOBAL = 1       /* num_layers * slots_per_layer slots shared by all layers */
+} ft_cache_policy;
 
 typedef struct {
     int32_t num_layers;
@@ -243,6 +254,7 @@ typedef struct {
     void* hbm_arena;                    /* device, caller-owned, 256-byte aligned */
     size_t hbm_arena_bytes;             /* >= ft_expert_stream_arena_bytes(cfg) */
     int64_t host_wait_timeout_ms;       /* bound on every host wait (<= 0: 10000) */
+    int32_t cache_policy;               /* ft_cache_policy; 0 (zero-initialised) = per layer */
 } ft_stream_cfg;
 
 /* Device bytes the stream needs in hbm_arena: two full-layer buffers plus
@@ -276,8 +288,9 @@ ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const voi
  * out[4] prefill layer copies, out[5] bounded-wait time in microseconds. */
 ft_status ft_expert_stream_stats(const ft_expert_stream* s, int32_t layer, uint64_t out[6]);
 
-/* Slot contents of one layer after the last step: out[slots_per_layer]
- * expert ids (-1 = empty). */
+/* Slot contents after the last step.  Per-layer cache: out[slots_per_layer]
+ * expert ids of `layer` (-1 = empty).  Global cache: layer must be -1 and
+ * out[num_layers * slots_per_layer] holds layer * E + expert (-1 = empty). */
 ft_status ft_expert_stream_slots(const ft_expert_stream* s, int32_t layer, int32_t* out);
 
 /* Empties every slot (next decode step starts cold) and zeroes the counters. */
@@ -293,7 +306,10 @@ void ft_expert_stream_destroy(ft_expert_stream* s);
  * sorted ascending, unique, n <= n_slots.  Every id already cached is a hit
  * and is touched first; then misses, in ascending id, each take the lowest
  * empty slot or else the slot not touched in this step with the smallest
- * stamp.  Stamp of ids[r] = step * E + r.  Outputs out_slot[n], out_hit[n]. */
+ * stamp.  Stamp of ids[r] = step * E + r.  Outputs out_slot[n], out_hit[n].
+ * The global cache calls it with E' = num_layers * E, ids layer * E + expert,
+ * n_slots = num_layers * slots_per_layer and step = the policy-step count
+ * (decode step * num_layers + layer). */
 ft_status ft_lru_step(int32_t E, int32_t n_slots, int32_t* content, int64_t* stamp, int32_t* where,
                       int64_t step, const int32_t* ids, int32_t n, int32_t* out_slot, uint8_t* out_hit);
 

@@ -185,6 +185,23 @@ def lru_sim(num_experts: int, n_slots: int, steps):
     return out_slot, out_hit, se, h.value, m.value
 
 
+def lru_sim_global(num_layers: int, num_experts: int, n_slots: int, routed):
+    """One LRU cache of n_slots slots shared by all layers, keyed by layer * E + expert
+    (global LRU at equal capacity: FreeToken article, dothoosh.com, "Benchmarks and real
+    performance").  routed[l][s]: expert ids of layer l at decode step s.  Policy steps run
+    in execution order (step 0 layers 0..L-1, step 1 ...), each the same policy as
+    lru_sim.  Returns (per-layer hits, per-layer misses, final slot contents)."""
+    L, E = num_layers, num_experts
+    n_steps = len(routed[0])
+    flat = [[l * E + int(e) for e in routed[l][s]] for s in range(n_steps) for l in range(L)]
+    _, hit, se, _, _ = lru_sim(L * E, n_slots, flat)
+    hits, misses = [0] * L, [0] * L
+    for i, h in enumerate(hit):
+        hits[i % L] += sum(h)
+        misses[i % L] += len(h) - sum(h)
+    return hits, misses, (se[-1].tolist() if len(flat) else [-1] * n_slots)
+
+
 def full_layer(shape: dict, x_bits, w_router, bias, weights: dict, logits32=None, tokens=None, n_threads: int = 0):
     """Convenience: logits (fp64) -> top-k on the given fp32 logits (or on the fp64 logits
     rounded to fp32 when none are given) -> y for the listed tokens."""

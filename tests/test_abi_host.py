@@ -122,6 +122,12 @@ def test_stream_config_rejected_on_host():
     with pytest.raises(F.FtError) as ei:          # NULL host pointers
         F.ft_expert_stream_create(cfg)
     assert ei.value.status == F.FT_ERR_INVALID_ARG
+    cfg.cache_policy = 2                          # not a ft_cache_policy
+    with pytest.raises(F.FtError) as ei:
+        F.ft_expert_stream_create(cfg)
+    assert ei.value.status == F.FT_ERR_INVALID_ARG and "cache_policy" in str(ei.value)
+    cfg.cache_policy = F.FT_CACHE_GLOBAL          # same arena size: the pool has L * S slots
+    assert F.ft_expert_stream_arena_bytes(cfg) == cfg.hbm_arena_bytes
 
 
 @pytest.mark.parametrize("seed", range(4))
@@ -156,3 +162,28 @@ def test_host_lru_rejects_unsorted_or_oversized():
         F.ft_lru_step(8, 2, content, stamp, where, 0, np.array([1, 2, 3], np.int32), o, hh)
     with pytest.raises(F.FtError):
         F.ft_lru_step(8, 2, content, stamp, where, 0, np.array([2, 1], np.int32), o[:2], hh[:2])
+
+
+def test_host_lru_policy_as_global_pool_matches_oracle():
+    """The global cache drives ft_lru_step over keys layer * E + expert, L * S slots and one
+    policy step per (decode step, layer); that must reproduce the oracle's global LRU."""
+    r = random.Random(5)
+    L, E, S = 3, 32, 4
+    steps = 50
+    routed = [[sorted(set(min(E - 1, int(r.paretovariate(0.9)) - 1 + r.randint(0, 4)) for _ in range(r.randint(1, 4))))
+               for _ in range(steps)] for _ in range(L)]
+    oh, om, oslots = oracle.lru_sim_global(L, E, L * S, routed)
+    content = np.full(L * S, -1, np.int32)
+    stamp = np.full(L * S, -1, np.int64)
+    where = np.full(L * E, -1, np.int32)
+    hits, misses = [0] * L, [0] * L
+    for s in range(steps):
+        for l in range(L):
+            keys = np.array([l * E + e for e in routed[l][s]], np.int32)
+            out_slot = np.empty(len(keys), np.int32)
+            out_hit = np.empty(len(keys), np.uint8)
+            F.ft_lru_step(L * E, L * S, content, stamp, where, s * L + l, keys, out_slot, out_hit)
+            hits[l] += int(out_hit.sum())
+            misses[l] += len(keys) - int(out_hit.sum())
+    assert (hits, misses) == (oh, om)
+    assert content.tolist() == oslots

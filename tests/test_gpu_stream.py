@@ -14,7 +14,7 @@ NL, SLOTS = 3, 4
 
 
 class Stack:
-    def __init__(self, wdtype=inputs.WDTYPE_MXFP4, zipf=True):
+    def __init__(self, wdtype=inputs.WDTYPE_MXFP4, zipf=True, cache_policy=F.FT_CACHE_PER_LAYER):
         import torch
         from gpu_util import DevLayer, ensure_built, shape_of
         ensure_built()
@@ -37,7 +37,7 @@ class Stack:
                 self.pinned.append(t)
             hl[l] = F.make_weights(ph.get("w13"), ph.get("w13_scale"), ph.get("w2"), ph.get("w2_scale"))
         self.host_layers = hl
-        cfg = F.ft_stream_cfg(NL, SLOTS, self.shape, hl, None, 0, 5000)
+        cfg = F.ft_stream_cfg(NL, SLOTS, self.shape, hl, None, 0, 5000, cache_policy)
         n = F.ft_expert_stream_arena_bytes(cfg)
         self.arena = torch.empty(n, dtype=torch.uint8, device="cuda")
         cfg.hbm_arena = self.arena.data_ptr()
@@ -115,6 +115,32 @@ def test_decode_follows_oracle_lru_and_equals_resident(stack):
         tot_m += m
     assert tot_m >= NL * 2          # cold start: the first step misses
     assert tot_h > 0                # Zipf-skewed routing revisits hot experts
+
+
+def test_global_cache_follows_oracle_global_lru_and_equals_resident():
+    g = Stack(cache_policy=F.FT_CACHE_GLOBAL)
+    try:
+        steps = 24
+        routed = [[] for _ in range(NL)]
+        for s in range(steps):
+            x = inputs.make_tokens(g.cfg, 1, seed=12, stream=s)
+            y, xl = g.run("decode", x)
+            for l, L in enumerate(g.layers):
+                yr, idx, lg = _resident(L, xl[l])
+                assert np.array_equal(y[l], yr), f"step {s} layer {l}: pooled-cache result != resident"
+                routed[l].append(sorted(set(idx.ravel().tolist())))
+        oh, om, oslots = oracle.lru_sim_global(NL, g.cfg.num_experts, NL * SLOTS, routed)
+        for l in range(NL):
+            st = F.ft_expert_stream_stats(g.handle, l)
+            assert (st[0], st[1], st[3]) == (oh[l], om[l], steps)
+        assert F.ft_expert_stream_slots(g.handle, -1, NL * SLOTS) == oslots
+        with pytest.raises(F.FtError) as ei:      # the pool has no per-layer view
+            F.ft_expert_stream_slots(g.handle, 0, SLOTS)
+        assert ei.value.status == F.FT_ERR_INVALID_ARG
+        F.ft_expert_stream_reset_cache(g.handle)
+        assert F.ft_expert_stream_slots(g.handle, -1, NL * SLOTS) == [-1] * (NL * SLOTS)
+    finally:
+        g.close()
 
 
 def test_injected_copy_failure_is_reported_and_rolled_back(stack):

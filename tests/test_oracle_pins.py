@@ -317,3 +317,48 @@ def test_lru_cold_start_and_capacity_errors():
     assert slot[0] == [1, 0] or slot[0] == [0, 1]
     with pytest.raises(ValueError):
         oracle.lru_sim(8, 2, [[1, 2, 3]])
+
+
+def test_global_lru_vs_brute_force_on_the_interleaved_trace():
+    r = random.Random(7)
+    L, E, n_slots = 3, 16, 9
+    routed = [[sorted(set(min(E - 1, int(r.paretovariate(1.0)) - 1 + r.randint(0, 3)) for _ in range(r.randint(1, 3))))
+               for _ in range(40)] for _ in range(L)]
+    hits, misses, slots = oracle.lru_sim_global(L, E, n_slots, routed)
+    flat = [[l * E + e for e in routed[l][s]] for s in range(40) for l in range(L)]
+    bslot, bhit, bslots = _brute_lru(L * E, n_slots, flat)
+    for l in range(L):
+        assert hits[l] == sum(sum(bhit[i]) for i in range(l, len(flat), L))
+        assert misses[l] == sum(len(bhit[i]) - sum(bhit[i]) for i in range(l, len(flat), L))
+    assert slots == bslots
+
+
+def test_global_lru_one_layer_is_the_per_layer_cache():
+    steps = [[3, 1], [1], [5], [3], [2, 5], [1, 3]]
+    _, hit, se, h, m = oracle.lru_sim(8, 2, steps)
+    gh, gm, gs = oracle.lru_sim_global(1, 8, 2, [steps])
+    assert (gh[0], gm[0]) == (h, m) and gs == se[-1].tolist()
+
+
+def test_global_lru_worked_example():
+    # layer 0 cycles through experts 0, 1, 2; layer 1 always uses expert 0.  Two slots per
+    # layer: layer 0's own LRU misses on every step (three ids round-robin through two
+    # slots).  Pooled (4 slots): after the first three steps everything is resident.
+    n = 12
+    routed = [[[s % 3] for s in range(n)], [[0] for _ in range(n)]]
+    ph0, pm0 = oracle.lru_sim(4, 2, routed[0])[3:5]
+    ph1, pm1 = oracle.lru_sim(4, 2, routed[1])[3:5]
+    assert (ph0, pm0, ph1, pm1) == (0, n, n - 1, 1)
+    gh, gm, gs = oracle.lru_sim_global(2, 4, 4, routed)
+    assert gm == [3, 1] and gh == [n - 3, n - 1]
+    assert sorted(gs) == [0, 1, 2, 4]          # keys: layer 0 experts 0-2, layer 1 expert 0
+
+
+def test_global_lru_compulsory_misses_only_when_everything_fits():
+    r = random.Random(3)
+    L, E = 4, 8
+    routed = [[sorted(set(r.randrange(E) for _ in range(3))) for _ in range(25)] for _ in range(L)]
+    distinct = [len(set(e for st in routed[l] for e in st)) for l in range(L)]
+    hits, misses, _ = oracle.lru_sim_global(L, E, L * E, routed)
+    assert misses == distinct
+    assert [h + m for h, m in zip(hits, misses)] == [sum(len(st) for st in routed[l]) for l in range(L)]
