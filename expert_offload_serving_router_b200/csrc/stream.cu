@@ -70,6 +70,44 @@ extern "C" ft_status ft_lru_step(int32_t E, int32_t n_slots, int32_t* content, i
     return FT_OK;
 }
 
+extern "C" ft_status ft_lru_resize(int32_t E, int32_t n_old, int32_t n_new, int32_t* content, int64_t* stamp,
+                                   int32_t* where, int32_t* move_from, int32_t* move_to, int32_t* n_moves) {
+    if (E <= 0 || n_old <= 0 || n_new <= 0 || !content || !stamp || !where || !n_moves ||
+        (n_new < n_old && (!move_from || !move_to)))
+        return fail(FT_ERR_INVALID_ARG, "ft_lru_resize: bad arguments");
+    *n_moves = 0;
+    if (n_new >= n_old) {                          // grow: new slots start empty
+        for (int i = n_old; i < n_new; ++i) { content[i] = -1; stamp[i] = -1; }
+        return FT_OK;
+    }
+    // shrink: keep the n_new most recently used experts (stamps are unique)
+    std::vector<int> occ;
+    for (int i = 0; i < n_old; ++i)
+        if (content[i] >= 0) occ.push_back(i);
+    std::sort(occ.begin(), occ.end(), [&](int a, int b) { return stamp[a] > stamp[b]; });
+    for (size_t r = size_t(n_new); r < occ.size(); ++r) {
+        const int i = occ[r];
+        where[content[i]] = -1;
+        content[i] = -1;
+        stamp[i] = -1;
+    }
+    // survivors above the new count move, in ascending old slot, to the lowest empty slot
+    int free_slot = 0;
+    for (int i = n_new; i < n_old; ++i) {
+        if (content[i] < 0) continue;
+        while (content[free_slot] >= 0) ++free_slot;   // exists: at most n_new survivors
+        content[free_slot] = content[i];
+        stamp[free_slot] = stamp[i];
+        where[content[i]] = free_slot;
+        move_from[*n_moves] = i;
+        move_to[*n_moves] = free_slot;
+        ++*n_moves;
+        content[i] = -1;
+        stamp[i] = -1;
+    }
+    return FT_OK;
+}
+
 struct LayerCache {
     std::vector<int32_t> content;   // [slots] expert id (global pool: layer * E + expert) or -1
     std::vector<int64_t> stamp;     // [slots]
@@ -81,6 +119,7 @@ struct ft_expert_stream {
     ft_stream_cfg cfg;
     std::vector<ft_moe_weights> host;
     int L, S, E, k;
+    int S_max;                      // slots per layer the arena holds (cfg.slots_per_layer)
     size_t b13, b13s, b2, b2s, expert_bytes, layer_bytes;
     uint8_t* buf[2];
     uint8_t* slots;                 // [L][S] expert slots, each [w13 | w13s | w2 | w2s]
@@ -181,6 +220,7 @@ ft_status ft_expert_stream_create(const ft_stream_cfg* cfg, ft_expert_stream** o
     st->cfg.host_layers = st->host.data();
     st->L = cfg->num_layers;
     st->S = cfg->slots_per_layer;
+    st->S_max = cfg->slots_per_layer;
     st->E = E;
     st->k = k;
     expert_sizes(cfg->shape, st->b13, st->b13s, st->b2, st->b2s);
@@ -190,7 +230,7 @@ ft_status ft_expert_stream_create(const ft_stream_cfg* cfg, ft_expert_stream** o
     st->buf[0] = base;
     st->buf[1] = base + st->layer_bytes;
     st->slots = base + 2 * st->layer_bytes;
-    st->dtable = reinterpret_cast<void**>(st->slots + size_t(st->L) * st->S * st->expert_bytes);
+    st->dtable = reinterpret_cast<void**>(st->slots + size_t(st->L) * st->S_max * st->expert_bytes);
     st->timeout_ms = cfg->host_wait_timeout_ms > 0 ? cfg->host_wait_timeout_ms : 10000;
     st->global = cfg->cache_policy == FT_CACHE_GLOBAL;
     reset_slots(st);
@@ -383,7 +423,7 @@ ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const voi
         uint64_t bytes = 0, nmiss = 0;
         for (size_t i = 0; i < ids.size(); ++i) {
             const int u = ids[i];
-            uint8_t* sp = s->slots + ((s->global ? 0 : size_t(l) * s->S) + slot[i]) * s->expert_bytes;
+            uint8_t* sp = s->slots + ((s->global ? 0 : size_t(l) * s->S_max) + slot[i]) * s->expert_bytes;
             uint8_t* p13 = sp;
             uint8_t* p13s = sp + a256(s->b13);
             uint8_t* p2 = p13s + a256(s->b13s);
@@ -481,6 +521,56 @@ ft_status ft_expert_stream_reset_cache(ft_expert_stream* s) {
     reset_slots(s);
     s->copy_count = 0;
     return FT_OK;
+}
+
+ft_status ft_expert_stream_set_slots(ft_expert_stream* s, int32_t slots_per_layer, void* compute_stream,
+                                     void* copy_stream) {
+    if (!s) return fail(FT_ERR_INVALID_ARG, "stream handle is NULL");
+    if (slots_per_layer < s->k || slots_per_layer > s->S_max)
+        return fail(FT_ERR_INVALID_ARG, "slots_per_layer %d must be in [k=%d, %d (arena)]", slots_per_layer, s->k,
+                    s->S_max);
+    if (slots_per_layer == s->S) return FT_OK;
+    ft_status st = cuda_state();
+    if (st) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(compute_stream), ps = static_cast<cudaStream_t>(copy_stream);
+    // the policy state: one per layer, or the pool (every layer's slots, layer-major)
+    const int n_caches = s->global ? 1 : s->L;
+    const int per = s->global ? s->L : 1;                     // slot counts scale by this
+    std::vector<std::vector<int32_t>> from(static_cast<size_t>(n_caches)), to(static_cast<size_t>(n_caches));
+    std::vector<int32_t> nmov(size_t(n_caches), 0);
+    for (int q = 0; q < n_caches; ++q) {
+        LayerCache& c = s->global ? s->pool : s->cache[size_t(q)];
+        const int n_old = per * s->S, n_new = per * slots_per_layer;
+        const int32_t keys = s->global ? s->L * s->E : s->E;
+        c.content.resize(size_t(std::max(n_old, n_new)), -1);
+        c.stamp.resize(size_t(std::max(n_old, n_new)), -1);
+        from[size_t(q)].resize(size_t(n_old));
+        to[size_t(q)].resize(size_t(n_old));
+        if ((st = ft_lru_resize(keys, n_old, n_new, c.content.data(), c.stamp.data(), c.where.data(),
+                                from[size_t(q)].data(), to[size_t(q)].data(), &nmov[size_t(q)])))
+            return st;
+        c.content.resize(size_t(n_new));
+        c.stamp.resize(size_t(n_new));
+    }
+    s->S = slots_per_layer;
+    // relocate the kept experts once every kernel already enqueued on the compute stream (which
+    // may still read the old slots) is done; the next step's kernels wait for the copies
+    bool any = false;
+    for (int32_t n : nmov) any = any || n > 0;
+    if (!any) return FT_OK;
+    if ((st = cuda_ok(cudaEventRecord(s->ids_ev, cs), "record compute"))) return st;
+    if ((st = cuda_ok(cudaStreamWaitEvent(ps, s->ids_ev, 0), "wait compute"))) return st;
+    for (int q = 0; q < n_caches; ++q) {
+        uint8_t* base = s->slots + (s->global ? 0 : size_t(q) * s->S_max) * s->expert_bytes;
+        for (int m = 0; m < nmov[size_t(q)]; ++m) {
+            cudaError_t e = cudaMemcpyAsync(base + size_t(to[size_t(q)][size_t(m)]) * s->expert_bytes,
+                                            base + size_t(from[size_t(q)][size_t(m)]) * s->expert_bytes,
+                                            s->expert_bytes, cudaMemcpyDeviceToDevice, ps);
+            if (e != cudaSuccess) return cuda_ok(e, "slot relocation copy");
+        }
+    }
+    if ((st = cuda_ok(cudaEventRecord(s->copy_ev, ps), "record relocation"))) return st;
+    return cuda_ok(cudaStreamWaitEvent(cs, s->copy_ev, 0), "wait relocation");
 }
 
 ft_status ft_expert_stream_inject_copy_failure(ft_expert_stream* s, int64_t n) {

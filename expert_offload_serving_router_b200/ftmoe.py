@@ -78,9 +78,11 @@ _SIGS = {
     "ft_expert_stream_stats": (c_i32, [c_vp, c_i32, ctypes.POINTER(c_u64)]),
     "ft_expert_stream_slots": (c_i32, [c_vp, c_i32, ctypes.POINTER(c_i32)]),
     "ft_expert_stream_reset_cache": (c_i32, [c_vp]),
+    "ft_expert_stream_set_slots": (c_i32, [c_vp, c_i32, c_vp, c_vp]),
     "ft_expert_stream_destroy": (None, [c_vp]),
     "ft_expert_stream_inject_copy_failure": (c_i32, [c_vp, c_i64]),
     "ft_lru_step": (c_i32, [c_i32, c_i32, c_vp, c_vp, c_vp, c_i64, c_vp, c_i32, c_vp, c_vp]),
+    "ft_lru_resize": (c_i32, [c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
 }
 
 
@@ -229,6 +231,17 @@ def ft_lru_step(E, n_slots, content, stamp, where, step, ids, out_slot, out_hit)
     _check(lib().ft_lru_step(E, n_slots, P(content), P(stamp), P(where), step, P(ids), len(ids), P(out_slot), P(out_hit)))
 
 
+def ft_lru_resize(E, n_old, n_new, content, stamp, where):
+    """Host-only resize of one LRU state (numpy int32 content/where, int64 stamp, each with room
+    for max(n_old, n_new) slots).  Returns the list of (from, to) slot moves."""
+    P = lambda a: a.ctypes.data_as(c_vp)
+    mf = (c_i32 * max(1, n_old))()
+    mt = (c_i32 * max(1, n_old))()
+    nm = c_i32()
+    _check(lib().ft_lru_resize(E, n_old, n_new, P(content), P(stamp), P(where), mf, mt, ctypes.byref(nm)))
+    return [(mf[i], mt[i]) for i in range(nm.value)]
+
+
 # ---------------------------------------------------------------- expert stream
 def ft_expert_stream_arena_bytes(cfg: ft_stream_cfg) -> int:
     return lib().ft_expert_stream_arena_bytes(ctypes.byref(cfg))
@@ -277,6 +290,10 @@ def ft_expert_stream_slots(handle, layer: int, n_slots: int) -> list[int]:
 
 def ft_expert_stream_reset_cache(handle):
     _check(lib().ft_expert_stream_reset_cache(handle))
+
+
+def ft_expert_stream_set_slots(handle, slots_per_layer: int, compute_stream=None, copy_stream=None):
+    _check(lib().ft_expert_stream_set_slots(handle, slots_per_layer, _s(compute_stream), _s(copy_stream)))
 
 
 def ft_expert_stream_destroy(handle):

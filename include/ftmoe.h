@@ -296,6 +296,19 @@ ft_status ft_expert_stream_slots(const ft_expert_stream* s, int32_t layer, int32
 /* Empties every slot (next decode step starts cold) and zeroes the counters. */
 ft_status ft_expert_stream_reset_cache(ft_expert_stream* s);
 
+/* Elastic slot budget (FreeToken article, dothoosh.com, "FreeToken architecture",
+ * mechanism 3: the GPU expert cache is rebuilt under a new VRAM budget at a safe point,
+ * without restarting or reloading the host set).  Call between decode steps.  New
+ * count in [k, cfg.slots_per_layer] (the arena was sized for cfg's count).  Growing adds
+ * empty slots.  Shrinking keeps each cache's most recently used experts (per layer: the
+ * slots_per_layer newest; global: num_layers * slots_per_layer newest), drops the rest,
+ * and moves kept experts that sit above the new count into the lowest empty slots
+ * (ascending old slot; ft_lru_resize).  The moves are device-to-device copies on
+ * copy_stream, ordered after all work already enqueued on compute_stream and before
+ * anything enqueued on it later.  Counters are kept. */
+ft_status ft_expert_stream_set_slots(ft_expert_stream* s, int32_t slots_per_layer, void* compute_stream,
+                                     void* copy_stream);
+
 void ft_expert_stream_destroy(ft_expert_stream* s);
 
 /* The host-side LRU policy of one layer's slot cache, one decode step (the
@@ -312,6 +325,16 @@ void ft_expert_stream_destroy(ft_expert_stream* s);
  * (decode step * num_layers + layer). */
 ft_status ft_lru_step(int32_t E, int32_t n_slots, int32_t* content, int64_t* stamp, int32_t* where,
                       int64_t step, const int32_t* ids, int32_t n, int32_t* out_slot, uint8_t* out_hit);
+
+/* Resize of one LRU cache state from n_old to n_new slots (host only, no CUDA call; the
+ * policy ft_expert_stream_set_slots applies).  content/stamp need room for
+ * max(n_old, n_new) entries; where[E].  Growing: slots n_old..n_new-1 become empty.
+ * Shrinking: the n_new occupied slots with the largest stamps are kept, the others
+ * emptied (where = -1); then every kept expert in a slot >= n_new, in ascending slot
+ * order, moves to the lowest empty slot < n_new; the moves are written to
+ * move_from[i] -> move_to[i], i < *n_moves (capacity n_old). */
+ft_status ft_lru_resize(int32_t E, int32_t n_old, int32_t n_new, int32_t* content, int64_t* stamp, int32_t* where,
+                        int32_t* move_from, int32_t* move_to, int32_t* n_moves);
 
 /* Test hook for failure handling: make the n-th host->device expert copy
  * enqueue (counting from 1 after this call) report failure (n = 0 disables).

@@ -202,6 +202,94 @@ def lru_sim_global(num_layers: int, num_experts: int, n_slots: int, routed):
     return hits, misses, (se[-1].tolist() if len(flat) else [-1] * n_slots)
 
 
+def lru_resize(content, stamp, where, n_new):
+    """Slot budget change of one LRU cache state (lists content/stamp, dict where), in place.
+    Growing appends empty slots.  Shrinking keeps the n_new occupied slots used most recently
+    (largest stamps), empties the rest, then moves each kept expert that sits at slot >= n_new,
+    in ascending slot order, to the lowest empty slot below n_new.  Returns the moves
+    [(from, to)].  (Elastic expert cache rebuilt under a new VRAM budget at a safe point:
+    FreeToken article, dothoosh.com, "FreeToken architecture", mechanism 3.)"""
+    n_old = len(content)
+    if n_new >= n_old:
+        content.extend([-1] * (n_new - n_old))
+        stamp.extend([-1] * (n_new - n_old))
+        return []
+    occupied = [i for i in range(n_old) if content[i] >= 0]
+    occupied.sort(key=lambda i: -stamp[i])
+    for i in occupied[n_new:]:
+        del where[content[i]]
+        content[i], stamp[i] = -1, -1
+    moves = []
+    for i in range(n_new, n_old):
+        if content[i] < 0:
+            continue
+        j = content.index(-1)
+        content[j], stamp[j] = content[i], stamp[i]
+        where[content[j]] = j
+        content[i], stamp[i] = -1, -1
+        moves.append((i, j))
+    del content[n_new:]
+    del stamp[n_new:]
+    return moves
+
+
+def _lru_run(num_keys: int, n_slots: int, steps, resize_before):
+    """The decode LRU policy (as lru_sim) in plain Python over policy steps, with slot-budget
+    changes {policy step: new slot count} applied before the given steps."""
+    content, stamp, where = [-1] * n_slots, [-1] * n_slots, {}
+    slots_out, hits_out = [], []
+    for s, step in enumerate(steps):
+        if s in resize_before:
+            lru_resize(content, stamp, where, resize_before[s])
+        ids = sorted(set(int(i) for i in step))
+        if len(ids) > len(content) or any(u < 0 or u >= num_keys for u in ids):
+            raise ValueError("step larger than the slot count or id out of range")
+        touched, sl, hit = set(), [None] * len(ids), [False] * len(ids)
+        for r, u in enumerate(ids):
+            if u in where:
+                touched.add(where[u])
+                stamp[where[u]] = s * num_keys + r
+                sl[r], hit[r] = where[u], True
+        for r, u in enumerate(ids):
+            if hit[r]:
+                continue
+            if -1 in content:
+                v = content.index(-1)
+            else:
+                v = min((i for i in range(len(content)) if i not in touched), key=lambda i: stamp[i])
+                del where[content[v]]
+            content[v], stamp[v], where[u] = u, s * num_keys + r, v
+            touched.add(v)
+            sl[r] = v
+        slots_out.append(sl)
+        hits_out.append(hit)
+    return slots_out, hits_out, content
+
+
+def lru_sim_resizable(num_experts: int, n_slots: int, steps, resize_before=None):
+    """Per-layer cache with slot-budget changes {decode step: new slots} before those steps.
+    Returns (slot, hit, final content, hits, misses)."""
+    sl, hit, content = _lru_run(num_experts, n_slots, steps, dict(resize_before or {}))
+    h = sum(sum(x) for x in hit)
+    return sl, hit, content, h, sum(len(x) for x in hit) - h
+
+
+def lru_sim_global_resizable(num_layers: int, num_experts: int, slots_per_layer: int, routed, resize_before=None):
+    """Global cache (num_layers * slots_per_layer slots, keys layer * E + expert) with budget
+    changes {decode step: new slots per layer} before layer 0 of those steps.  Returns
+    (per-layer hits, per-layer misses, final content)."""
+    L, E = num_layers, num_experts
+    n_steps = len(routed[0])
+    flat = [[l * E + int(e) for e in routed[l][s]] for s in range(n_steps) for l in range(L)]
+    rb = {s * L: L * n for s, n in (resize_before or {}).items()}
+    _, hit, content = _lru_run(L * E, L * slots_per_layer, flat, rb)
+    hits, misses = [0] * L, [0] * L
+    for i, h in enumerate(hit):
+        hits[i % L] += sum(h)
+        misses[i % L] += len(h) - sum(h)
+    return hits, misses, content
+
+
 def full_layer(shape: dict, x_bits, w_router, bias, weights: dict, logits32=None, tokens=None, n_threads: int = 0):
     """Convenience: logits (fp64) -> top-k on the given fp32 logits (or on the fp64 logits
     rounded to fp32 when none are given) -> y for the listed tokens."""

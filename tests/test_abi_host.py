@@ -187,3 +187,29 @@ def test_host_lru_policy_as_global_pool_matches_oracle():
             misses[l] += len(keys) - int(out_hit.sum())
     assert (hits, misses) == (oh, om)
     assert content.tolist() == oslots
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_host_lru_resize_matches_oracle(seed):
+    r = random.Random(300 + seed)
+    E = 64
+    n_old = r.randint(1, 12)
+    n_new = r.randint(1, 16)
+    ids = r.sample(range(E), n_old)
+    stamps = r.sample(range(1000), n_old)
+    occ = [r.random() < 0.75 for _ in range(n_old)]
+    content = [e if o else -1 for e, o in zip(ids, occ)]
+    stamp = [t if o else -1 for t, o in zip(stamps, occ)]
+    where = {e: i for i, e in enumerate(content) if e >= 0}
+    oc, os_, ow = list(content), list(stamp), dict(where)
+    omoves = oracle.lru_resize(oc, os_, ow, n_new)
+    cap = max(n_old, n_new)
+    c = np.full(cap, -1, np.int32); c[:n_old] = content
+    st = np.full(cap, -1, np.int64); st[:n_old] = stamp
+    w = np.full(E, -1, np.int32)
+    for e, i in where.items():
+        w[e] = i
+    moves = F.ft_lru_resize(E, n_old, n_new, c, st, w)
+    assert moves == omoves
+    assert c[:n_new].tolist() == oc and st[:n_new].tolist() == os_
+    assert {e: int(w[e]) for e in range(E) if w[e] >= 0} == ow

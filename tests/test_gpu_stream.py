@@ -143,6 +143,46 @@ def test_global_cache_follows_oracle_global_lru_and_equals_resident():
         g.close()
 
 
+@pytest.mark.parametrize("policy", [F.FT_CACHE_PER_LAYER, F.FT_CACHE_GLOBAL])
+def test_slot_budget_change_between_steps(policy):
+    """Shrink the budget to the minimum (k slots per layer) and grow it back between decode
+    steps: results stay equal to the resident layers, hits/misses and slot contents follow the
+    oracle's resizable LRU."""
+    g = Stack(cache_policy=policy)
+    try:
+        steps, k = 30, g.cfg.top_k
+        resize = {10: k, 20: SLOTS}
+        routed = [[] for _ in range(NL)]
+        for s in range(steps):
+            if s in resize:
+                F.ft_expert_stream_set_slots(g.handle, resize[s], copy_stream=g.copy_stream)
+            x = inputs.make_tokens(g.cfg, 1, seed=15, stream=s)
+            y, xl = g.run("decode", x)
+            for l, L in enumerate(g.layers):
+                yr, idx, lg = _resident(L, xl[l])
+                assert np.array_equal(y[l], yr), f"step {s} layer {l}: result after budget change != resident"
+                routed[l].append(sorted(set(idx.ravel().tolist())))
+        E = g.cfg.num_experts
+        if policy == F.FT_CACHE_GLOBAL:
+            oh, om, oc = oracle.lru_sim_global_resizable(NL, E, SLOTS, routed, resize)
+            assert F.ft_expert_stream_slots(g.handle, -1, NL * SLOTS) == oc
+        else:
+            oh, om = [], []
+            for l in range(NL):
+                _, _, oc, h, m = oracle.lru_sim_resizable(E, SLOTS, routed[l], resize)
+                oh.append(h)
+                om.append(m)
+                assert F.ft_expert_stream_slots(g.handle, l, SLOTS) == oc
+        for l in range(NL):
+            st = F.ft_expert_stream_stats(g.handle, l)
+            assert (st[0], st[1]) == (oh[l], om[l])
+        with pytest.raises(F.FtError) as ei:      # beyond what the arena holds
+            F.ft_expert_stream_set_slots(g.handle, SLOTS + 1, copy_stream=g.copy_stream)
+        assert ei.value.status == F.FT_ERR_INVALID_ARG
+    finally:
+        g.close()
+
+
 def test_injected_copy_failure_is_reported_and_rolled_back(stack):
     F.ft_expert_stream_reset_cache(stack.handle)
     x0 = inputs.make_tokens(stack.cfg, 1, seed=13, stream=0)

@@ -362,3 +362,43 @@ def test_global_lru_compulsory_misses_only_when_everything_fits():
     hits, misses, _ = oracle.lru_sim_global(L, E, L * E, routed)
     assert misses == distinct
     assert [h + m for h, m in zip(hits, misses)] == [sum(len(st) for st in routed[l]) for l in range(L)]
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_python_lru_run_equals_c_simulator(seed):
+    r = random.Random(40 + seed)
+    E, n_slots = r.choice([(8, 3), (32, 8), (256, 32)])
+    steps = [[min(E - 1, int(r.paretovariate(1.0)) - 1 + r.randint(0, 2)) for _ in range(r.randint(0, min(6, n_slots)))]
+             for _ in range(50)]
+    cslot, chit, cse, ch, cm = oracle.lru_sim(E, n_slots, steps)
+    pslot, phit, pcontent, ph, pm = oracle.lru_sim_resizable(E, n_slots, steps)
+    assert (pslot, phit, ph, pm) == (cslot, chit, ch, cm)
+    assert pcontent == cse[-1].tolist()
+    routed = [steps[i::3] for i in range(3)]
+    n = min(len(x) for x in routed)
+    routed = [x[:n] for x in routed]
+    assert oracle.lru_sim_global_resizable(3, E, n_slots, routed)[:2] == tuple(oracle.lru_sim_global(3, E, 3 * n_slots, routed)[:2])
+
+
+def test_lru_resize_worked_example():
+    # four slots holding experts 7, 3, 5, 9 last used at stamps 40, 10, 30, 20; shrink to two:
+    # keep the two newest (7 @ 40 in slot 0, 5 @ 30 in slot 2), drop 3 and 9, move 5 to slot 1
+    content, stamp = [7, 3, 5, 9], [40, 10, 30, 20]
+    where = {7: 0, 3: 1, 5: 2, 9: 3}
+    assert oracle.lru_resize(content, stamp, where, 2) == [(2, 1)]
+    assert content == [7, 5] and stamp == [40, 30] and where == {7: 0, 5: 1}
+    # grow back to four: two empty slots, the next misses fill the lowest empty slot first
+    assert oracle.lru_resize(content, stamp, where, 4) == []
+    assert content == [7, 5, -1, -1]
+    # a trace: step 0 puts 1, 2 in slots 0, 1; step 1 puts 5, 6 in slots 2, 3; shrinking to two
+    # keeps 5 and 6 (newest) and moves them to slots 0 and 1; step 2: 6 hits, 7 replaces the
+    # untouched 5; growing to three adds slot 2, which step 3's miss (5) takes
+    slot, hit, final, h, m = oracle.lru_sim_resizable(16, 4, [[1, 2], [5, 6], [6, 7], [5]], {2: 2, 3: 3})
+    assert slot == [[0, 1], [2, 3], [1, 0], [2]]
+    assert hit == [[False, False], [False, False], [True, False], [False]]
+    assert final == [7, 6, 5] and (h, m) == (1, 6)
+
+
+def test_lru_resize_rejects_a_step_larger_than_the_new_budget():
+    with pytest.raises(ValueError):
+        oracle.lru_sim_resizable(16, 4, [[1, 2], [1, 3, 4], [4]], {1: 2})
