@@ -148,6 +148,19 @@ def cpu_baseline(cfg, layer_np, budget_s=15.0):
                       f"{dt:.1f} s)"}
 
 
+def max_over_ranks(torch, dist, ms, device="cuda"):
+    """The slowest replica's device-timed milliseconds, returned on every rank."""
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, tokens_per_rank, ms_max):
+    """Whole-job throughput of `world` replicas that each process tokens_per_rank tokens per
+    step, timed by the slowest one (weak scaling: per-GPU work is fixed)."""
+    return world * tokens_per_rank / (ms_max * 1e-3)
+
+
 def run_reference(args, rank):
     """Reference arm: the fp64 CPU oracle, as it stands, on the host cores."""
     if rank != 0:
@@ -379,10 +392,8 @@ def measure_e2e(torch, dist, F, L, ctx, T, steps, warmup, world):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": world * T / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+        ms = max_over_ranks(torch, dist, ms)
+    return {"value": job_tokens_per_s(world, T, ms), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
             "d2h_bytes_per_step": T * H * 2, "ms_per_step": ms}
 
 
@@ -574,11 +585,9 @@ def main():
     pre = measure_prefill(torch, F, L, T, args.steps, args.warmup, torch.cuda.current_stream(), rank, local)
     ms_step = pre["ms_step"]
     if world > 1:
-        t = torch.tensor([ms_step], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+        ms_step = max_over_ranks(torch, dist, ms_step)
         dist.barrier()
-    value = world * T / (ms_step * 1e-3)
+    value = job_tokens_per_s(world, T, ms_step)
     tc_peak = tc_sus if pre["total_ms"] > 1000.0 else tc_burst
     traffic = recorded_traffic("moe_gemm_gateup_qwen3_a3b_T4096.md", "gemm_sm100.cu")
     e2e = None if args.no_e2e else measure_e2e(torch, dist, F, L, pre["ctx"], T, args.steps, args.warmup, world)
