@@ -205,7 +205,6 @@ __global__ void __launch_bounds__(256, 2) decode_down_bulk_kernel(DecodeArgs a, 
     }
     pdl_wait();   // h from the gate/up kernel
     const int gpr = RPB / 4;
-    const int nvec = MX ? F / 32 : F / 8;       // 16-byte weight vectors per row
     for (int it = warp; it < n_active * gpr; it += 8) {
         const int slot = it / gpr, j0 = 4 * (it - slot * gpr);
         if (!mbar_wait(&full[slot], 0, nullptr)) { s_bad = 1; continue; }

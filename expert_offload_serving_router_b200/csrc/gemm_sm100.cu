@@ -31,7 +31,6 @@ namespace ftmoe {
 
 constexpr int kBK = 64;                        // K per stage (one 128-byte swizzle atom of bf16)
 constexpr int kAHalfBytes = 128 * kBK * 2;     // 16 KB: one 128-row MMA operand
-constexpr int kATileBytes = 2 * kAHalfBytes;   // 32 KB: 256 weight rows per tile
 constexpr int kBTileBytes = kGemmBN * kBK * 2; // 32 KB: up to 256 token rows
 constexpr int kAccCols = 256;                  // one accumulator = 128 lanes x 256 fp32 columns
 constexpr int kNumBMaps = 5;                   // activation boxes of 16, 32, 64, 128, 256 rows
@@ -117,6 +116,72 @@ __device__ __forceinline__ int bmap_index(int n) {   // smallest box of 16 << i 
     int i = 0;
     while (i < kNumBMaps - 1 && (16 << i) < n) ++i;
     return i;
+}
+
+// Epilogue of one tile for one warp: TMEM lanes 32q..32q+31 (tbase already includes them
+// and the accumulator buffer), accumulator half hh at column hh * kAccCols, weight-row group
+// rg_base + rg_step * hh; this warp takes 32-column chunks part, part + kParts, ...  Two chunks
+// are loaded per tcgen05.wait, each transposed through the warp's 2 KB buffer xb so the global
+// stores are 16-byte vectors along the token row (gate/up: SwiGLU of the interleaved halves).
+template <int kParts>
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, const Tile& tl, int halves, uint32_t tbase,
+                                              int rg_base, int rg_step, int q, int part, int lane, uint16_t* xb) {
+    const int nch = (tl.nvalid + 31) >> 5;
+    const int per_half = (nch - part + kParts - 1) / kParts;   // chunks c = part, part + kParts, ...
+    const int items = halves * per_half;
+    for (int it = 0; it < items; it += 2) {
+        float v[2][32];
+        int hh[2], cc[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int iu = it + u < items ? it + u : it;
+            hh[u] = iu / per_half;
+            cc[u] = part + kParts * (iu - hh[u] * per_half);
+            tmem_ld32_nowait(tbase + uint32_t(hh[u] * kAccCols + cc[u] * 32), v[u]);
+        }
+        tmem_wait_ld(v[0], v[1]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (it + u >= items) break;
+            const int c = cc[u], rg = rg_base + rg_step * hh[u];
+            if (p.mode == 0) {
+                const int fl = lane & 15;
+                const bool lo = lane < 16;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float send = lo ? v[u][16 + i] : v[u][i];
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+                    const float gt = lo ? v[u][i] : recv;
+                    const float up = lo ? recv : v[u][16 + i];
+                    xb[(lo ? i : 16 + i) * 16 + fl] = f2bf(silu_mul(gt, up));
+                }
+                __syncwarp();
+                const int fbase = rg * 64 + 16 * q;
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int ch = lane + 32 * r, tok = ch >> 1, pp = ch & 1;
+                    const int n = c * 32 + tok;
+                    if (n < tl.nvalid)
+                        *reinterpret_cast<uint4*>(p.out + size_t(tl.row0 + n) * p.out_ld + fbase + 8 * pp) =
+                            *reinterpret_cast<const uint4*>(xb + tok * 16 + 8 * pp);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) xb[j * 32 + lane] = f2bf(v[u][j]);
+                __syncwarp();
+                const int hbase = rg * 128 + 32 * q;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int ch = lane + 32 * r, tok = ch >> 2, pp = ch & 3;
+                    const int n = c * 32 + tok;
+                    if (n < tl.nvalid)
+                        *reinterpret_cast<uint4*>(p.out + size_t(tl.row0 + n) * p.out_ld + hbase + 8 * pp) =
+                            *reinterpret_cast<const uint4*>(xb + tok * 32 + 8 * pp);
+                }
+            }
+            __syncwarp();
+        }
+    }
 }
 
 // HV = 2: 256 weight rows per tile, both TMEM accumulators belong to one tile (single
@@ -276,63 +341,8 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
             const Tile tl = decode_tile<HV>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
             if (!mbar_wait(&tfull[buf], acc_phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const int nch = (tl.nvalid + 31) >> 5;
-            const int per_half = (nch - part + kParts - 1) / kParts;   // chunks c = part, part + kParts, ...
-            const int items = tl.halves * per_half;
-            for (int it = 0; it < items; it += 2) {
-                float v[2][32];
-                int hh[2], cc[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int iu = it + u < items ? it + u : it;
-                    hh[u] = iu / per_half;
-                    cc[u] = part + kParts * (iu - hh[u] * per_half);
-                    tmem_ld32_nowait(tmem_base + (uint32_t(q * 32) << 16) + uint32_t((buf * HV + hh[u]) * kAccCols + cc[u] * 32),
-                                     v[u]);
-                }
-                tmem_wait_ld(v[0], v[1]);
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    if (it + u >= items) break;
-                    const int c = cc[u], rg = tl.m * HV + hh[u];
-                    if (p.mode == 0) {
-                        const int fl = lane & 15;
-                        const bool lo = lane < 16;
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float send = lo ? v[u][16 + i] : v[u][i];
-                            const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-                            const float gt = lo ? v[u][i] : recv;
-                            const float up = lo ? recv : v[u][16 + i];
-                            xb[(lo ? i : 16 + i) * 16 + fl] = f2bf(silu_mul(gt, up));
-                        }
-                        __syncwarp();
-                        const int fbase = rg * 64 + 16 * q;
-#pragma unroll
-                        for (int r = 0; r < 2; ++r) {
-                            const int ch = lane + 32 * r, tok = ch >> 1, pp = ch & 1;
-                            const int n = c * 32 + tok;
-                            if (n < tl.nvalid)
-                                *reinterpret_cast<uint4*>(p.out + size_t(tl.row0 + n) * p.out_ld + fbase + 8 * pp) =
-                                    *reinterpret_cast<const uint4*>(xb + tok * 16 + 8 * pp);
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) xb[j * 32 + lane] = f2bf(v[u][j]);
-                        __syncwarp();
-                        const int hbase = rg * 128 + 32 * q;
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const int ch = lane + 32 * r, tok = ch >> 2, pp = ch & 3;
-                            const int n = c * 32 + tok;
-                            if (n < tl.nvalid)
-                                *reinterpret_cast<uint4*>(p.out + size_t(tl.row0 + n) * p.out_ld + hbase + 8 * pp) =
-                                    *reinterpret_cast<const uint4*>(xb + tok * 32 + 8 * pp);
-                        }
-                    }
-                    __syncwarp();
-                }
-            }
+            epilogue_tile<kParts>(p, tl, tl.halves, tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * HV * kAccCols),
+                                  tl.m * HV, 1, q, part, lane, xb);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -420,6 +430,188 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(2 * kAccCols));
     }
+}
+
+// ------------------------------------------------------------------ CTA-pair gate/up (BF16)
+// Two CTAs of a cluster share every MMA (tcgen05.mma.cta_group::2, M = 256): CTA r supplies
+// 128 weight rows of each MMA and half of the token tile (rows r*N/2 .. of it) from its own
+// shared memory and keeps its 128 accumulator rows in its own TMEM.  A pair tile is 512
+// weight rows (two MMAs, four 128-row groups: CTA r holds groups 4m + r and 4m + 2 + r) x up
+// to 256 tokens.  Per SM a stage then carries 32 KB of weights and at most 16 KB of tokens
+// for the same MMA work as the single-CTA 256 x 256 tile's 64 KB, so four stages fit.
+// Only the leader (rank 0) waits for operands and issues MMAs: both CTAs' TMA copies count on
+// its `full` barrier, its commits arrive on the `empty` / `tfull` / `done` barriers of both
+// CTAs, and both CTAs' epilogue warps arrive on its `tempty` barrier.  No TMA multicast.
+constexpr int kPairSt = 4;
+constexpr int kPairATile = 2 * kAHalfBytes;            // 32 KB: two 128-row weight groups
+constexpr int kPairBTile = 128 * kBK * 2;              // 16 KB: up to 128 token rows
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+moe_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sw,
+                     const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
+                     const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_b3,
+                     const __grid_constant__ CUtensorMap tm_b4, GemmParams p) {
+    constexpr int kEpiWarps = 8;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kPairSt * kPairATile;
+    uint8_t* sX = sB + kPairSt * kPairBTile;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sX + kEpiWarps * kXposeBytes);
+    uint64_t* empty = full + kPairSt;
+    uint64_t* tfull = empty + kPairSt;
+    uint64_t* tempty = tfull + 1;
+    uint64_t* mma_done = tempty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* ntile_off = const_cast<int*>(reinterpret_cast<volatile int*>(tmem_slot + 2));
+    int* s_off = ntile_off + 260;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int cid = int(cluster_id_x()), ncl = int(cluster_count_x());
+    const int G = p.G;
+    for (int i = tid; i <= G; i += blockDim.x) {
+        ntile_off[i] = p.sched[2 + i];
+        s_off[i] = p.offsets[i];
+    }
+    if (tid == 0) {
+        for (int st = 0; st < kPairSt; ++st) {
+            mbar_init(&full[st], 1);            // the leader's producer arrives (with all bytes expected)
+            mbar_init(&empty[st], 1);           // the leader's MMA commit
+        }
+        mbar_init(tfull, 1);
+        mbar_init(tempty, 2 * kEpiWarps);       // every epilogue warp of both CTAs
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                     "r"(2 * kAccCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t full_lead = mapa_rank(su32(full), 0);      // the leader's full[0]
+    const uint32_t tempty_lead = mapa_rank(su32(tempty), 0);
+
+    const int total = ntile_off[G] * p.m_tiles;
+    const int nk = p.K / kBK;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            const CUtensorMap* bm[kNumBMaps] = {&tm_b0, &tm_b1, &tm_b2, &tm_b3, &tm_b4};
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued[kPairSt];
+            uint32_t issued_par[kPairSt];
+            for (int st = 0; st < kPairSt; ++st) issued[st] = 0;
+            bool ok = true;
+            for (int t = cid; t < total && ok; t += ncl) {
+                const Tile tl = decode_tile<4>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+                const bool shared_grp = p.has_shared && tl.g == p.E;
+                const int nh = ((tl.nvalid + 15) & ~15) >> 1;   // token rows per CTA
+                int bi = 0;
+                while (bi < kNumBMaps - 1 && (8 << bi) < nh) ++bi;
+                const uint32_t bbytes = uint32_t(p.b_rows[bi]) * kBK * 2;
+                const CUtensorMap* m = shared_grp ? &tm_sw : &tm_w;
+                const int e = shared_grp ? 0 : tl.g;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    uint8_t* a = sA + stage * kPairATile;
+                    uint8_t* b = sB + stage * kPairBTile;
+                    const int k0 = kb * kBK;
+                    const uint32_t bar = full_lead + uint32_t(stage) * 8u;
+                    if (rank == 0) mbar_expect_tx(&full[stage], 2u * (uint32_t(kPairATile) + bbytes));
+                    for (int h = 0; h < 2; ++h) {
+                        const int rg = tl.m * 4 + 2 * h + int(rank);
+                        tma_5d_pair(m, bar, a + h * kAHalfBytes, k0, 0, 0, rg * 4, e);
+                    }
+                    tma_2d_pair(bm[bi], bar, b, k0, tl.row0 + int(rank) * nh);
+                    issued[stage] = 1;
+                    issued_par[stage] = phase;
+                    if (++stage == kPairSt) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+            // drain: the leader sees its full barriers complete (both CTAs' bytes landed); the
+            // peer sees its empty barriers released (the leader consumed what it copied)
+            for (int st = 0; st < kPairSt; ++st)
+                if (issued[st]) {
+                    if (rank == 0) mbar_wait(&full[st], issued_par[st], nullptr);
+                    else mbar_wait(&empty[st], issued_par[st], nullptr);
+                }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (lane == 0) {
+            if (rank == 0) {
+                int stage = 0;
+                uint32_t phase = 0, acc_phase = 0;
+                bool ok = true;
+                for (int t = cid; t < total && ok; t += ncl) {
+                    const Tile tl = decode_tile<4>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+                    const int N = (tl.nvalid + 15) & ~15;
+                    const uint32_t idesc = idesc_bf16(256, N);
+                    if (!mbar_wait_cluster(tempty, acc_phase ^ 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int kb = 0; kb < nk; ++kb) {
+                        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint64_t bd = sdesc_sw128(su32(sB + stage * kPairBTile));
+                        for (int h = 0; h < 2; ++h) {
+                            const uint64_t ad = sdesc_sw128(su32(sA + stage * kPairATile + h * kAHalfBytes));
+                            const uint32_t dtm = tmem_base + uint32_t(h * kAccCols);
+#pragma unroll
+                            for (int kk = 0; kk < kBK / 16; ++kk)
+                                umma_bf16_pair(dtm, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+                        }
+                        umma_commit_pair_both(&empty[stage]);
+                        if (++stage == kPairSt) { stage = 0; phase ^= 1; }
+                    }
+                    if (!ok) break;
+                    umma_commit_pair_both(tfull);
+                    acc_phase ^= 1;
+                }
+                if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+                umma_commit_pair_both(mma_done);     // completion of every MMA issued above, in both CTAs
+            }
+            mbar_wait(mma_done, 0, nullptr);
+        }
+    } else if (warp < 2 + kEpiWarps) {
+        // ------------------------------------------------ epilogue (both CTAs, own 128 rows)
+        const int q = warp & 3;
+        const int part = (warp - 2) >> 2;
+        constexpr int kParts = kEpiWarps / 4;
+        uint16_t* xb = reinterpret_cast<uint16_t*>(sX + (warp - 2) * kXposeBytes);
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int t = cid; t < total; t += ncl) {
+            const Tile tl = decode_tile<4>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+            if (!mbar_wait(tfull, acc_phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            epilogue_tile<kParts>(p, tl, 2, tmem_base + (uint32_t(q * 32) << 16), tl.m * 4 + int(rank), 2, q, part,
+                                  lane, xb);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_lead);
+            acc_phase ^= 1;
+        }
+        if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
+    }
+    // teardown: every MMA of the pair is complete (mma_done) and both CTAs are past their last
+    // TMEM read and remote arrival before the pair's TMEM is freed and either CTA exits
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(2 * kAccCols));
 }
 
 // ------------------------------------------------------------------ host side
@@ -511,6 +703,42 @@ int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
     p.ws = L.wscale;
     p.swq = static_cast<const uint8_t*>(L.sw);
     p.sws = L.swscale;
+    if (!mx && L.mode == 0 && hv == 2 && p.m_rows % 4 == 0) {
+        // CTA pairs: each CTA loads half of a token tile, so the token boxes are 8 .. 128 rows
+        GemmParams pp = p;
+        pp.m_tiles = p.m_rows / 4;
+        CUtensorMap tbp[kNumBMaps]{};
+        const int rR8 = (L.R + 7) & ~7;
+        for (int i = 0; i < kNumBMaps; ++i) {
+            pp.b_rows[i] = (8 << i) < rR8 ? (8 << i) : rR8;
+            uint64_t dims[2] = {uint64_t(K), uint64_t(L.R)};
+            uint64_t str[1] = {uint64_t(K) * 2};
+            uint32_t box[2] = {kBK, uint32_t(pp.b_rows[i])};
+            if (!make_map(&tbp[i], L.act, 2, dims, str, box)) return 1;
+        }
+        static int max_clusters = 0;
+        const size_t smem = 1024 + size_t(kPairSt) * (kPairATile + kPairBTile) + 8 * kXposeBytes + 256 + 8 * 260;
+        if (!max_clusters) {
+            if (cudaFuncSetAttribute(moe_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+                cudaSuccess)
+                return 2;
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3(2 * (num_sms() / 2));
+            cfg.blockDim = dim3(320);
+            cfg.dynamicSmemBytes = smem;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, moe_gemm_pair_kernel, &cfg) != cudaSuccess || n <= 0) {
+                cudaGetLastError();
+                n = num_sms() / 2;
+            }
+            max_clusters = n;
+        }
+        int clusters = max_clusters;
+        const int pair_tiles = L.max_tiles * pp.m_tiles;
+        if (pair_tiles < clusters) clusters = pair_tiles > 0 ? pair_tiles : 1;
+        moe_gemm_pair_kernel<<<2 * clusters, 320, smem, st>>>(tw, tsw, tbp[0], tbp[1], tbp[2], tbp[3], tbp[4], pp);
+        return cudaGetLastError() == cudaSuccess ? 0 : 2;
+    }
     int grid = num_sms();
     const int max_tiles = L.max_tiles * p.m_tiles;
     if (max_tiles < grid) grid = max_tiles > 0 ? max_tiles : 1;

@@ -117,6 +117,81 @@ __device__ __forceinline__ void tmem_wait_ld(float (&a)[32], float (&b)[32]) {
     tmem_fence_regs(b + 16);
 }
 
+// ------------------------------------------------------------------ CTA pairs (cluster of 2)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_count_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+// every thread of both CTAs; orders the barrier initialisations before any remote arrival
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_acq_cluster(uint64_t* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(su32(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// bounded wait on a barrier that the peer CTA also arrives on
+static __device__ __noinline__ bool mbar_wait_cluster(uint64_t* b, uint32_t parity, volatile int* abort) {
+    if (mbar_try_acq_cluster(b, parity)) return true;
+    const uint64_t t0 = gtimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_acq_cluster(b, parity)) return true;
+        if ((i & 31) == 0) {
+            if (abort && *abort) return false;
+            if (gtimer() - t0 > kWaitNs) return false;
+        }
+    }
+}
+// TMA tile loads into this CTA's shared memory whose completion is counted on the pair
+// leader's barrier (cluster address): no multicast, each CTA fetches only its own tile.
+__device__ __forceinline__ void tma_2d_pair(const CUtensorMap* m, uint32_t bar_cluster, void* dst, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(su32(dst)), "l"(m), "r"(bar_cluster), "r"(c0), "r"(c1) : "memory");
+}
+__device__ __forceinline__ void tma_5d_pair(const CUtensorMap* m, uint32_t bar_cluster, void* dst, int c0, int c1, int c2,
+                                            int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        ::"r"(su32(dst)), "l"(m), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4) : "memory");
+}
+// one MMA over the pair: M = 256 (128 rows of A from each CTA), N columns (N/2 rows of B
+// from each CTA), accumulator rows split the same way between the two CTAs' TMEM
+__device__ __forceinline__ void umma_bf16_pair(uint32_t dtm, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(dtm), "l"(ad), "l"(bd), "r"(idesc), "r"(acc));
+}
+// completion of the pair's earlier MMAs arrives on the barrier at this offset in both CTAs
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar) {
+    const uint16_t mask = 3;
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 ::"r"(su32(bar)), "h"(mask) : "memory");
+}
+
 // ------------------------------------------------------------------ host side
 // Tensor map over a row-major tensor, dims/strides innermost first (strides in bytes,
 // rank-1 entries), 128-byte swizzle unless given, zero fill outside the tensor.
