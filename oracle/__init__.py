@@ -57,6 +57,10 @@ def lib():
         L.oracle_unit_rms.argtypes = [i32, i32, P, dbl, P]
         L.oracle_lru_sim.restype = i32
         L.oracle_lru_sim.argtypes = [i32, i32, i32, P, P, P, P, P, P, P]
+        L.oracle_e4m3_round.restype = dbl
+        L.oracle_e4m3_round.argtypes = [dbl]
+        L.oracle_mxfp8_qdq.argtypes = [i64, P, P]
+        L.oracle_expert_ffn_mxfp8_act.argtypes = [i32, i32, i32, P, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -288,6 +292,30 @@ def lru_sim_global_resizable(num_layers: int, num_experts: int, slots_per_layer:
         hits[i % L] += sum(h)
         misses[i % L] += len(h) - sum(h)
     return hits, misses, content
+
+
+def e4m3_round(v: float) -> float:
+    return lib().oracle_e4m3_round(float(v))
+
+
+def mxfp8_qdq(v) -> np.ndarray:
+    """Block-scaled E4M3 quantise-dequantise (blocks of 32 along the last axis)."""
+    a = _c(v, np.float64)
+    out = np.empty_like(a)
+    lib().oracle_mxfp8_qdq(a.size, _p(a), _p(out))
+    return out
+
+
+def expert_ffn_mxfp8_act(wdtype: int, hidden: int, ffn: int, w13, w13_scale, w2, w2_scale, x64) -> np.ndarray:
+    """expert_ffn with x and h quantised to MXFP8 (E4M3 + E8M0 per 32), for error studies of a
+    block-scaled MMA path; not the method's arithmetic."""
+    w13 = np.ascontiguousarray(w13)
+    w2 = np.ascontiguousarray(w2)
+    x = _c(x64, np.float64)
+    o = np.empty(hidden, dtype=np.float64)
+    lib().oracle_expert_ffn_mxfp8_act(hidden, ffn, wdtype, _p(w13), _p(_c(w13_scale, np.uint8)), _p(w2),
+                                      _p(_c(w2_scale, np.uint8)), _p(x), _p(o))
+    return o
 
 
 def full_layer(shape: dict, x_bits, w_router, bias, weights: dict, logits32=None, tokens=None, n_threads: int = 0):

@@ -260,6 +260,71 @@ int oracle_moe_layer(int T, int H, int F, int E, int k, int S, int wdtype,
     return bad ? -1 : 0;
 }
 
+/* ---------- error study: block-scaled (MXFP8) activations ------------- */
+
+/* Nearest E4M3 value (OCP 8-bit float E4M3: 1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits, no infinities; largest normal 448 = 1.75 * 2^8, smallest normal 2^-6, subnormal step
+ * 2^-9), ties to even, magnitudes above 448 saturated to 448 (the MX v1.0 spec leaves
+ * overflow handling to the implementation; saturation is the conversion it recommends). */
+double oracle_e4m3_round(double v)
+{
+    double a = fabs(v);
+    if (a == 0.0) return 0.0 * v;
+    int e = (int)floor(log2(a));
+    if (e < -6) e = -6;                       /* subnormal range: fixed step 2^-9 */
+    double step = ldexp(1.0, e - 3);
+    double q = a / step;
+    double r = floor(q);
+    double d = q - r;
+    if (d > 0.5 || (d == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    double out = r * step;
+    if (out > 448.0) out = 448.0;
+    return v < 0 ? -out : out;
+}
+
+/* MXFP8 (E4M3) quantise-dequantise of n values in blocks of 32 (OCP Microscaling Formats
+ * v1.0, conversion of a block of scalars to MX: shared scale X = 2^(floor(log2(max |v|)) -
+ * emax_elem), emax_elem = 8 for E4M3; element P_i = round_E4M3(v_i / X); value = X * P_i).
+ * A block of zeros keeps scale 1.  n % 32 == 0. */
+void oracle_mxfp8_qdq(long n, const double* v, double* out)
+{
+    for (long b = 0; b < n; b += 32) {
+        double amax = 0.0;
+        for (int i = 0; i < 32; ++i) if (fabs(v[b + i]) > amax) amax = fabs(v[b + i]);
+        double X = amax > 0.0 ? ldexp(1.0, (int)floor(log2(amax)) - 8) : 1.0;
+        for (int i = 0; i < 32; ++i) out[b + i] = X * oracle_e4m3_round(v[b + i] / X);
+    }
+}
+
+/* The expert FFN of oracle_expert_ffn with both activation operands (x before gate/up, h
+ * before down) passed through oracle_mxfp8_qdq, as a block-scaled MMA with E4M3 activations
+ * would see them; products and sums stay fp64.  H % 32 == 0, F % 32 == 0. */
+void oracle_expert_ffn_mxfp8_act(int H, int F, int wdtype, const void* w13, const uint8_t* w13_scale,
+                                 const void* w2, const uint8_t* w2_scale, const double* x, double* o)
+{
+    double* xq = (double*)malloc(sizeof(double) * (size_t)H);
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    double* hq = (double*)malloc(sizeof(double) * (size_t)F);
+    oracle_mxfp8_qdq(H, x, xq);
+    for (int f = 0; f < F; ++f) {
+        double a = 0.0, b = 0.0;
+        for (int i = 0; i < H; ++i) {
+            a += w_elem(wdtype, w13, w13_scale, H, f, i) * xq[i];
+            b += w_elem(wdtype, w13, w13_scale, H, F + f, i) * xq[i];
+        }
+        h[f] = a / (1.0 + exp(-a)) * b;
+    }
+    oracle_mxfp8_qdq(F, h, hq);
+    for (int i = 0; i < H; ++i) {
+        double s = 0.0;
+        for (int f = 0; f < F; ++f) s += w_elem(wdtype, w2, w2_scale, F, i, f) * hq[f];
+        o[i] = s;
+    }
+    free(xq);
+    free(h);
+    free(hq);
+}
+
 /* ---------- stacked-layer chaining ------------------------------------- */
 
 /* x_next[t,:] = y[t,:] / sqrt(mean_h y[t,h]^2 + eps), fp64. */
