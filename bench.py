@@ -476,6 +476,34 @@ def measure_stack(torch, F, rank, hbm_gbs):
                           "h2d_gbs": out["host_bytes"] / (pf_ms * 1e-3) / 1e9,
                           "frac_of_h2d_probe": out["host_bytes"] / (pf_ms * 1e-3) / 1e9 / best,
                           "layer_copy_ms_at_probe": layer_bytes / (best * 1e9) * 1e3}
+        # the same prefill streaming only each layer's routed experts (no copy/compute overlap)
+        F.ft_expert_stream_reset_cache(handle)
+        e0.record()
+        F.ft_expert_stream_prefill_routed(handle, Tp, x, wr, bs, yl, xl, ws, copy_stream=copy_stream)
+        e1.record()
+        torch.cuda.synchronize()
+        rt_ms = e0.elapsed_time(e1)
+        out["prefill_routed"] = {"T": Tp, "ms": rt_ms, "tokens_per_s": Tp / (rt_ms * 1e-3),
+                                 "h2d_bytes": F.ft_expert_stream_stats(handle, -1)[2]}
+        del ws, yl, xl
+        # a short prompt: whole layers vs routed experts only
+        Ts = 64
+        xsm = Layer.dev(torch, inputs.make_tokens(cfg, Ts, seed=0, stream=501))
+        ws = torch.empty(F.ft_moe_workspace_bytes(shape, Ts), dtype=torch.uint8, device="cuda")
+        F.ft_moe_workspace_init(ws)
+        yl = torch.empty((nl, Ts, H), dtype=torch.int16, device="cuda")
+        xl = torch.empty((nl, Ts, H), dtype=torch.int16, device="cuda")
+        small = {"T": Ts}
+        for mode, fn in (("full_layer", F.ft_expert_stream_prefill), ("routed_only", F.ft_expert_stream_prefill_routed)):
+            fn(handle, Ts, xsm, wr, bs, yl, xl, ws, copy_stream=copy_stream)       # warm-up
+            torch.cuda.synchronize()
+            F.ft_expert_stream_reset_cache(handle)
+            e0.record()
+            fn(handle, Ts, xsm, wr, bs, yl, xl, ws, copy_stream=copy_stream)
+            e1.record()
+            torch.cuda.synchronize()
+            small[mode] = {"ms": e0.elapsed_time(e1), "h2d_bytes": F.ft_expert_stream_stats(handle, -1)[2]}
+        out["prefill_short_prompt"] = small
         del ws, yl, xl
         # decode: cold cache, 256 single-token steps, first with a cache per layer, then with
         # the same total slot count pooled across layers (global LRU at equal capacity)

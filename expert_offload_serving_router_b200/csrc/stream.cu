@@ -126,6 +126,7 @@ struct ft_expert_stream {
     void** dtable;                  // device [L][E][4]
     void** htable;                  // pinned host mirror [L][E][4]
     int32_t* hids;                  // pinned [kSmallRoute * kMaxTopK]
+    int32_t* hoff;                  // pinned [kMaxExperts + 2]: group offsets for routed-only prefill
     cudaEvent_t ready[2], freed[2], ids_ev, copy_ev;
     std::vector<LayerCache> cache;  // per-layer counters; per-layer policy: also the slot state
     bool global = false;            // FT_CACHE_GLOBAL: slot state lives in `pool`
@@ -236,6 +237,7 @@ ft_status ft_expert_stream_create(const ft_stream_cfg* cfg, ft_expert_stream** o
     reset_slots(st);
     cudaError_t e = cudaHostAlloc(reinterpret_cast<void**>(&st->htable), size_t(st->L) * E * 4 * sizeof(void*), cudaHostAllocDefault);
     if (e == cudaSuccess) e = cudaHostAlloc(reinterpret_cast<void**>(&st->hids), sizeof(int32_t) * kSmallRoute * kMaxTopK, cudaHostAllocDefault);
+    if (e == cudaSuccess) e = cudaHostAlloc(reinterpret_cast<void**>(&st->hoff), sizeof(int32_t) * (kMaxExperts + 2), cudaHostAllocDefault);
     for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
         e = cudaEventCreateWithFlags(&st->ready[i], cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->freed[i], cudaEventDisableTiming);
@@ -261,6 +263,7 @@ void ft_expert_stream_destroy(ft_expert_stream* s) {
     if (s->copy_ev) cudaEventDestroy(s->copy_ev);
     if (s->htable) cudaFreeHost(s->htable);
     if (s->hids) cudaFreeHost(s->hids);
+    if (s->hoff) cudaFreeHost(s->hoff);
     delete s;
 }
 
@@ -348,6 +351,91 @@ ft_status ft_expert_stream_prefill(ft_expert_stream* s, int32_t T, const void* x
         }
     }
     return FT_OK;
+}
+
+ft_status ft_expert_stream_prefill_routed(ft_expert_stream* s, int32_t T, const void* x, const float* const* w_router,
+                                          const float* const* bias, void* y_layers, void* x_layers, void* ws,
+                                          size_t ws_bytes, void* compute_stream, void* copy_stream) {
+    ft_status st = check_common(s, T, x, w_router, y_layers, x_layers, ws, ws_bytes);
+    if (st) return st;
+    if (T == 0) return FT_OK;
+    if (T <= ft_get_decode_max_tokens())
+        return fail(FT_ERR_UNSUPPORTED, "prefill needs T > decode threshold (%d)", ft_get_decode_max_tokens());
+    if ((st = cuda_state())) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(compute_stream), ps = static_cast<cudaStream_t>(copy_stream);
+    const ft_moe_shape& sh = s->cfg.shape;
+    const int E = s->E;
+    const size_t TH = size_t(T) * sh.hidden;
+    uint16_t* xl = static_cast<uint16_t*>(x_layers);
+    uint16_t* yl = static_cast<uint16_t*>(y_layers);
+    const WsLayout Lw = make_layout(sh, T);
+    int32_t* idx = ws_at<int32_t>(ws, Lw.topk_idx);
+    float* gw = ws_at<float>(ws, Lw.topk_w);
+    int32_t* offsets = ws_at<int32_t>(ws, Lw.offsets);
+    int32_t* sorted_flat = ws_at<int32_t>(ws, Lw.sorted_flat);
+    int32_t* inv_pos = ws_at<int32_t>(ws, Lw.inv_pos);
+    void* xs = ws_at<uint16_t>(ws, Lw.x_sorted);
+    void* os = ws_at<uint16_t>(ws, Lw.o_sorted);
+    if ((st = cuda_ok(cudaMemcpyAsync(xl, x, TH * 2, cudaMemcpyDeviceToDevice, cs), "copy x"))) return st;
+    // buffer 0 may still be read by an earlier call's kernels
+    if ((st = cuda_ok(cudaStreamWaitEvent(ps, s->freed[0], 0), "wait freed"))) return st;
+    for (int l = 0; l < s->L; ++l) {
+        LayerCache& c = s->cache[size_t(l)];
+        const uint16_t* xcur = xl + size_t(l) * TH;
+        // 1. route and permute on the GPU, read the group offsets back (the one host wait)
+        if ((st = ft_moe_route(&sh, T, xcur, w_router[l], bias ? bias[l] : nullptr, idx, gw, nullptr, ws, ws_bytes, cs)))
+            return st;
+        if ((st = ft_moe_permute(&sh, T, idx, xcur, offsets, sorted_flat, inv_pos, xs, ws, ws_bytes, cs))) return st;
+        if ((st = cuda_ok(cudaMemcpyAsync(s->hoff, offsets, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToHost, cs),
+                          "offsets D2H")))
+            return st;
+        if ((st = cuda_ok(cudaEventRecord(s->ids_ev, cs), "record offsets"))) return st;
+        const auto t0 = std::chrono::steady_clock::now();
+        for (;;) {
+            cudaError_t q = cudaEventQuery(s->ids_ev);
+            if (q == cudaSuccess) break;
+            if (q != cudaErrorNotReady) return cuda_ok(q, "wait for the group offsets");
+            if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(s->timeout_ms))
+                return fail(FT_ERR_TIMEOUT, "layer %d: group offsets not back within %lld ms", l, (long long)s->timeout_ms);
+            std::this_thread::yield();
+        }
+        c.wait_us += uint64_t(std::chrono::duration_cast<std::chrono::microseconds>(std::chrono::steady_clock::now() - t0).count());
+        // 2. copy only the routed experts into their places in the layer buffer.  Every kernel
+        //    that read the buffer before (the previous layer) finished before this layer's
+        //    routing ran, so the copies may start now.
+        const ft_moe_weights& h = s->host[size_t(l)];
+        const ft_moe_weights d = layer_view(s, l, s->buf[0]);
+        uint64_t bytes = 0;
+        for (int e = 0; e < E; ++e) {
+            if (s->hoff[e + 1] == s->hoff[e]) continue;
+            cudaError_t ce = cudaMemcpyAsync(static_cast<uint8_t*>(const_cast<void*>(d.w13)) + size_t(e) * s->b13,
+                                             static_cast<const uint8_t*>(h.w13) + size_t(e) * s->b13, s->b13,
+                                             cudaMemcpyHostToDevice, ps);
+            if (ce == cudaSuccess && s->b13s)
+                ce = cudaMemcpyAsync(const_cast<uint8_t*>(d.w13_scale) + size_t(e) * s->b13s, h.w13_scale + size_t(e) * s->b13s,
+                                     s->b13s, cudaMemcpyHostToDevice, ps);
+            if (ce == cudaSuccess)
+                ce = cudaMemcpyAsync(static_cast<uint8_t*>(const_cast<void*>(d.w2)) + size_t(e) * s->b2,
+                                     static_cast<const uint8_t*>(h.w2) + size_t(e) * s->b2, s->b2, cudaMemcpyHostToDevice, ps);
+            if (ce == cudaSuccess && s->b2s)
+                ce = cudaMemcpyAsync(const_cast<uint8_t*>(d.w2_scale) + size_t(e) * s->b2s, h.w2_scale + size_t(e) * s->b2s,
+                                     s->b2s, cudaMemcpyHostToDevice, ps);
+            if (ce != cudaSuccess) return cuda_ok(ce, "routed expert host->device copy");
+            bytes += s->b13 + s->b13s + s->b2 + s->b2s;
+        }
+        c.h2d += bytes;
+        c.prefill_copies += 1;
+        if ((st = cuda_ok(cudaEventRecord(s->ready[0], ps), "record ready"))) return st;
+        if ((st = cuda_ok(cudaStreamWaitEvent(cs, s->ready[0], 0), "wait ready"))) return st;
+        // 3. experts and combine from the layer buffer
+        if ((st = ft_moe_experts(&sh, T, &d, xcur, xs, offsets, sorted_flat, os, ws, ws_bytes, cs))) return st;
+        if ((st = ft_moe_combine(&sh, T, os, inv_pos, gw, yl + size_t(l) * TH, cs))) return st;
+        if (l + 1 < s->L) {
+            st = ft_moe_unit_rms(T, sh.hidden, yl + size_t(l) * TH, xl + size_t(l + 1) * TH, 1e-6f, cs);
+            if (st) return st;
+        }
+    }
+    return cuda_ok(cudaEventRecord(s->freed[0], cs), "record freed");
 }
 
 ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const void* x, const float* const* w_router,

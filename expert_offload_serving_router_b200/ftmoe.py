@@ -74,6 +74,7 @@ _SIGS = {
     "ft_expert_stream_arena_bytes": (c_sz, [ctypes.POINTER(ft_stream_cfg)]),
     "ft_expert_stream_create": (c_i32, [ctypes.POINTER(ft_stream_cfg), ctypes.POINTER(c_vp)]),
     "ft_expert_stream_prefill": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "ft_expert_stream_prefill_routed": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
     "ft_expert_stream_decode_step": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
     "ft_expert_stream_stats": (c_i32, [c_vp, c_i32, ctypes.POINTER(c_u64)]),
     "ft_expert_stream_slots": (c_i32, [c_vp, c_i32, ctypes.POINTER(c_i32)]),
@@ -265,6 +266,15 @@ def ft_expert_stream_prefill(handle, T, x, w_router, bias, y_layers, x_layers, w
     _check(lib().ft_expert_stream_prefill(handle, T, _p(x), ctypes.addressof(wr), ctypes.addressof(bs) if bs else None,
                                           _p(y_layers), _p(x_layers), _p(ws), _nbytes(ws, ws_bytes),
                                           _s(compute_stream), _s(copy_stream)))
+
+
+def ft_expert_stream_prefill_routed(handle, T, x, w_router, bias, y_layers, x_layers, ws, ws_bytes=None,
+                                    compute_stream=None, copy_stream=None):
+    wr = _ptr_array(w_router)
+    bs = _ptr_array(bias) if bias is not None else None
+    _check(lib().ft_expert_stream_prefill_routed(handle, T, _p(x), ctypes.addressof(wr),
+                                                 ctypes.addressof(bs) if bs else None, _p(y_layers), _p(x_layers),
+                                                 _p(ws), _nbytes(ws, ws_bytes), _s(compute_stream), _s(copy_stream)))
 
 
 def ft_expert_stream_decode_step(handle, T, x, w_router, bias, y_layers, x_layers, ws, ws_bytes=None,

@@ -276,6 +276,21 @@ ft_status ft_expert_stream_prefill(ft_expert_stream* s, int32_t T, const void* x
                                    void* y_layers, void* x_layers, void* ws, size_t ws_bytes,
                                    void* compute_stream, void* copy_stream);
 
+/* All layers over T tokens (T > decode threshold), streaming only the experts
+ * each layer's router picks: per layer, route and permute on compute_stream,
+ * read the group offsets back (one bounded host wait), copy the routed experts
+ * host->HBM into their places in a layer buffer on copy_stream, then run the
+ * experts and the combine.  Copies cannot overlap the layer's own compute (its
+ * routing is needed first), so this pays off when a batch routes to a small
+ * part of the expert set; the pages' prefill streams whole layers instead
+ * ("full-layer double buffering": FreeToken article, dothoosh.com, "FreeToken
+ * architecture", mechanism 2).  Same arguments and results as prefill (the
+ * same kernels on the same data: bit-identical outputs). */
+ft_status ft_expert_stream_prefill_routed(ft_expert_stream* s, int32_t T, const void* x,
+                                          const float* const* w_router, const float* const* bias,
+                                          void* y_layers, void* x_layers, void* ws, size_t ws_bytes,
+                                          void* compute_stream, void* copy_stream);
+
 /* One decode step over T tokens (T <= decode threshold), all layers, through
  * the LRU expert-slot cache.  Same arguments as prefill. */
 ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const void* x,

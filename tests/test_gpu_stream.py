@@ -52,7 +52,8 @@ class Stack:
         ws = workspace(self.shape, T)
         y = torch.empty((NL, T, H), dtype=torch.int16, device="cuda")
         xl = torch.empty((NL, T, H), dtype=torch.int16, device="cuda")
-        fn = F.ft_expert_stream_prefill if kind == "prefill" else F.ft_expert_stream_decode_step
+        fn = {"prefill": F.ft_expert_stream_prefill, "prefill_routed": F.ft_expert_stream_prefill_routed,
+              "decode": F.ft_expert_stream_decode_step}[kind]
         fn(self.handle, T, dev(x), [L.t["w_router"] for L in self.layers], [L.t.get("bias") for L in self.layers],
            y, xl, ws, copy_stream=self.copy_stream)
         F.ft_moe_check(ws)
@@ -92,6 +93,23 @@ def test_prefill_streamed_equals_resident_and_oracle(stack):
             assert np.all(np.abs(got - want) <= 2.0 ** -7 * np.abs(want) + 1e-30)
     st = F.ft_expert_stream_stats(stack.handle, -1)
     assert st[4] == NL       # one full-layer copy per layer
+
+
+def test_routed_only_prefill_equals_full_layer_prefill(stack):
+    T = 40
+    x = inputs.make_tokens(stack.cfg, T, seed=21)
+    y_full, xl_full = stack.run("prefill", x)
+    F.ft_expert_stream_reset_cache(stack.handle)          # zero the counters
+    y_r, xl_r = stack.run("prefill_routed", x)
+    assert np.array_equal(y_r, y_full) and np.array_equal(xl_r, xl_full)
+    # exactly the experts each layer's router picked crossed the link
+    cfg = stack.cfg
+    per_expert = 3 * cfg.hidden * cfg.ffn // 2 + 3 * cfg.hidden * cfg.ffn // 32   # MXFP4 codes + scales
+    for l, L in enumerate(stack.layers):
+        _, idx, _ = _resident(L, xl_r[l])
+        st = F.ft_expert_stream_stats(stack.handle, l)
+        assert st[2] == len(set(idx.ravel().tolist())) * per_expert
+        assert st[4] == 1
 
 
 def test_decode_follows_oracle_lru_and_equals_resident(stack):
