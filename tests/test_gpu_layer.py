@@ -84,19 +84,28 @@ def test_small_custom_layers(wd, S, T):
     full_check(L, x, n_rows=T)
 
 
+@pytest.mark.parametrize("S", [0, 1])
+def test_cta_pair_gemm_shapes(S):
+    """Long-K BF16 gate/up with F a multiple of 256 runs on CTA pairs: routed and shared groups,
+    ragged token tiles."""
+    L = layer("custom", hidden=1536, ffn=256, num_experts=8, top_k=2, num_shared=S, config_id=70 + S)
+    x = inputs.make_tokens(L.cfg, 300, seed=8)
+    full_check(L, x, n_rows=40)
+
+
 def test_all_experts_selected_k_equals_E():
     L = layer("custom", hidden=128, ffn=64, num_experts=4, top_k=4, config_id=90)
     x = inputs.make_tokens(L.cfg, 50, seed=6)
     full_check(L, x, n_rows=50)
 
 
-@pytest.mark.parametrize("T", [700, 9])
-def test_skewed_routing_multi_tile_and_empty_groups(T):
+@pytest.mark.parametrize("T,hidden,ffn", [(700, 256, 128), (9, 256, 128), (700, 1536, 512)])
+def test_skewed_routing_multi_tile_and_empty_groups(T, hidden, ffn):
     """A bias sends every token to experts 3 and 5: two groups of T rows (several 256-row
-    tiles on the GEMM path), six empty groups."""
+    tiles on the GEMM path), six empty groups; hidden 1536 takes the CTA-pair gate/up GEMM."""
     from gpu_util import DevLayer, ensure_built
     ensure_built()
-    cfg = inputs.custom_config(hidden=256, ffn=128, num_experts=8, top_k=2, config_id=91)
+    cfg = inputs.custom_config(hidden=hidden, ffn=ffn, num_experts=8, top_k=2, config_id=91)
     d = inputs.make_layer(cfg, seed=7)
     d["bias"] = np.zeros(8, np.float32)
     d["bias"][[3, 5]] = 50.0
