@@ -213,3 +213,16 @@ def test_host_lru_resize_matches_oracle(seed):
     assert moves == omoves
     assert c[:n_new].tolist() == oc and st[:n_new].tolist() == os_
     assert {e: int(w[e]) for e in range(E) if w[e] >= 0} == ow
+
+
+def test_stream_calls_reject_a_null_handle_on_host():
+    """Every expert-stream entry point validates its handle before touching CUDA."""
+    for call in (lambda: F.ft_expert_stream_set_slots(None, 8, compute_stream=0, copy_stream=0),
+                 lambda: F.ft_expert_stream_reset_cache(None),
+                 lambda: F.ft_expert_stream_stats(None, -1),
+                 lambda: F.ft_expert_stream_slots(None, 0, 4),
+                 lambda: F.ft_expert_stream_prefill_routed(None, 64, FAKE, [FAKE], None, FAKE, FAKE, FAKE, 1 << 30,
+                                                           compute_stream=0, copy_stream=0)):
+        with pytest.raises(F.FtError) as ei:
+            call()
+        assert ei.value.status == F.FT_ERR_INVALID_ARG
