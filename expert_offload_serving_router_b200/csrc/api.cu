@@ -184,6 +184,7 @@ ft_status ft_moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 }
 
 ft_status ft_moe_check(void* ws, void* stream) {
+    FT_TRACE("ft_moe_check");
     if (!ws) return fail(FT_ERR_INVALID_ARG, "workspace is NULL");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     ft_status s = cuda_ok(cudaStreamSynchronize(st), "stream synchronize");
@@ -202,6 +203,7 @@ ft_status ft_moe_check(void* ws, void* stream) {
 
 ft_status ft_moe_route(const ft_moe_shape* shape, int32_t T, const void* x, const float* w_router, const float* bias,
                        int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t ws_bytes, void* stream) {
+    FT_TRACE("ft_moe_route");
     ft_status s = check_shape(shape);
     if (s) return s;
     if (T < 0) return fail(FT_ERR_INVALID_ARG, "T < 0");
@@ -223,6 +225,7 @@ ft_status ft_moe_route(const ft_moe_shape* shape, int32_t T, const void* x, cons
 ft_status ft_moe_permute(const ft_moe_shape* shape, int32_t T, const int32_t* topk_idx, const void* x, int32_t* offsets,
                          int32_t* sorted_flat, int32_t* inv_pos, void* x_sorted, void* ws, size_t ws_bytes,
                          void* stream) {
+    FT_TRACE("ft_moe_permute");
     ft_status s = check_shape(shape);
     if (s) return s;
     if (T < 0) return fail(FT_ERR_INVALID_ARG, "T < 0");
@@ -244,6 +247,7 @@ ft_status ft_moe_permute(const ft_moe_shape* shape, int32_t T, const int32_t* to
 ft_status ft_moe_experts(const ft_moe_shape* shape, int32_t T, const ft_moe_weights* weights, const void* x,
                          const void* x_sorted, const int32_t* offsets, const int32_t* sorted_flat, void* o_sorted,
                          void* ws, size_t ws_bytes, void* stream) {
+    FT_TRACE("ft_moe_experts");
     ft_status s = check_shape(shape);
     if (s) return s;
     if (T < 0) return fail(FT_ERR_INVALID_ARG, "T < 0");
@@ -286,16 +290,19 @@ static ft_status gemm_stage_entry(int mode, const ft_moe_shape* shape, int32_t T
 ft_status ft_moe_experts_gateup(const ft_moe_shape* shape, int32_t T, const ft_moe_weights* weights,
                                 const void* x_sorted, const int32_t* offsets, void* h, void* ws, size_t ws_bytes,
                                 void* stream) {
+    FT_TRACE("ft_moe_experts_gateup");
     return gemm_stage_entry(0, shape, T, weights, x_sorted, offsets, h, ws, ws_bytes, stream);
 }
 
 ft_status ft_moe_experts_down(const ft_moe_shape* shape, int32_t T, const ft_moe_weights* weights, const void* h,
                               const int32_t* offsets, void* o_sorted, void* ws, size_t ws_bytes, void* stream) {
+    FT_TRACE("ft_moe_experts_down");
     return gemm_stage_entry(1, shape, T, weights, h, offsets, o_sorted, ws, ws_bytes, stream);
 }
 
 ft_status ft_moe_combine(const ft_moe_shape* shape, int32_t T, const void* o_sorted, const int32_t* inv_pos,
                          const float* topk_w, void* y, void* stream) {
+    FT_TRACE("ft_moe_combine");
     ft_status s = check_shape(shape);
     if (s) return s;
     if (T < 0) return fail(FT_ERR_INVALID_ARG, "T < 0");
@@ -313,6 +320,7 @@ ft_status ft_moe_combine(const ft_moe_shape* shape, int32_t T, const void* o_sor
 ft_status ft_moe_layer_forward(const ft_moe_shape* shape, int32_t T, const void* x, const float* w_router,
                                const float* bias, const ft_moe_weights* weights, void* y, int32_t* topk_idx_out,
                                float* logits_out, void* ws, size_t ws_bytes, void* stream) {
+    FT_TRACE("ft_moe_layer_forward");
     ft_status s = check_shape(shape);
     if (s) return s;
     if (T < 0) return fail(FT_ERR_INVALID_ARG, "T < 0");
@@ -355,6 +363,7 @@ ft_status ft_moe_layer_forward(const ft_moe_shape* shape, int32_t T, const void*
 }
 
 ft_status ft_moe_unit_rms(int32_t T, int32_t H, const void* in, void* out, float eps, void* stream) {
+    FT_TRACE("ft_moe_unit_rms");
     if (T < 0 || H <= 0 || H % 8) return fail(FT_ERR_INVALID_ARG, "need T >= 0 and H a positive multiple of 8");
     if (T == 0) return FT_OK;
     if (!in || !out || !al(in, 16) || !al(out, 16)) return fail(FT_ERR_INVALID_ARG, "in/out NULL or not 16-byte aligned");

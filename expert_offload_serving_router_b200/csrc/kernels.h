@@ -1,9 +1,21 @@
 // Internal launcher declarations shared by the kernel files and the C-ABI layer.
 #pragma once
 #include "common.cuh"
+#include <nvtx3/nvToolsExt.h>
 #include "permute_small.cuh"
 
 namespace ftmoe {
+
+// NVTX range around one public entry point (named in profiler timelines; no cost without a
+// profiler attached).
+struct TraceRange {
+    explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange&) = delete;
+    TraceRange& operator=(const TraceRange&) = delete;
+};
+#define FT_TRACE(name) ::ftmoe::TraceRange ft_trace_range_(name)
+
 
 struct DecodeArgs {
     int T, k, E, S, H, F, wdtype;

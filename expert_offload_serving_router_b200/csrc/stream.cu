@@ -314,6 +314,7 @@ extern "C" {
 ft_status ft_expert_stream_prefill(ft_expert_stream* s, int32_t T, const void* x, const float* const* w_router,
                                    const float* const* bias, void* y_layers, void* x_layers, void* ws, size_t ws_bytes,
                                    void* compute_stream, void* copy_stream) {
+    FT_TRACE("ft_expert_stream_prefill");
     ft_status st = check_common(s, T, x, w_router, y_layers, x_layers, ws, ws_bytes);
     if (st) return st;
     if (T == 0) return FT_OK;
@@ -356,6 +357,7 @@ ft_status ft_expert_stream_prefill(ft_expert_stream* s, int32_t T, const void* x
 ft_status ft_expert_stream_prefill_routed(ft_expert_stream* s, int32_t T, const void* x, const float* const* w_router,
                                           const float* const* bias, void* y_layers, void* x_layers, void* ws,
                                           size_t ws_bytes, void* compute_stream, void* copy_stream) {
+    FT_TRACE("ft_expert_stream_prefill_routed");
     ft_status st = check_common(s, T, x, w_router, y_layers, x_layers, ws, ws_bytes);
     if (st) return st;
     if (T == 0) return FT_OK;
@@ -441,6 +443,7 @@ ft_status ft_expert_stream_prefill_routed(ft_expert_stream* s, int32_t T, const 
 ft_status ft_expert_stream_decode_step(ft_expert_stream* s, int32_t T, const void* x, const float* const* w_router,
                                        const float* const* bias, void* y_layers, void* x_layers, void* ws,
                                        size_t ws_bytes, void* compute_stream, void* copy_stream) {
+    FT_TRACE("ft_expert_stream_decode_step");
     ft_status st = check_common(s, T, x, w_router, y_layers, x_layers, ws, ws_bytes);
     if (st) return st;
     if (T == 0) return FT_OK;
@@ -613,6 +616,7 @@ ft_status ft_expert_stream_reset_cache(ft_expert_stream* s) {
 
 ft_status ft_expert_stream_set_slots(ft_expert_stream* s, int32_t slots_per_layer, void* compute_stream,
                                      void* copy_stream) {
+    FT_TRACE("ft_expert_stream_set_slots");
     if (!s) return fail(FT_ERR_INVALID_ARG, "stream handle is NULL");
     if (slots_per_layer < s->k || slots_per_layer > s->S_max)
         return fail(FT_ERR_INVALID_ARG, "slots_per_layer %d must be in [k=%d, %d (arena)]", slots_per_layer, s->k,
