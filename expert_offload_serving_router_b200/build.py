@@ -1,6 +1,6 @@
 """Build libftmoe.so in-tree with nvcc for sm_100a (B200).
 
-    python -m expert_offload_serving_router_b200.build [--force] [--verbose]
+    python -m expert_offload_serving_router_b200.build [--force] [--verbose] [--debug-bounds]
 
 Each csrc/*.cu is compiled to an object under _build/ (parallel), then linked into
 expert_offload_serving_router_b200/libftmoe.so with the CUDA runtime linked statically.
@@ -20,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libftmoe.so")
+DEBUG_LIB = os.path.join(PKG, "libftmoe_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]
@@ -44,15 +45,23 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None, debug_bounds: bool = False) -> str:
+    """debug_bounds: build libftmoe_debug.so instead, with FT_DEBUG_BOUNDS=1 (extra device-side
+    checks of every permutation and of the decode slot table; select it with FTMOE_LIB)."""
+    if debug_bounds:
+        return _build_into(os.path.join(BUILD, "debug"), DEBUG_LIB, force, verbose, ["-DFT_DEBUG_BOUNDS=1", *(extra or [])])
+    return _build_into(BUILD, LIB, force, verbose, extra)
+
+
+def _build_into(build_dir: str, lib: str, force: bool, verbose: bool, extra: list[str] | None) -> str:
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdrs = _headers()
     cc = nvcc()
     jobs = []
     objs = []
     for s in srcs:
-        o = os.path.join(BUILD, os.path.basename(s) + ".o")
+        o = os.path.join(build_dir, os.path.basename(s) + ".o")
         objs.append(o)
         if force or _stale(o, [s] + hdrs):
             cmd = [cc, *ARCH, *FLAGS, *(extra or []), "-c", s, "-o", o]
@@ -67,16 +76,16 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
                 sys.stderr.write(r.stdout + r.stderr)
             if r.returncode:
                 raise RuntimeError("nvcc failed: " + " ".join(cmd))
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or jobs or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [cc, *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static", "-lpthread"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode:
             sys.stderr.write(r.stdout + r.stderr)
             raise RuntimeError("link failed")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, debug_bounds="--debug-bounds" in sys.argv))

@@ -196,6 +196,7 @@ ft_status ft_moe_check(void* ws, void* stream) {
         cudaMemset(ws, 0, sizeof flag);
         return fail(FT_ERR_DEVICE_CHECK, flag == kDevErrBadExpert ? "a routed expert id was outside [0, E)"
                                          : flag == kDevErrTimeout ? "a grouped-GEMM pipeline wait timed out"
+                                         : flag == kDevErrBounds  ? "a debug-bounds check failed (permutation or slot table)"
                                                                   : "device check failed (code %u)", flag);
     }
     return FT_OK;

@@ -131,6 +131,10 @@ inline WsLayout make_layout(const ft_moe_shape& s, int T) {
 }
 
 // device error codes written into ws err[0]
-enum : uint32_t { kDevErrNone = 0, kDevErrBadExpert = 1, kDevErrTimeout = 2, kDevErrShape = 3 };
+enum : uint32_t { kDevErrNone = 0, kDevErrBadExpert = 1, kDevErrTimeout = 2, kDevErrShape = 3, kDevErrBounds = 4 };
+
+#ifndef FT_DEBUG_BOUNDS
+#define FT_DEBUG_BOUNDS 0
+#endif
 
 }  // namespace ftmoe

@@ -262,6 +262,10 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
     const int P = a.T * a.k, R = P + (a.S ? a.T : 0);
     const int G = a.E + (a.S ? 1 : 0);
+    {
+        cudaError_t ce = launch_slot_table_check(a.sched, G, a.E, a.eptr, a.wdtype == FT_W_MXFP4, a.err, st);
+        if (ce != cudaSuccess) return ce;
+    }
     const int na_max = R < G ? R : G;
     const bool mx = a.wdtype == FT_W_MXFP4;
     int TB = 1;

@@ -76,6 +76,10 @@ cudaError_t launch_route(int T, int H, int E, int k, int S, const uint16_t* x, c
 cudaError_t launch_route_tc(int T, int H, int E, int k, const uint16_t* x, const float* wr, const float* bias,
                             int32_t* topk_idx, float* topk_w, float* logits, uint16_t* planes, float* part,
                             uint32_t* err, cudaStream_t st);
+// debug-bounds build only (no-ops otherwise): permutation invariants, decode slot table
+cudaError_t launch_perm_check(const int32_t* idx, int T, int k, int E, int S, const PermOut& out, cudaStream_t st);
+cudaError_t launch_slot_table_check(const int32_t* sched, int G, int E, const void* const* eptr, int mx, uint32_t* err,
+                                    cudaStream_t st);
 cudaError_t launch_permute(int T, int k, int E, int S, int H, const int32_t* idx, const uint16_t* x,
                            uint16_t* x_sorted, int32_t* chunk_cnt, int32_t* chunk_base, int32_t* local_rank,
                            const PermOut& out, cudaStream_t st);

@@ -208,14 +208,16 @@ cudaError_t launch_permute(int T, int k, int E, int S, int H, const int32_t* idx
     const int P = T * k, R = P + (S ? T : 0);
     if (R <= 1024) {
         perm_small_kernel<<<1, 256, 0, st>>>(idx, T, k, E, S, out, x, x_sorted, H);
-        return cudaGetLastError();
+    } else {
+        const int C = (R + kPermChunk - 1) / kPermChunk;
+        PermArgs a{T, k, E, S, H, idx, x, x_sorted, chunk_cnt, chunk_base, local_rank, out};
+        perm_count_kernel<<<C, 256, 0, st>>>(a);
+        perm_scan_kernel<<<1, 1024, 0, st>>>(a, C);
+        perm_scatter_kernel<<<(R + kScatterItems - 1) / kScatterItems, 256, 0, st>>>(a);
     }
-    const int C = (R + kPermChunk - 1) / kPermChunk;
-    PermArgs a{T, k, E, S, H, idx, x, x_sorted, chunk_cnt, chunk_base, local_rank, out};
-    perm_count_kernel<<<C, 256, 0, st>>>(a);
-    perm_scan_kernel<<<1, 1024, 0, st>>>(a, C);
-    perm_scatter_kernel<<<(R + kScatterItems - 1) / kScatterItems, 256, 0, st>>>(a);
-    return cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_perm_check(idx, T, k, E, S, out, st);
 }
 
 }  // namespace ftmoe

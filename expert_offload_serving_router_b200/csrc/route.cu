@@ -131,7 +131,9 @@ cudaError_t launch_route(int T, int H, int E, int k, int S, const uint16_t* x, c
         at[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = at;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, route_small_kernel, a);
+        cudaError_t e = cudaLaunchKernelEx(&cfg, route_small_kernel, a);
+        if (e != cudaSuccess || !perm) return e;
+        return launch_perm_check(topk_idx, T, k, E, S, *perm, st);
     }
     if (perm) return cudaErrorInvalidValue;   // the fused permutation exists only for decode-sized batches
     return launch_route_tc(T, H, E, k, x, wr, bias, topk_idx, topk_w, logits, planes, part, err, st);

@@ -14,7 +14,9 @@ import os
 import re
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libftmoe.so")
+# FTMOE_LIB selects another build of the same library (e.g. libftmoe_debug.so, the
+# debug-bounds build); default: the in-tree libftmoe.so
+LIB_PATH = os.environ.get("FTMOE_LIB") or os.path.join(PKG, "libftmoe.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "ftmoe.h")
 
 FT_OK, FT_ERR_INVALID_ARG, FT_ERR_UNSUPPORTED, FT_ERR_CUDA, FT_ERR_WORKSPACE, FT_ERR_NOT_PINNED, \
