@@ -161,6 +161,14 @@ def job_tokens_per_s(world, tokens_per_rank, ms_max):
     return world * tokens_per_rank / (ms_max * 1e-3)
 
 
+def overlap_efficiency(copy_ms: float, compute_ms: float, layers: int, wall_ms: float) -> float:
+    """Double-buffered layer streaming: the ideal wall time is the first layer's copy, then per
+    layer the longer of the next layer's copy and this layer's compute (the last layer has no
+    next copy).  Returns ideal / measured (1.0 = copies and compute overlap perfectly)."""
+    ideal = copy_ms + (layers - 1) * max(copy_ms, compute_ms) + compute_ms
+    return ideal / wall_ms
+
+
 def run_reference(args, rank):
     """Reference arm: the fp64 CPU oracle, as it stands, on the host cores."""
     if rank != 0:
@@ -656,6 +664,14 @@ def main():
             del Lx, px
             torch.cuda.empty_cache()
     stack = measure_stack(torch, F, rank, hbm_gbs) if args.stack else None
+    if stack and extra and "prefill" in stack:
+        # copy time per layer from the pinned-copy probe, compute time per layer from the same
+        # layer shape measured resident (DSV4-Flash-shaped prefill at the stack's T)
+        pf = stack["prefill"]
+        comp = extra["dsv4_flash"]["prefill"]["ms_step"]
+        pf["layer_compute_ms_resident"] = comp
+        pf["overlap_efficiency"] = overlap_efficiency(pf["layer_copy_ms_at_probe"], comp,
+                                                      inputs.STACK["num_layers"], pf["ms"])
 
     if rank != 0:
         if world > 1:

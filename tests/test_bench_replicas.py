@@ -59,3 +59,11 @@ def test_reference_arm_runs_on_rank_zero_only():
     with contextlib.redirect_stdout(buf):
         assert bench.run_reference(Args(), 1) is None
     assert buf.getvalue() == ""
+
+
+def test_overlap_efficiency_formula():
+    # 8 layers, copies slower than compute: ideal = copy + 7 * copy + compute
+    assert bench.overlap_efficiency(60.0, 5.0, 8, 60 * 8 + 5) == pytest.approx(1.0)
+    assert bench.overlap_efficiency(60.0, 5.0, 8, 2 * (60 * 8 + 5)) == pytest.approx(0.5)
+    # compute-bound layers: ideal = copy + 7 * compute + compute
+    assert bench.overlap_efficiency(2.0, 10.0, 8, 2.0 + 80.0) == pytest.approx(1.0)
