@@ -7,6 +7,7 @@
 #include <string>
 
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace ftmoe {
 
@@ -34,6 +35,9 @@ static int init_decode_max() {
 }
 static int g_decode_max = init_decode_max();
 int decode_max() { return g_decode_max; }
+
+static unsigned long long g_gemm_wait_ns = kWaitNs;
+unsigned long long gemm_wait_ns() { return g_gemm_wait_ns; }
 
 static bool al(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -169,6 +173,12 @@ int32_t ft_set_decode_max_tokens(int32_t t) {
 }
 
 int32_t ft_get_decode_max_tokens(void) { return g_decode_max; }
+
+uint64_t ft_set_pipeline_wait_limit_ns(uint64_t ns) {
+    const unsigned long long prev = g_gemm_wait_ns;
+    g_gemm_wait_ns = ns ? ns : kWaitNs;
+    return prev;
+}
 
 size_t ft_moe_workspace_bytes(const ft_moe_shape* shape, int32_t max_tokens) {
     if (check_shape(shape) != FT_OK || max_tokens < 0) return 0;

@@ -85,6 +85,8 @@ cudaError_t launch_permute(int T, int k, int E, int S, int H, const int32_t* idx
                            const PermOut& out, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st);
+// bound (ns without progress) on each pipeline wait of the grouped GEMMs (api.cu)
+unsigned long long gemm_wait_ns();
 cudaError_t launch_combine(int T, int H, int k, int S, int R, const uint16_t* o, const int32_t* inv_pos,
                            const float* gw, uint16_t* y, cudaStream_t st);
 cudaError_t launch_unit_rms(int T, int H, const uint16_t* in, uint16_t* out, float eps, cudaStream_t st);

@@ -7,7 +7,7 @@
 
 namespace ftmoe {
 
-constexpr unsigned long long kWaitNs = 4000000000ull;  // 4 s bound on any wait
+constexpr unsigned long long kWaitNs = 4000000000ull;  // 4 s: default bound on a wait
 
 __device__ __forceinline__ uint32_t su32(const void* p) { return uint32_t(__cvta_generic_to_shared(p)); }
 
@@ -32,15 +32,18 @@ __device__ __forceinline__ uint64_t gtimer() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Bounded wait.  Gives up when `abort` is raised by another role or after kWaitNs.
-static __device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort) {
+// Bounded wait.  Gives up when `abort` is raised by another role or after `limit` ns without
+// the phase completing.  Pipeline waits pass the launch's limit; drains and teardown waits
+// keep the default.
+static __device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort,
+                                              unsigned long long limit = kWaitNs) {
     if (mbar_try(b, parity)) return true;
     const uint64_t t0 = gtimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try(b, parity)) return true;
         if ((i & 31) == 0) {
             if (abort && *abort) return false;
-            if (gtimer() - t0 > kWaitNs) return false;
+            if (gtimer() - t0 > limit) return false;
         }
     }
 }
@@ -154,14 +157,15 @@ __device__ __forceinline__ bool mbar_try_acq_cluster(uint64_t* b, uint32_t parit
     return ok != 0;
 }
 // bounded wait on a barrier that the peer CTA also arrives on
-static __device__ __noinline__ bool mbar_wait_cluster(uint64_t* b, uint32_t parity, volatile int* abort) {
+static __device__ __noinline__ bool mbar_wait_cluster(uint64_t* b, uint32_t parity, volatile int* abort,
+                                                      unsigned long long limit = kWaitNs) {
     if (mbar_try_acq_cluster(b, parity)) return true;
     const uint64_t t0 = gtimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_acq_cluster(b, parity)) return true;
         if ((i & 31) == 0) {
             if (abort && *abort) return false;
-            if (gtimer() - t0 > kWaitNs) return false;
+            if (gtimer() - t0 > limit) return false;
         }
     }
 }

@@ -57,6 +57,7 @@ _SIGS = {
     "ft_version": (ctypes.c_char_p, []),
     "ft_set_decode_max_tokens": (c_i32, [c_i32]),
     "ft_get_decode_max_tokens": (c_i32, []),
+    "ft_set_pipeline_wait_limit_ns": (c_u64, [c_u64]),
     "ft_moe_workspace_bytes": (c_sz, [ctypes.POINTER(ft_moe_shape), c_i32]),
     "ft_moe_workspace_init": (c_i32, [c_vp, c_sz, c_vp]),
     "ft_moe_check": (c_i32, [c_vp, c_vp]),
@@ -168,6 +169,10 @@ def ft_set_decode_max_tokens(t: int) -> int:
 
 def ft_get_decode_max_tokens() -> int:
     return lib().ft_get_decode_max_tokens()
+
+
+def ft_set_pipeline_wait_limit_ns(ns: int) -> int:
+    return lib().ft_set_pipeline_wait_limit_ns(ns)
 
 
 def ft_moe_workspace_bytes(shape: ft_moe_shape, max_tokens: int) -> int:

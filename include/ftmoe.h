@@ -39,10 +39,20 @@
  *   - Errors are return codes; ft_last_error() gives a thread-local message.
  *     Argument errors are detected on the host before any CUDA call.  An
  *     asynchronous CUDA error from earlier work surfaces as FT_ERR_CUDA.
- *   - Supported shapes: H % 128 == 0, F % 64 == 0, 1 <= k <= 8, k <= E <= 256,
- *     S in {0, 1}; MXFP4 additionally needs H % 32 == 0 and F % 32 == 0
- *     (implied).  T may be 0 (nothing is launched).  Larger T than the
- *     max_tokens the workspace was sized for returns FT_ERR_WORKSPACE.
+ *   - Supported shapes: H % 128 == 0, H <= 16384, F % 64 == 0, F <= 4096,
+ *     1 <= k <= 8, k <= E <= 256, S in {0, 1} (FT_ERR_UNSUPPORTED otherwise):
+ *     the grouped GEMMs tile weights in groups of 128 rows (64 gate + 64 up
+ *     rows for gate/up, 128 hidden rows for down).  MXFP4 additionally needs
+ *     H % 32 == 0 and F % 32 == 0 (implied).  T may be 0 (nothing is
+ *     launched).  Larger T than the max_tokens the workspace was sized for
+ *     returns FT_ERR_WORKSPACE.
+ *   - Activation precision: x, h and y are bf16 and every product is exact
+ *     with fp32 accumulation, except on the decode path (T <= threshold) with
+ *     MXFP4 weights, where the GEMVs multiply in f16: the activations (x, and
+ *     h for the down projection) are rounded to f16 there, which is exact for
+ *     2^-17 <= |v| <= 65504; |v| > 65504 becomes +-inf and below 2^-17 the
+ *     absolute error is at most 2^-25.  The grouped GEMM path (prefill) keeps
+ *     bf16 activations.
  *
  * Layouts (all row-major, innermost dimension last):
  *   x        [T, H]  bf16           topk_idx [T, k] int32     topk_w [T, k] fp32
@@ -122,6 +132,18 @@ const char* ft_version(void);
 int32_t ft_set_decode_max_tokens(int32_t t);
 int32_t ft_get_decode_max_tokens(void);
 
+/* Bound on every pipeline wait of the grouped-GEMM kernels (steps 3 and 4 when
+ * T > decode threshold): the time, in ns, a role waits for a stage without
+ * progress before it gives up.  Default 4 s (4000000000); ns = 0 restores the
+ * default.  Process-wide, applies to launches enqueued after the call; returns
+ * the previous bound.  A wait that runs out makes the kernel give up cleanly:
+ * it records a timeout in the workspace status word (ft_moe_check then
+ * returns FT_ERR_DEVICE_CHECK), lets the copies and MMAs it issued finish,
+ * frees its tensor memory and returns; that call's outputs are undefined and
+ * the next call is unaffected.  Lets failure handling be tested without a
+ * GPU fault (a bound too short for the pipeline makes the waits run out). */
+uint64_t ft_set_pipeline_wait_limit_ns(uint64_t ns);
+
 /* Bytes of scratch any call below needs for up to max_tokens tokens
  * (0 on invalid shape). */
 size_t ft_moe_workspace_bytes(const ft_moe_shape* shape, int32_t max_tokens);
@@ -167,11 +189,15 @@ ft_status ft_moe_permute(const ft_moe_shape* shape, int32_t T, const int32_t* to
  * Limit: R = T*k + S*T <= 65536 rows, else FT_ERR_UNSUPPORTED before any
  * launch.  The first call on each device looks the array's device address up
  * (cudaGetSymbolAddress) and caches it; make that first call before any stream
- * capture.  Every call shares the array and it keeps the last call's contents:
- * calls that overlap on the GPU race.  No allocation of any kind.  An id
- * outside [0,E) drops its pair (offsets[E+S] < R shows it).  The tile schedule
- * that ft_moe_permute leaves in its ws for ft_moe_experts is not produced for
- * the caller here. */
+ * capture.  The cached address lives as long as the device's context: do not
+ * cudaDeviceReset that device after the first call.  `stream` must belong to
+ * the current device (else FT_ERR_INVALID_ARG).  Every call shares the array
+ * and it keeps the last call's contents: calls that overlap on the GPU race.
+ * No allocation of any kind.  An id outside [0,E) drops its pair, and
+ * offsets[E+S] < R is the only sign of it: the device status word that
+ * ft_moe_check reads for a workspace (also the debug-bounds build's checks) is
+ * not reported by this entry point.  The tile schedule that ft_moe_permute
+ * leaves in its ws for ft_moe_experts is not produced for the caller here. */
 ft_status ft_moe_permute_noalloc(const ft_moe_shape* shape, int32_t T, const int32_t* topk_idx, const void* x,
                                  int32_t* offsets, int32_t* sorted_flat, int32_t* inv_pos, void* x_sorted,
                                  void* stream);

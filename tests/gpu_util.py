@@ -114,3 +114,21 @@ def sample_rows(T: int, n: int, seed: int = 0) -> np.ndarray:
         return np.arange(T, dtype=np.int32)
     r = np.random.default_rng(seed).choice(T, size=n - 2, replace=False)
     return np.unique(np.concatenate([[0, T - 1], r])).astype(np.int32)
+
+
+def group_rows(idx: np.ndarray, num_experts: int, num_shared: int = 0, tile: int = 256) -> np.ndarray:
+    """Tokens whose rows cover every non-empty expert group of the permutation the routing
+    idx gives (the oracle's stable counting sort): the first row of every `tile`-row token
+    tile of each group (the grouped GEMM's tiles) and the group's last row (its ragged tail).
+    The shared group (S = 1) holds every token in order, so it is covered by any rows."""
+    T, k = idx.shape
+    offsets, sf, _ = oracle.permute(idx, num_experts, num_shared)
+    picks = []
+    for g in range(num_experts):
+        lo, hi = int(offsets[g]), int(offsets[g + 1])
+        if hi == lo:
+            continue
+        picks.extend(range(lo, hi, tile))
+        picks.append(hi - 1)
+    flat = sf[np.asarray(picks, dtype=np.int64)]
+    return np.unique(np.where(flat < T * k, flat // k, flat - T * k)).astype(np.int32)

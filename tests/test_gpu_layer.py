@@ -24,9 +24,13 @@ def layer(name, **kw):
 
 
 def full_check(L, x, n_rows=12, seed=0):
-    from gpu_util import check_logits, check_y, oracle_rows, run_layer, sample_rows
+    """Whole layer on the GPU; routing compared for every token, outputs for a seeded sample of
+    n_rows tokens plus, at every size, tokens covering each non-empty expert group (the first
+    row of each 256-row token tile and the group's last row)."""
+    from gpu_util import check_logits, check_y, group_rows, oracle_rows, run_layer, sample_rows
     y, idx, lg = run_layer(L, x)
-    rows = sample_rows(x.shape[0], n_rows, seed)
+    rows = np.union1d(sample_rows(x.shape[0], n_rows, seed),
+                      group_rows(idx, L.cfg.num_experts, L.cfg.num_shared)).astype(np.int32)
     check_logits(x, L, lg, rows)
     oidx, og, y64 = oracle_rows(L, x, lg, rows)
     assert np.array_equal(idx, oidx), "routing differs from the oracle's top-k on the GPU logits"
@@ -85,6 +89,23 @@ def test_small_custom_layers(wd, S, T):
 
 
 @pytest.mark.parametrize("S", [0, 1])
+@pytest.mark.parametrize("T", [3, 300, 1100])
+def test_mxfp4_cta_pair_gemm_shapes(S, T):
+    """MXFP4 layers whose gate/up (K = 1024) and down (K = 512) GEMMs both run on the CTA-pair
+    kernel with TMA-streamed codes: routed and shared groups, ragged token tiles, groups of
+    more than 256 rows (T = 1100), and a decode-sized batch forced onto the grouped GEMM."""
+    L = layer("custom", hidden=1024, ffn=512, num_experts=8, top_k=2, num_shared=S, wdtype=inputs.WDTYPE_MXFP4,
+              config_id=60 + S)
+    x = inputs.make_tokens(L.cfg, T, seed=9)
+    prev = F.ft_set_decode_max_tokens(0) if T <= 32 else None
+    try:
+        full_check(L, x, n_rows=min(T, 48))
+    finally:
+        if prev is not None:
+            F.ft_set_decode_max_tokens(prev)
+
+
+@pytest.mark.parametrize("S", [0, 1])
 def test_cta_pair_gemm_shapes(S):
     """Long-K BF16 gate/up with F a multiple of 256 runs on CTA pairs: routed and shared groups,
     ragged token tiles."""
@@ -99,13 +120,15 @@ def test_all_experts_selected_k_equals_E():
     full_check(L, x, n_rows=50)
 
 
-@pytest.mark.parametrize("T,hidden,ffn", [(700, 256, 128), (9, 256, 128), (700, 1536, 512)])
-def test_skewed_routing_multi_tile_and_empty_groups(T, hidden, ffn):
+@pytest.mark.parametrize("T,hidden,ffn,wd", [(700, 256, 128, 0), (9, 256, 128, 0), (700, 1536, 512, 0),
+                                            (700, 1024, 512, 1)])
+def test_skewed_routing_multi_tile_and_empty_groups(T, hidden, ffn, wd):
     """A bias sends every token to experts 3 and 5: two groups of T rows (several 256-row
-    tiles on the GEMM path), six empty groups; hidden 1536 takes the CTA-pair gate/up GEMM."""
+    tiles on the GEMM path), six empty groups; hidden 1536 takes the CTA-pair BF16 gate/up
+    GEMM, the MXFP4 case (hidden 1024, ffn 512) the CTA-pair MXFP4 GEMMs."""
     from gpu_util import DevLayer, ensure_built
     ensure_built()
-    cfg = inputs.custom_config(hidden=hidden, ffn=ffn, num_experts=8, top_k=2, config_id=91)
+    cfg = inputs.custom_config(hidden=hidden, ffn=ffn, num_experts=8, top_k=2, wdtype=wd, config_id=91 + wd)
     d = inputs.make_layer(cfg, seed=7)
     d["bias"] = np.zeros(8, np.float32)
     d["bias"][[3, 5]] = 50.0
