@@ -1,19 +1,21 @@
 #!/usr/bin/env python
 """Benchmark: MoE-layer tokens/s on B200 and the roofline fraction of the dominant kernel.
 
-Workload (headline): the Qwen3-A3B-shaped MoE layer -- hidden 2048, expert FFN 768
-(SwiGLU), 128 experts, top-8 with a Zipf(s=1) rank-scaled router bias, BF16 weights
-N(0, 0.02^2) -- on a 4096-token prefill batch (x ~ N(0,1) bf16).  One step = one pass of
-the whole hot path: route (fp32 logits + top-k + gates), permute (counting sort + row
-gather), grouped gate/up GEMM with fused SwiGLU, grouped down GEMM, combine.  Weights
-(1.21 GB) and the permuted activations exceed the 126 MB L2, so every step streams
-from HBM without an explicit flush.  Decode batches (1/4/16 tokens) are reported in
-an extra object, timed while rotating over 4 weight copies so that no batch finds its
-experts in L2.  --extra adds the other layer shapes (DeepSeek-V4-Flash-shaped MXFP4,
-Gemma-4-26B-A4B-shaped with a shared expert, the tiny layer) and --stack the
-expert-offload stack (8 DSV4-Flash-shaped layers served from pinned host memory).
+Workload (headline): the DeepSeek-V4-Flash-shaped MoE layer -- hidden 4096, expert FFN
+2048 (SwiGLU), 256 experts, top-6, MXFP4 expert weights (E2M1 codes uniform over the 16
+codes, one E8M0 scale per 32 elements uniform on 2^-8..2^-4) -- on an 8192-token prefill
+batch (x ~ N(0,1) bf16).  This is the largest layer shape that runs on one GPU.  One step
+= one pass of the whole hot path: route (fp32 logits + top-k + gates), permute (counting
+sort + row gather), grouped gate/up GEMM with fused SwiGLU, grouped down GEMM, combine.
+The expert weights (3.42 GB) and the permuted activations exceed the 126 MB L2, so every
+step streams from HBM without an explicit flush.  Decode batches of the same layer (1 and
+8 tokens) are reported in an extra object, timed while rotating over 4 weight copies so
+that no batch finds its experts in L2.  By default the line also carries the other layer
+shapes (Qwen3-A3B-shaped BF16 with a Zipf-skewed router, Gemma-4-26B-A4B-shaped with a
+shared expert, the tiny layer: prefill and decode) and the expert-offload stack (8
+DSV4-Flash-shaped layers served from pinned host memory); --no-extra / --no-stack skip them.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--extra] [--stack]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extra] [--no-stack]
 
 Multi-GPU: the layer forward does not shard (one GPU per layer by construction), so
 N > 1 runs N independent replicas, one process per GPU under torchrun; value is the
@@ -36,8 +38,8 @@ sys.path.insert(0, ROOT)
 
 from expert_offload_serving_router_b200 import inputs  # noqa: E402
 
-WORKLOAD = "qwen3_a3b"
-PREFILL_T = 4096
+WORKLOAD = "dsv4_flash"
+PREFILL_T = 8192
 PREFILL_SIZES = {"qwen3_a3b": 4096, "dsv4_flash": 8192, "gemma4_26b_a4b": 2048, "tiny": 64}
 METRIC = "MoE-layer tokens/s (decode & prefill) and % of HBM / tensor-core roofline"
 LAUNCHES_PER_STEP = 3 + 3 + 1 + 1 + 1   # router (plane split, GEMM, top-k), permute (count/scan/scatter), gate/up, down, combine
@@ -576,6 +578,45 @@ def measure_stack(torch, F, rank, hbm_gbs):
     return out
 
 
+def measure_hbm_ceiling(torch, sizes_mb=(8, 16, 32, 64, 76, 128, 256, 512, 1024, 2048), iters=20):
+    """Streaming throughput a plain read (torch's float32 sum) and a device-to-device copy reach
+    for transfers of a given size, rotating over enough buffers (>= 1 GiB together) that L2 never
+    holds the next one.  GB/s counts the bytes read (read) or read + written (copy)."""
+    out = []
+    for mb in sizes_mb:
+        n = mb << 20
+        k = max(4, -(-(1 << 30) // n))
+        bufs = [torch.empty(n // 4, dtype=torch.float32, device="cuda").normal_() for _ in range(k)]
+        dst = torch.empty(n // 4, dtype=torch.float32, device="cuda")
+        row = {"mbytes": mb}
+        for kind in ("read", "copy"):
+            def op(i):
+                if kind == "read":
+                    return bufs[i % k].sum()
+                return dst.copy_(bufs[i % k])
+            for i in range(3):
+                op(i)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(iters):
+                op(i)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / iters
+            moved = n if kind == "read" else 2 * n
+            row[kind] = {"us": us, "gbs": moved / (us * 1e-6) / 1e9}
+        out.append(row)
+        del bufs, dst
+        torch.cuda.empty_cache()
+    return out
+
+
+EXTRA_WORKLOADS = [("qwen3_a3b", [1, 4, 16]), ("gemma4_26b_a4b", [1]), ("tiny", [])]
+HEADLINE_DECODE = [1, 8]
+ROOFLINE_SUMMARY = ("moe_gemm_mxfp4_dsv4_flash_T8192.md", "gemm_mx_sm100.cu")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -585,15 +626,19 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-batch measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
-    ap.add_argument("--decode-tokens", default="1,4,16", help="decode batch sizes to time (comma list)")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other layer shapes")
+    ap.add_argument("--no-stack", action="store_true", help="skip the expert-offload stack")
+    ap.add_argument("--decode-tokens", default=None, help="decode batch sizes to time (comma list)")
     ap.add_argument("--decode-only", default=None, metavar="CONFIG",
                     help="time only decode batches of this layer shape (for profiling)")
     ap.add_argument("--prefill-only", default=None, metavar="CONFIG",
                     help="time only prefill steps of this layer shape at its prefill size (for profiling)")
-    ap.add_argument("--extra", action="store_true", help="also measure the other layer shapes")
-    ap.add_argument("--stack", action="store_true", help="also measure the expert-offload stack")
+    ap.add_argument("--prefill-tokens", type=int, default=None,
+                    help="with --prefill-only: the batch size (default: the shape's prefill size)")
+    ap.add_argument("--hbm-ceiling", action="store_true",
+                    help="only time plain streaming reads and copies of decode-sized transfers")
     args = ap.parse_args()
-    args.decode_tokens = [int(v) for v in args.decode_tokens.split(",") if v]
+    dec_tokens = None if args.decode_tokens is None else [int(v) for v in args.decode_tokens.split(",") if v]
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
@@ -616,10 +661,16 @@ def main():
     F.lib()
     hbm_gbs, tc_burst, tc_sus, peak_src = peaks()
 
+    if args.hbm_ceiling:
+        if rank == 0:
+            print(json.dumps({"mode": "hbm-ceiling", "peak_gbs": hbm_gbs, "peak_source": peak_src,
+                              "sizes": measure_hbm_ceiling(torch)}), flush=True)
+        return
+
     if args.decode_only:
         cfg = inputs.CONFIGS[args.decode_only]
         L = Layer(torch, F, cfg, inputs.make_layer(cfg, seed=0))
-        dec = measure_decode(torch, F, L, args.decode_tokens, rank, hbm_gbs)
+        dec = measure_decode(torch, F, L, dec_tokens or list(cfg.decode_tokens), rank, hbm_gbs)
         if rank == 0:
             print(json.dumps({"mode": "decode-only", "workload": f"{cfg.name} decode", "decode": dec}), flush=True)
         return
@@ -627,7 +678,7 @@ def main():
     if args.prefill_only:
         cfg = inputs.CONFIGS[args.prefill_only]
         Lp = Layer(torch, F, cfg, inputs.make_layer(cfg, seed=0))
-        Tp = PREFILL_SIZES.get(args.prefill_only, PREFILL_T)
+        Tp = args.prefill_tokens or PREFILL_SIZES[args.prefill_only]
         px = measure_prefill(torch, F, Lp, Tp, args.steps, args.warmup, torch.cuda.current_stream(), rank)
         if rank == 0:
             print(json.dumps({"mode": "prefill-only", "workload": f"{cfg.name} prefill, T={Tp}",
@@ -647,30 +698,32 @@ def main():
         dist.barrier()
     value = job_tokens_per_s(world, T, ms_step)
     tc_peak = tc_sus if pre["total_ms"] > 1000.0 else tc_burst
-    traffic = recorded_traffic("moe_gemm_gateup_qwen3_a3b_T4096.md", "gemm_sm100.cu")
+    traffic = recorded_traffic(*ROOFLINE_SUMMARY)
     e2e = None if args.no_e2e else measure_e2e(torch, dist, F, L, pre["ctx"], T, args.steps, args.warmup, world)
-    decode = None if args.no_decode else measure_decode(torch, F, L, args.decode_tokens, rank, hbm_gbs)
+    decode = None if args.no_decode else measure_decode(torch, F, L, dec_tokens or HEADLINE_DECODE, rank, hbm_gbs)
+    headline_ms = pre["ms_step"]
+    del L, pre["ctx"]
+    torch.cuda.empty_cache()
     extra = None
-    if args.extra:
+    if not args.no_extra:
         extra = {}
-        for name, Tds in [("dsv4_flash", [1, 8]), ("gemma4_26b_a4b", [1]), ("tiny", [])]:
+        for name, Tds in EXTRA_WORKLOADS:
             Tp = PREFILL_SIZES[name]
             c = inputs.CONFIGS[name]
             Lx = Layer(torch, F, c, inputs.make_layer(c, seed=0))
             px = measure_prefill(torch, F, Lx, Tp, 10, 3, torch.cuda.current_stream(), rank)
             extra[name] = {"prefill": summarize_prefill(px, hbm_gbs, tc_burst)}
-            if Tds:
+            if Tds and not args.no_decode:
                 extra[name]["decode"] = measure_decode(torch, F, Lx, Tds, rank, hbm_gbs)
             del Lx, px
             torch.cuda.empty_cache()
-    stack = measure_stack(torch, F, rank, hbm_gbs) if args.stack else None
-    if stack and extra and "prefill" in stack:
+    stack = None if args.no_stack else measure_stack(torch, F, rank, hbm_gbs)
+    if stack and "prefill" in stack:
         # copy time per layer from the pinned-copy probe, compute time per layer from the same
-        # layer shape measured resident (DSV4-Flash-shaped prefill at the stack's T)
+        # layer shape measured resident (the headline DSV4-Flash-shaped prefill at the stack's T)
         pf = stack["prefill"]
-        comp = extra["dsv4_flash"]["prefill"]["ms_step"]
-        pf["layer_compute_ms_resident"] = comp
-        pf["overlap_efficiency"] = overlap_efficiency(pf["layer_copy_ms_at_probe"], comp,
+        pf["layer_compute_ms_resident"] = headline_ms
+        pf["overlap_efficiency"] = overlap_efficiency(pf["layer_copy_ms_at_probe"], headline_ms,
                                                       inputs.STACK["num_layers"], pf["ms"])
 
     if rank != 0:
@@ -681,23 +734,26 @@ def main():
     if world == 1 and not args.no_cpu:
         cpu = cpu_baseline(cfg, layer_np)
     sp = summarize_prefill(pre, hbm_gbs, tc_peak)
+    launches = LAUNCHES_PER_STEP * args.steps
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded numpy: N(0,0.02^2) bf16 weights, "
-                                                       "N(0,1) bf16 tokens, Zipf(1) router bias)",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy: MXFP4 codes uniform over the 16 E2M1 codes, E8M0 scales 2^-8..2^-4, "
+                "N(0,1) bf16 tokens, N(0,0.02^2) fp32 router)",
         "config": {"workload": f"{WORKLOAD} MoE layer prefill, T={T}", "hidden": cfg.hidden, "ffn": cfg.ffn,
-                   "experts": cfg.num_experts, "top_k": cfg.top_k, "tokens": T, "weights": "bf16",
+                   "experts": cfg.num_experts, "top_k": cfg.top_k, "tokens": T,
+                   "weights": "mxfp4 (E2M1 + E8M0 per 32, dequantised exactly to bf16 in the GEMM load path)",
                    "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (1.21 GB weights + 134 MB permuted rows per step), no flush"},
-        "roofline": {"bound": "tensor", "kernel": "moe_gemm_kernel<bf16> gate/up + SwiGLU",
+                   "l2": "inputs larger than L2 (3.42 GB weights + 403 MB permuted rows per step), no flush"},
+        "roofline": {"bound": "tensor", "kernel": "grouped GEMM (MXFP4 weights) gate/up + SwiGLU",
                      "achieved": pre["gateup_tflops"], "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": pre["gateup_tflops"] / tc_peak,
                      "peak_source": f"{peak_src} bf16 {'sustained' if tc_peak == tc_sus else 'burst'}",
                      "algorithmic_flops_per_launch": pre["gateup_flops"], "traffic": traffic},
         "stages_ms": sp["stage_ms"], "down_gemm_tflops": pre["down_tflops"],
         "experts_frac_of_peak": sp["experts_frac_tc"], "experts_frac_of_hbm": sp["experts_frac_hbm"],
-        "e2e": e2e, "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": pre["clocks"],
+        "e2e": e2e, "gpu_launches": launches, "clocks": pre["clocks"],
         "cpu_baseline": cpu, "decode": decode, "other_workloads": extra, "offload_stack": stack,
     }
     print(json.dumps(line), flush=True)
