@@ -18,7 +18,9 @@
 // any stream capture.  All calls share the one array and it keeps the last call's
 // contents, so calls whose work overlaps on the GPU (other streams, other host threads)
 // race on it.  Nothing in it has to start at zero: every count, base, rank and schedule
-// entry a call reads is written earlier in the same call.
+// entry a call reads is written earlier in the same call.  The device status word inside the
+// array (out-of-range ids, the debug-bounds build's permutation re-check) is never read back:
+// on this entry point an out-of-range id shows only as offsets[E+S] < R.
 #include <mutex>
 
 #include "kernels.h"
@@ -41,11 +43,21 @@ constexpr int kNoAllocMaxDevices = 64;
 static std::mutex g_scratch_mu;
 static void* g_scratch_addr[kNoAllocMaxDevices] = {};
 
-// Device address of g_permute_scratch on the current device, looked up once per device.
-static ft_status scratch_address(void** out) {
+// Device address of g_permute_scratch on the current device, looked up once per device.  The
+// cached address stays valid for the life of the device's primary context (a cudaDeviceReset
+// would invalidate it).  A stream of another device than the current one is rejected: the
+// address would belong to the wrong GPU.
+static ft_status scratch_address(cudaStream_t stream, void** out) {
     int dev = 0;
     ft_status s = cuda_ok(cudaGetDevice(&dev), "cudaGetDevice");
     if (s) return s;
+    if (stream) {
+        int sdev = -1;
+        if ((s = cuda_ok(cudaStreamGetDevice(stream, &sdev), "cudaStreamGetDevice"))) return s;
+        if (sdev != dev)
+            return fail(FT_ERR_INVALID_ARG, "ft_moe_permute_noalloc: the stream belongs to device %d but device %d is "
+                        "current", sdev, dev);
+    }
     if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(FT_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kNoAllocMaxDevices);
     std::lock_guard<std::mutex> lock(g_scratch_mu);
     if (!g_scratch_addr[dev]) {
@@ -79,7 +91,7 @@ extern "C" ft_status ft_moe_permute_noalloc(const ft_moe_shape* shape, int32_t T
         return fail(FT_ERR_INVALID_ARG, "x_sorted needs a 16-byte aligned x and x_sorted");
     if ((s = cuda_state())) return s;
     void* base = nullptr;
-    if ((s = scratch_address(&base))) return s;
+    if ((s = scratch_address(static_cast<cudaStream_t>(stream), &base))) return s;
     PermOut po{offsets, sorted_flat, inv_pos, ws_at<int32_t>(base, kNaSched), ws_at<uint32_t>(base, kNaErr)};
     return cuda_ok(launch_permute(T, shape->top_k, shape->num_experts, shape->num_shared, shape->hidden, topk_idx,
                                   static_cast<const uint16_t*>(x), static_cast<uint16_t*>(x_sorted),
