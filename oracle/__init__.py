@@ -61,6 +61,8 @@ def lib():
         L.oracle_e4m3_round.argtypes = [dbl]
         L.oracle_mxfp8_qdq.argtypes = [i64, P, P]
         L.oracle_expert_ffn_mxfp8_act.argtypes = [i32, i32, i32, P, P, P, P, P, P]
+        L.oracle_mxfp8x2_qdq.argtypes = [i64, P, P]
+        L.oracle_expert_ffn_mxfp8_planes.argtypes = [i32, i32, i32, i32, P, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -315,6 +317,28 @@ def expert_ffn_mxfp8_act(wdtype: int, hidden: int, ffn: int, w13, w13_scale, w2,
     o = np.empty(hidden, dtype=np.float64)
     lib().oracle_expert_ffn_mxfp8_act(hidden, ffn, wdtype, _p(w13), _p(_c(w13_scale, np.uint8)), _p(w2),
                                       _p(_c(w2_scale, np.uint8)), _p(x), _p(o))
+    return o
+
+
+def mxfp8x2_qdq(v) -> np.ndarray:
+    """Two-plane block-scaled E4M3 split: high plane = mxfp8_qdq(v), low plane = mxfp8_qdq of
+    the remainder; returns high + low (blocks of 32 along the last axis)."""
+    a = _c(v, np.float64)
+    out = np.empty_like(a)
+    lib().oracle_mxfp8x2_qdq(a.size, _p(a), _p(out))
+    return out
+
+
+def expert_ffn_mxfp8_planes(planes: int, wdtype: int, hidden: int, ffn: int, w13, w13_scale, w2, w2_scale,
+                            x64) -> np.ndarray:
+    """expert_ffn with x and h quantised to `planes` MXFP8 planes (1 or 2), for error studies
+    of a block-scaled MMA path; not the method's arithmetic."""
+    w13 = np.ascontiguousarray(w13)
+    w2 = np.ascontiguousarray(w2)
+    x = _c(x64, np.float64)
+    o = np.empty(hidden, dtype=np.float64)
+    lib().oracle_expert_ffn_mxfp8_planes(planes, hidden, ffn, wdtype, _p(w13), _p(_c(w13_scale, np.uint8)), _p(w2),
+                                         _p(_c(w2_scale, np.uint8)), _p(x), _p(o))
     return o
 
 

@@ -296,16 +296,34 @@ void oracle_mxfp8_qdq(long n, const double* v, double* out)
     }
 }
 
+/* Two-plane MXFP8 split of n values: the high plane is the MXFP8 quantise-dequantise of v
+ * (oracle_mxfp8_qdq), the low plane the same of the remainder v - high, each plane with its
+ * own E8M0 block scales; the result is high + low, which is what a block-scaled MMA run once
+ * per plane into one fp32 accumulator multiplies.  n % 32 == 0. */
+void oracle_mxfp8x2_qdq(long n, const double* v, double* out)
+{
+    double* hi = (double*)malloc(sizeof(double) * (size_t)n);
+    double* r = (double*)malloc(sizeof(double) * (size_t)n);
+    oracle_mxfp8_qdq(n, v, hi);
+    for (long i = 0; i < n; ++i) r[i] = v[i] - hi[i];
+    oracle_mxfp8_qdq(n, r, out);
+    for (long i = 0; i < n; ++i) out[i] += hi[i];
+    free(hi);
+    free(r);
+}
+
 /* The expert FFN of oracle_expert_ffn with both activation operands (x before gate/up, h
- * before down) passed through oracle_mxfp8_qdq, as a block-scaled MMA with E4M3 activations
- * would see them; products and sums stay fp64.  H % 32 == 0, F % 32 == 0. */
-void oracle_expert_ffn_mxfp8_act(int H, int F, int wdtype, const void* w13, const uint8_t* w13_scale,
-                                 const void* w2, const uint8_t* w2_scale, const double* x, double* o)
+ * before down) passed through the MXFP8 quantiser of `planes` planes (1: oracle_mxfp8_qdq,
+ * 2: oracle_mxfp8x2_qdq), as a block-scaled MMA with E4M3 activations would see them; products
+ * and sums stay fp64.  H % 32 == 0, F % 32 == 0. */
+void oracle_expert_ffn_mxfp8_planes(int planes, int H, int F, int wdtype, const void* w13, const uint8_t* w13_scale,
+                                    const void* w2, const uint8_t* w2_scale, const double* x, double* o)
 {
     double* xq = (double*)malloc(sizeof(double) * (size_t)H);
     double* h = (double*)malloc(sizeof(double) * (size_t)F);
     double* hq = (double*)malloc(sizeof(double) * (size_t)F);
-    oracle_mxfp8_qdq(H, x, xq);
+    if (planes == 2) oracle_mxfp8x2_qdq(H, x, xq);
+    else oracle_mxfp8_qdq(H, x, xq);
     for (int f = 0; f < F; ++f) {
         double a = 0.0, b = 0.0;
         for (int i = 0; i < H; ++i) {
@@ -314,7 +332,8 @@ void oracle_expert_ffn_mxfp8_act(int H, int F, int wdtype, const void* w13, cons
         }
         h[f] = a / (1.0 + exp(-a)) * b;
     }
-    oracle_mxfp8_qdq(F, h, hq);
+    if (planes == 2) oracle_mxfp8x2_qdq(F, h, hq);
+    else oracle_mxfp8_qdq(F, h, hq);
     for (int i = 0; i < H; ++i) {
         double s = 0.0;
         for (int f = 0; f < F; ++f) s += w_elem(wdtype, w2, w2_scale, F, i, f) * hq[f];
@@ -323,6 +342,13 @@ void oracle_expert_ffn_mxfp8_act(int H, int F, int wdtype, const void* w13, cons
     free(xq);
     free(h);
     free(hq);
+}
+
+/* One-plane form of oracle_expert_ffn_mxfp8_planes (E4M3 activations). */
+void oracle_expert_ffn_mxfp8_act(int H, int F, int wdtype, const void* w13, const uint8_t* w13_scale,
+                                 const void* w2, const uint8_t* w2_scale, const double* x, double* o)
+{
+    oracle_expert_ffn_mxfp8_planes(1, H, F, wdtype, w13, w13_scale, w2, w2_scale, x, o);
 }
 
 /* ---------- stacked-layer chaining ------------------------------------- */

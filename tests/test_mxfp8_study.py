@@ -100,3 +100,60 @@ def test_block_scaled_activations_miss_the_mxfp4_tolerance():
                                                             L["w2"][e], L["w2_scale"][e], xs[t])
     rel = np.abs(ymx - y64).max() / np.abs(y64).max()
     assert 3e-2 < rel < 0.1, rel       # measured 0.056 on this seed
+
+
+def test_two_plane_split_grid_and_error_bound():
+    """Pins of the two-plane split without re-running its formula: both planes lie on their own
+    block grids (E4M3 value times a power-of-two scale set by the plane's block maximum, the
+    rounding being pinned by brute force above), the remainder after both planes is bounded by
+    half an E4M3 ulp of the remainder after the first, and values already on the first plane's
+    grid leave an empty second plane."""
+    rng = np.random.default_rng(3)
+    v = rng.normal(size=32 * 64) * np.exp2(rng.integers(-10, 10, size=64)).repeat(32)
+    hi = oracle.mxfp8_qdq(v)
+    both = oracle.mxfp8x2_qdq(v)
+    lo = both - hi
+    r1 = v - hi
+    for b in range(0, v.size, 32):
+        for plane, ref in ((hi[b:b + 32], v[b:b + 32]), (lo[b:b + 32], r1[b:b + 32])):
+            amax = np.abs(ref).max()
+            if amax == 0:
+                assert np.all(plane == 0)
+                continue
+            X = 2.0 ** (math.floor(math.log2(amax)) - 8)
+            assert all(oracle.e4m3_round(t / X) == t / X for t in plane)
+        rb, r2 = r1[b:b + 32], (v - both)[b:b + 32]
+        X2 = 2.0 ** (math.floor(math.log2(np.abs(rb).max())) - 8) if np.abs(rb).max() > 0 else 1.0
+        normal = (np.abs(rb) >= X2 * 2.0 ** -6) & (np.abs(rb) <= 448 * X2)
+        assert np.all(np.abs(r2)[normal] <= 2.0 ** -4 * np.abs(rb)[normal])
+        # the second plane's subnormal step bounds what it cannot resolve
+        assert np.all(np.abs(r2)[~normal & (np.abs(rb) < X2 * 2.0 ** -6)] <= X2 * 2.0 ** -10)
+    grid = np.array([1.5, -3.0, 448.0, 0.0] * 8) * 2.0 ** -3
+    assert np.array_equal(oracle.mxfp8x2_qdq(grid), grid)
+
+
+def test_two_plane_block_scaled_activations_meet_the_mxfp4_tolerance():
+    """The same DeepSeek-V4-Flash-shaped MXFP4 layer with x and h each carried as two E4M3 planes
+    (high + remainder, own E8M0 scales): the error falls far inside 3e-2 * max|ref|, so a
+    block-scaled E2M1 x E4M3 MMA run once per activation plane could meet the tolerance."""
+    cfg = inputs.custom_config(name="dsv4_like", hidden=4096, ffn=2048, num_experts=8, top_k=6,
+                               wdtype=inputs.WDTYPE_MXFP4, config_id=97)
+    L = inputs.make_layer(cfg, seed=0)
+    T, H, F = 4, cfg.hidden, cfg.ffn
+    x = inputs.make_tokens(cfg, T, seed=0)
+    idx, g = oracle.topk(oracle.router_logits(x, L["w_router"]).astype(np.float32), cfg.top_k)
+    shape = dict(hidden=H, ffn=F, num_experts=cfg.num_experts, top_k=cfg.top_k, num_shared=0, wdtype=cfg.wdtype)
+    y64 = oracle.moe_layer(shape, x, idx, g, L)
+    xs = inputs.bf16_bits_to_f32(x).astype(np.float64)
+    rel = {}
+    for planes in (1, 2):
+        ymx = np.zeros_like(y64)
+        for t in range(T):
+            for j in range(cfg.top_k):
+                e = idx[t, j]
+                ymx[t] += g[t, j] * oracle.expert_ffn_mxfp8_planes(planes, cfg.wdtype, H, F, L["w13"][e],
+                                                                   L["w13_scale"][e], L["w2"][e],
+                                                                   L["w2_scale"][e], xs[t])
+        rel[planes] = np.abs(ymx - y64).max() / np.abs(y64).max()
+    assert 3e-2 < rel[1] < 0.1, rel          # the one-plane form of the study above
+    assert rel[2] < 3e-3, rel                 # two planes: an order of magnitude inside 3e-2
