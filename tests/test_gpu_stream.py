@@ -14,16 +14,19 @@ NL, SLOTS = 3, 4
 
 
 class Stack:
-    def __init__(self, wdtype=inputs.WDTYPE_MXFP4, zipf=True, cache_policy=F.FT_CACHE_PER_LAYER):
+    def __init__(self, wdtype=inputs.WDTYPE_MXFP4, zipf=True, cache_policy=F.FT_CACHE_PER_LAYER, cfg=None,
+                 nl=NL, slots=SLOTS, config_id=None):
         import torch
         from gpu_util import DevLayer, ensure_built, shape_of
         ensure_built()
-        self.cfg = inputs.custom_config(hidden=256, ffn=128, num_experts=16, top_k=2, wdtype=wdtype,
-                                        zipf_bias=zipf, config_id=95)
-        self.layers = [DevLayer(self.cfg, inputs.make_layer(self.cfg, seed=0, layer=l)) for l in range(NL)]
+        self.cfg = cfg or inputs.custom_config(hidden=256, ffn=128, num_experts=16, top_k=2, wdtype=wdtype,
+                                               zipf_bias=zipf, config_id=95)
+        self.nl, self.slots = nl, slots
+        self.layers = [DevLayer(self.cfg, inputs.make_layer(self.cfg, seed=0, layer=l, zipf=zipf, config_id=config_id))
+                       for l in range(nl)]
         self.shape = shape_of(self.cfg)
         self.pinned = []
-        hl = (F.ft_moe_weights * NL)()
+        hl = (F.ft_moe_weights * nl)()
         for l, L in enumerate(self.layers):
             ph = {}
             for key in ("w13", "w13_scale", "w2", "w2_scale"):
@@ -37,7 +40,7 @@ class Stack:
                 self.pinned.append(t)
             hl[l] = F.make_weights(ph.get("w13"), ph.get("w13_scale"), ph.get("w2"), ph.get("w2_scale"))
         self.host_layers = hl
-        cfg = F.ft_stream_cfg(NL, SLOTS, self.shape, hl, None, 0, 5000, cache_policy)
+        cfg = F.ft_stream_cfg(nl, slots, self.shape, hl, None, 0, 20000, cache_policy)
         n = F.ft_expert_stream_arena_bytes(cfg)
         self.arena = torch.empty(n, dtype=torch.uint8, device="cuda")
         cfg.hbm_arena = self.arena.data_ptr()
@@ -50,8 +53,8 @@ class Stack:
         from gpu_util import dev, host, workspace
         T, H = x.shape
         ws = workspace(self.shape, T)
-        y = torch.empty((NL, T, H), dtype=torch.int16, device="cuda")
-        xl = torch.empty((NL, T, H), dtype=torch.int16, device="cuda")
+        y = torch.empty((self.nl, T, H), dtype=torch.int16, device="cuda")
+        xl = torch.empty((self.nl, T, H), dtype=torch.int16, device="cuda")
         fn = {"prefill": F.ft_expert_stream_prefill, "prefill_routed": F.ft_expert_stream_prefill_routed,
               "decode": F.ft_expert_stream_decode_step}[kind]
         fn(self.handle, T, dev(x), [L.t["w_router"] for L in self.layers], [L.t.get("bias") for L in self.layers],
@@ -61,6 +64,7 @@ class Stack:
 
     def close(self):
         F.ft_expert_stream_destroy(self.handle)
+        self.handle = None
 
 
 @pytest.fixture(scope="module")
@@ -248,3 +252,48 @@ def test_unpinned_host_memory_is_rejected():
     with pytest.raises(F.FtError) as ei:
         F.ft_expert_stream_create(c)
     assert ei.value.status == F.FT_ERR_NOT_PINNED
+
+
+def test_deepseek_v4_flash_shaped_stack_prefill_and_decode():
+    """Two DeepSeek-V4-Flash-shaped MXFP4 layers (hidden 4096, FFN 2048, 256 experts, top-6,
+    13.37 MB per expert, Zipf-skewed routers) served from pinned host memory with 32 HBM slots
+    per layer: the full-layer-streamed 8192-token prefill and 16 single-token decode steps
+    through the slot cache (256-entry pointer tables) equal the resident layers bit for bit, the
+    cache follows the oracle's LRU, and sampled outputs match the fp64 oracle."""
+    from gpu_util import check_y, oracle_rows, sample_rows
+    st = inputs.STACK
+    cfg = inputs.CONFIGS[st["layer"]]
+    nl, slots = 2, st["slots_per_layer"]
+    g = Stack(cfg=cfg, nl=nl, slots=slots, zipf=True, config_id=st["config_id"])
+    try:
+        T = st["prefill_tokens"]
+        x = inputs.make_tokens(cfg, T, seed=31)
+        y, xl = g.run("prefill", x)
+        assert np.array_equal(xl[0], x)
+        for l, L in enumerate(g.layers):
+            yr, idx, lg = _resident(L, xl[l])
+            assert np.array_equal(y[l], yr), f"prefill layer {l}: streamed != resident"
+            rows = sample_rows(T, 8, seed=l)
+            _, _, y64 = oracle_rows(L, xl[l], lg, rows)
+            check_y(y[l][rows], y64, cfg.wdtype, f"stack prefill layer {l}")
+        assert F.ft_expert_stream_stats(g.handle, -1)[4] == nl
+
+        F.ft_expert_stream_reset_cache(g.handle)
+        steps = 16
+        routed = [[] for _ in range(nl)]
+        for s in range(steps):
+            xd = inputs.make_tokens(cfg, 1, seed=32, stream=s)
+            y, xl = g.run("decode", xd)
+            for l, L in enumerate(g.layers):
+                yr, idx, lg = _resident(L, xl[l])
+                assert np.array_equal(y[l], yr), f"decode step {s} layer {l}: slot-cache result != resident"
+                routed[l].append(sorted(set(idx.ravel().tolist())))
+        per_expert = 3 * cfg.hidden * cfg.ffn // 2 + 3 * cfg.hidden * cfg.ffn // 32
+        for l in range(nl):
+            oslot, ohit, ose, h, m = oracle.lru_sim(cfg.num_experts, slots, routed[l])
+            stl = F.ft_expert_stream_stats(g.handle, l)
+            assert (stl[0], stl[1], stl[3]) == (h, m, steps)
+            assert stl[2] == m * per_expert            # every miss copied one whole expert
+            assert F.ft_expert_stream_slots(g.handle, l, slots) == ose[-1].tolist()
+    finally:
+        g.close()
