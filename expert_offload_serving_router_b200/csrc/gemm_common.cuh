@@ -61,6 +61,31 @@ __device__ __forceinline__ void e2m1x8_bf16(uint32_t w, uint32_t scale2, uint32_
         asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o[i]) : "r"(x), "r"(scale2));
     }
 }
+// The same eight codes by bit placement: the three magnitude bits of a code moved to bf16 bits
+// 6..8 and its sign to bit 15 form exactly E2M1(code) * 2^-126 (code magnitude 1 -> the bf16
+// subnormal 2^-127; e = 1..3 -> normals), so one exact multiply by 2^(s - 1) gives
+// E2M1 * 2^(s - 127).  Valid for scale bytes s <= 128 (2^(s - 1) must be a finite bf16);
+// scale2m1 = bf16x2 of 2^(s - 1).  Per output word: one byte permute pairs codes 2i (low half)
+// and 2i+1 (high half) with zero bytes around them, a shift places the magnitude, one
+// multiply-add moves the sign from bit 9 to bit 15 (adds sign * (2^15 - 2^9)).
+__device__ __forceinline__ void e2m1x8_bf16_place(uint32_t w, uint32_t scale2m1, uint32_t (&o)[4]) {
+    const uint32_t lo = w & 0x0F0F0F0Fu;           // codes 0, 2, 4, 6 (one per byte)
+    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;    // codes 1, 3, 5, 7
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        // bytes: lo.byte i, 0, hi.byte i, 0 (a selector with its top bit set replicates the sign
+        // of the selected byte, < 0x80 here, so it yields 0; __byte_perm would drop that bit)
+        uint32_t pr;
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(pr) : "r"(lo), "r"(hi), "r"(0x8080u | uint32_t(i) | (uint32_t(4 + i) << 8)));
+        const uint32_t v = (pr << 6) + (pr & 0x00080008u) * 0xFC0u;
+        asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o[i]) : "r"(v), "r"(scale2m1));
+    }
+}
+// bf16x2 of 2^(s - 1) for the bit-placement decode (s <= 128)
+__device__ __forceinline__ uint32_t e8m0_place_bf16x2(uint32_t s) {
+    const uint32_t b = (s + 126u) << 7;
+    return b | (b << 16);
+}
 __device__ __forceinline__ uint32_t e8m0_bf16x2(uint32_t s) {
     uint32_t b = s == 0 ? 0x0040u : (s == 255 ? 0x7FC0u : (s << 7));
     return b | (b << 16);

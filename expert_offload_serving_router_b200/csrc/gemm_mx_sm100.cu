@@ -17,17 +17,26 @@
 // hit every bank once) per 128-row group, and every fourth unit also brings the rows'
 // next 16 scale bytes (eight K steps).  The ring is three units (six K steps) deep, so the
 // global-memory latency of the weights is hidden behind the MMAs of the steps before.
-// Eight converter warps then turn one K step of codes into the bf16 A operand in the
-// 128-byte swizzle the MMA reads (one weight row per thread), with byte-permute lookups
-// for the E2M1 magnitudes and an exact power-of-two multiply by the E8M0 scale.
+// Two groups of four converter warps, taking alternate K steps, turn a K step of codes into
+// the bf16 A operand in the 128-byte swizzle the MMA reads, and arrive on the leader's barrier
+// after a proxy fence; while one group's step waits on its fence and cluster arrive, the other
+// converts.  A word of eight codes becomes four bf16x2 words by bit placement (magnitude bits
+// to bf16 bits 6..8 and the sign to bit 15 give the E2M1 value times 2^-126 exactly; one
+// `mul.rn.bf16x2` by 2^(s-1) applies the E8M0 scale); blocks whose scale byte exceeds 128
+// (2^(s-1) would not be a finite bf16) take byte-permute table lookups and a multiply by 2^(s-127).
+// At the end of a tile the same warps run the epilogue (the tile's accumulators -> h with
+// SwiGLU, or -> o_sorted): eight warps, two per TMEM lane quarter, so the kernel has ten warps
+// and 168 registers per thread.
 //
 // Warp roles (both CTAs unless stated):
-//   warp 0        TMA producer of the token tile (completion counted on the leader's barrier)
+//   warp 0        lane 0: TMA producer of the token tile (completion counted on the leader's
+//                 barrier); lane 1: TMA producer of the code units and scale groups (own CTA,
+//                 own barriers)
 //   warp 1        TMEM allocation (cta_group::2, 512 columns); in the leader, the
 //                 single-thread MMA issuer
-//   warps 2-5     epilogue: TMEM lane quarter (warp & 3), both accumulators, SwiGLU for gate/up
-//   warps 6-13    converters: thread c builds row (c & 127) of 128-row group (c >> 7)
-//   warp 14       TMA producer of the code units and scale groups (own CTA, own barriers)
+//   warps 2-9     two groups of four converter warps taking alternate K steps (thread r of a
+//                 group builds row r of both 128-row groups of its steps); at a tile's end,
+//                 its epilogue (TMEM lane quarter warp & 3, column chunks of the group's parity)
 // Every wait is bounded: on timeout a role raises the CTA's abort flag, records
 // kDevErrTimeout, drains the copies it issued, and every thread of both CTAs still reaches
 // the teardown (MMAs complete, TMEM freed).
@@ -46,15 +55,15 @@ constexpr int kMxGroupK = 512;                         // K elements per scale g
 constexpr int kMxUnitsPerGroup = kMxGroupK / kMxUnitK; // 4
 constexpr int kMxScaleHalf = 128 * 16;                 // 2 KB
 constexpr int kMxScaleTile = 2 * kMxScaleHalf;         // 4 KB
-constexpr int kMxEpiWarps = 4;
-constexpr int kMxConvWarps = 8;
-constexpr int kMxConvWarp0 = 2 + kMxEpiWarps;          // 6
-constexpr int kMxCodeWarp = kMxConvWarp0 + kMxConvWarps;   // 14
-constexpr int kMxThreads = 32 * (kMxCodeWarp + 1);     // 480
+constexpr int kMxConvWarps = 8;                        // two groups of four, alternating K steps
+constexpr int kMxConvWarp0 = 2;
+constexpr int kMxThreads = 32 * (kMxConvWarp0 + kMxConvWarps);   // 320: at most three warps per SM
+                                                                  // sub-partition, 168 registers
+constexpr int kMxXposeWarps = kMxConvWarps;
 
 __host__ __device__ constexpr size_t mx_pair_smem_bytes() {
     return 1024 + size_t(kMxSt) * (kMxATile + kMxBTile) + size_t(kMxCSt) * kMxUnitTile + 2 * kMxScaleTile +
-           kMxEpiWarps * kXposeBytes + 256 + 8 * 260;
+           kMxXposeWarps * kXposeBytes + 256 + 8 * 260;
 }
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) {
@@ -79,7 +88,7 @@ moe_gemm_mx_pair_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_c
     uint8_t* sC = sB + kMxSt * kMxBTile;
     uint8_t* sS = sC + kMxCSt * kMxUnitTile;
     uint8_t* sX = sS + 2 * kMxScaleTile;
-    uint64_t* bfull = reinterpret_cast<uint64_t*>(sX + kMxEpiWarps * kXposeBytes);
+    uint64_t* bfull = reinterpret_cast<uint64_t*>(sX + kMxXposeWarps * kXposeBytes);
     uint64_t* afull = bfull + kMxSt;
     uint64_t* empty = afull + kMxSt;
     uint64_t* cfull = empty + kMxSt;
@@ -103,7 +112,7 @@ moe_gemm_mx_pair_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_c
     if (tid == 0) {
         for (int s = 0; s < kMxSt; ++s) {
             mbar_init(&bfull[s], 1);                      // the leader's producer (both CTAs' bytes)
-            mbar_init(&afull[s], 2 * kMxConvWarps);       // every converter warp of both CTAs
+            mbar_init(&afull[s], kMxConvWarps);           // one converter group (4 warps) of each CTA
             mbar_init(&empty[s], 1);                      // the leader's MMA commit
         }
         for (int s = 0; s < kMxCSt; ++s) {
@@ -111,7 +120,7 @@ moe_gemm_mx_pair_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_c
             mbar_init(&cempty[s], kMxConvWarps);          // own converter warps
         }
         mbar_init(tfull, 1);
-        mbar_init(tempty, 2 * kMxEpiWarps);
+        mbar_init(tempty, 2 * kMxConvWarps);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -167,107 +176,8 @@ moe_gemm_mx_pair_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_c
                     if (rank == 0) mbar_wait(&bfull[s], issued_par[s], nullptr);
                     else mbar_wait(&empty[s], issued_par[s], nullptr);
                 }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer (leader only)
-        if (lane == 0) {
-            if (rank == 0) {
-                int stage = 0;
-                uint32_t phase = 0, acc_phase = 0;
-                bool ok = true;
-                for (int t = cid; t < total && ok; t += ncl) {
-                    const Tile tl = decode_tile<4>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
-                    const int N = (tl.nvalid + 15) & ~15;
-                    const uint32_t idesc = idesc_bf16(256, N);
-                    if (!mbar_wait_cluster(tempty, acc_phase ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int kb = 0; kb < nk; ++kb) {
-                        if (!mbar_wait(&bfull[stage], phase, abort_flag, p.wait_ns)) { ok = false; break; }
-                        if (!mbar_wait_cluster(&afull[stage], phase, abort_flag, p.wait_ns)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint64_t bd = sdesc_sw128(su32(sB + stage * kMxBTile));
-                        for (int h = 0; h < 2; ++h) {
-                            const uint64_t ad = sdesc_sw128(su32(sA + stage * kMxATile + h * kAHalfBytes));
-                            const uint32_t dtm = tmem_base + uint32_t(h * kAccCols);
-#pragma unroll
-                            for (int kk = 0; kk < kBK / 16; ++kk)
-                                umma_bf16_pair(dtm, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
-                        }
-                        umma_commit_pair_both(&empty[stage]);
-                        if (++stage == kMxSt) { stage = 0; phase ^= 1; }
-                    }
-                    if (!ok) break;
-                    umma_commit_pair_both(tfull);
-                    acc_phase ^= 1;
-                }
-                if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
-                umma_commit_pair_both(mma_done);     // completion of every MMA issued above, in both CTAs
-            }
-            mbar_wait(mma_done, 0, nullptr);
-        }
-    } else if (warp < kMxConvWarp0) {
-        // ------------------------------------------------ epilogue (both CTAs, own 128 rows)
-        const int q = warp & 3;
-        uint16_t* xb = reinterpret_cast<uint16_t*>(sX + (warp - 2) * kXposeBytes);
-        uint32_t acc_phase = 0;
-        bool ok = true;
-        for (int t = cid; t < total; t += ncl) {
-            const Tile tl = decode_tile<4>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
-            if (!mbar_wait(tfull, acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
-            tc_fence_after();
-            epilogue_tile<1>(p, tl, 2, tmem_base + (uint32_t(q * 32) << 16), tl.m * 4 + int(rank), 2, q, 0, lane, xb);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(tempty_lead);
-            acc_phase ^= 1;
-        }
-        if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
-    } else if (warp < kMxCodeWarp) {
-        // ------------------------------------------------ converters: codes (smem) -> bf16 A (smem)
-        const int ct = tid - 32 * kMxConvWarp0;   // 0..255
-        const int h = ct >> 7, row = ct & 127;
-        const int xsw = (row >> 1) & 3;          // SW64 chunk permutation of this code row
-        int stage = 0, cst = 0, grp = 0;
-        uint32_t phase = 0, cph = 0;
-        uint4 sreg = make_uint4(0, 0, 0, 0);
-        bool ok = true;
-        for (int t = cid; t < total && ok; t += ncl) {
-            for (int kb = 0; kb < nk; ++kb) {
-                const int j = kb & 1;
-                if (j == 0 && !mbar_wait(&cfull[cst], cph, abort_flag, p.wait_ns)) { ok = false; break; }
-                if ((kb & 7) == 0)
-                    sreg = lds128(sS + (grp & 1) * kMxScaleTile + h * kMxScaleHalf + row * 16);
-                const uint8_t* crow = sC + cst * kMxUnitTile + h * kMxUnitHalf + row * 64;
-                const uint4 c0 = lds128(crow + (((2 * j) ^ xsw) << 4));
-                const uint4 c1 = lds128(crow + (((2 * j + 1) ^ xsw) << 4));
-                if (j == 1) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&cempty[cst]);
-                    if (++cst == kMxCSt) { cst = 0; cph ^= 1; }
-                }
-                if ((kb & 7) == 7) ++grp;
-                const uint32_t sw = (kb & 4) ? ((kb & 2) ? sreg.w : sreg.z) : ((kb & 2) ? sreg.y : sreg.x);
-                const uint32_t sp = sw >> (16 * (kb & 1));
-                const uint32_t s0 = e8m0_bf16x2(sp & 0xFF), s1 = e8m0_bf16x2((sp >> 8) & 0xFF);
-                if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
-                uint8_t* arow = sA + stage * kMxATile + h * kAHalfBytes + row * 128;
-                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-                for (int cch = 0; cch < 8; ++cch) {   // 16-byte chunk cch = elements 8cch .. 8cch+7
-                    uint32_t o[4];
-                    e2m1x8_bf16(words[cch], cch < 4 ? s0 : s1, o);
-                    sts128(arow + ((cch ^ (row & 7)) << 4), o[0], o[1], o[2], o[3]);
-                }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(afull_lead + uint32_t(stage) * 8u);
-                if (++stage == kMxSt) { stage = 0; phase ^= 1; }
-            }
-        }
-        if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
-    } else {
-        // ------------------------------------------------ code-unit + scale-group producer (own CTA)
-        if (lane == 0) {
+        } else if (lane == 1) {
+            // -------------------------------------------- code-unit + scale-group producer (own CTA)
             int cst = 0, grp = 0;
             uint32_t cph = 0;
             int issued[kMxCSt];
@@ -308,6 +218,125 @@ moe_gemm_mx_pair_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_c
             for (int s = 0; s < kMxCSt; ++s)
                 if (issued[s]) mbar_wait(&cfull[s], issued_par[s], nullptr);
         }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (lane == 0) {
+            if (rank == 0) {
+                int stage = 0;
+                uint32_t phase = 0, acc_phase = 0;
+                bool ok = true;
+                for (int t = cid; t < total && ok; t += ncl) {
+                    const Tile tl = decode_tile<4>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+                    const int N = (tl.nvalid + 15) & ~15;
+                    const uint32_t idesc = idesc_bf16(256, N);
+                    if (!mbar_wait_cluster(tempty, acc_phase ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int kb = 0; kb < nk; ++kb) {
+                        if (!mbar_wait(&bfull[stage], phase, abort_flag, p.wait_ns)) { ok = false; break; }
+                        if (!mbar_wait_cluster(&afull[stage], phase, abort_flag, p.wait_ns)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint64_t bd = sdesc_sw128(su32(sB + stage * kMxBTile));
+                        for (int h = 0; h < 2; ++h) {
+                            const uint64_t ad = sdesc_sw128(su32(sA + stage * kMxATile + h * kAHalfBytes));
+                            const uint32_t dtm = tmem_base + uint32_t(h * kAccCols);
+#pragma unroll
+                            for (int kk = 0; kk < kBK / 16; ++kk)
+                                umma_bf16_pair(dtm, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+                        }
+                        umma_commit_pair_both(&empty[stage]);
+                        if (++stage == kMxSt) { stage = 0; phase ^= 1; }
+                    }
+                    if (!ok) break;
+                    umma_commit_pair_both(tfull);
+                    acc_phase ^= 1;
+                }
+                if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+                umma_commit_pair_both(mma_done);     // completion of every MMA issued above, in both CTAs
+            }
+            mbar_wait(mma_done, 0, nullptr);
+        }
+    } else {
+        // ------------------------------------------------ converters: codes (smem) -> bf16 A (smem)
+        // Two groups of four warps take alternate K steps (group gi the steps n = gi mod 2 of
+        // the CTA's running step count n, i.e. half gi of every code unit), so the latency of
+        // one step's conversion, proxy fence and cluster arrive overlaps the other group's
+        // step.  Thread `row` of a group builds that row of both 128-row groups of the stage.
+        const int gi = (warp - kMxConvWarp0) >> 2;
+        const int row = tid - 32 * kMxConvWarp0 - 128 * gi;   // 0..127
+        const int xsw = (row >> 1) & 3;                       // SW64 chunk permutation of this code row
+        uint4 sreg[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        bool ok = true;
+        int n = gi;                                           // this CTA's running K-step index
+        uint32_t acc_phase = 0;
+        for (int t = cid; t < total && ok; t += ncl) {
+            for (int kb = gi; kb < nk; kb += 2, n += 2) {
+                const int u = n >> 1;                         // code unit; its half j = gi
+                const int cst = u % kMxCSt;
+                const uint32_t cph = uint32_t(u / kMxCSt) & 1u;
+                const int stage = n % kMxSt;
+                const uint32_t phase = uint32_t(n / kMxSt) & 1u;
+                if (!mbar_wait(&cfull[cst], cph, abort_flag, p.wait_ns)) { ok = false; break; }
+                if ((kb & 7) < 2)                             // first step of a scale group this group sees
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        sreg[h] = lds128(sS + ((n >> 3) & 1) * kMxScaleTile + h * kMxScaleHalf + row * 16);
+                uint4 c0[2], c1[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint8_t* crow = sC + cst * kMxUnitTile + h * kMxUnitHalf + row * 64;
+                    c0[h] = lds128(crow + (((2 * gi) ^ xsw) << 4));
+                    c1[h] = lds128(crow + (((2 * gi + 1) ^ xsw) << 4));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cempty[cst]);
+                if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint4 sv = sreg[h];
+                    const uint32_t sw = (kb & 4) ? ((kb & 2) ? sv.w : sv.z) : ((kb & 2) ? sv.y : sv.x);
+                    const uint32_t sp = sw >> (16 * (kb & 1));
+                    const uint32_t b0 = sp & 0xFF, b1 = (sp >> 8) & 0xFF;
+                    const bool place = b0 <= 128u && b1 <= 128u;   // 2^(s-1) finite in bf16
+                    const uint32_t s0 = place ? e8m0_place_bf16x2(b0) : e8m0_bf16x2(b0);
+                    const uint32_t s1 = place ? e8m0_place_bf16x2(b1) : e8m0_bf16x2(b1);
+                    uint8_t* arow = sA + stage * kMxATile + h * kAHalfBytes + row * 128;
+                    const uint32_t words[8] = {c0[h].x, c0[h].y, c0[h].z, c0[h].w, c1[h].x, c1[h].y, c1[h].z, c1[h].w};
+                    if (place) {
+#pragma unroll
+                        for (int cch = 0; cch < 8; ++cch) {
+                            uint32_t o[4];
+                            e2m1x8_bf16_place(words[cch], cch < 4 ? s0 : s1, o);
+                            sts128(arow + ((cch ^ (row & 7)) << 4), o[0], o[1], o[2], o[3]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int cch = 0; cch < 8; ++cch) {   // 16-byte chunk cch = elements 8cch .. 8cch+7
+                            uint32_t o[4];
+                            e2m1x8_bf16(words[cch], cch < 4 ? s0 : s1, o);
+                            sts128(arow + ((cch ^ (row & 7)) << 4), o[0], o[1], o[2], o[3]);
+                        }
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(afull_lead + uint32_t(stage) * 8u);
+            }
+            if (ok) {
+                // this tile's accumulators -> h / o_sorted: warp (lane quarter warp & 3) takes
+                // the column chunks of parity gi
+                const Tile tl = decode_tile<4>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+                if (!mbar_wait(tfull, acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
+                tc_fence_after();
+                uint16_t* xb = reinterpret_cast<uint16_t*>(sX + (warp - kMxConvWarp0) * kXposeBytes);
+                epilogue_tile<2>(p, tl, 2, tmem_base + (uint32_t((warp & 3) * 32) << 16), tl.m * 4 + int(rank), 2,
+                                 warp & 3, gi, lane, xb);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(tempty_lead);
+                acc_phase ^= 1;
+            }
+        }
+        if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
     }
     // teardown: every MMA of the pair is complete (mma_done) and both CTAs are past their last
     // TMEM read and remote arrival before the pair's TMEM is freed and either CTA exits
