@@ -277,36 +277,59 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
     }
 }
 
-// ------------------------------------------------------------------ CTA-pair gate/up (BF16)
+// ------------------------------------------------------------------ CTA pairs (BF16)
 // Two CTAs of a cluster share every MMA (tcgen05.mma.cta_group::2, M = 256): CTA r supplies
 // 128 weight rows of each MMA and half of the token tile (rows r*N/2 .. of it) from its own
-// shared memory and keeps its 128 accumulator rows in its own TMEM.  A pair tile is 512
-// weight rows (two MMAs, four 128-row groups: CTA r holds groups 4m + r and 4m + 2 + r) x up
-// to 256 tokens.  Per SM a stage then carries 32 KB of weights and at most 16 KB of tokens
-// for the same MMA work as the single-CTA 256 x 256 tile's 64 KB, so four stages fit.
+// shared memory and keeps its 128 accumulator rows in its own TMEM.
+//   HPC = 2 (gate/up, long K): a pair tile is 512 weight rows (two MMAs, four 128-row groups:
+//           CTA r holds groups 4m + r and 4m + 2 + r) x up to 256 tokens; both accumulators
+//           (2 x 256 columns) belong to one tile.  Per SM a stage carries 32 KB of weights and
+//           at most 16 KB of tokens for the work the single-CTA 256 x 256 tile does with 64 KB,
+//           so four stages fit.
+//   HPC = 1 (down, short K): a pair tile is 256 weight rows (one MMA, CTA r holds group
+//           2m + r) x up to 256 tokens; the accumulators are double buffered (2 x 256 columns)
+//           so a tile's epilogue overlaps the next tile's MMAs, and six 32 KB stages fit.  Each
+//           CTA reads half the token tile of the single-CTA kernel per FLOP (the token tile is
+//           the larger operand of the down GEMM).
+// A group index at or beyond m_rows (the last pair tile of an odd group count) is zero-filled
+// by TMA and its results are not stored.
 // Only the leader (rank 0) waits for operands and issues MMAs: both CTAs' TMA copies count on
 // its `full` barrier, its commits arrive on the `empty` / `tfull` / `done` barriers of both
 // CTAs, and both CTAs' epilogue warps arrive on its `tempty` barrier.  No TMA multicast.
-constexpr int kPairSt = 4;
-constexpr int kPairATile = 2 * kAHalfBytes;            // 32 KB: two 128-row weight groups
 constexpr int kPairBTile = 128 * kBK * 2;              // 16 KB: up to 128 token rows
+template <int HPC> struct PairCfg {
+    static constexpr int kATile = HPC * kAHalfBytes;
+    static constexpr int kSt = HPC == 2 ? 4 : 6;
+    static constexpr int kNBuf = HPC == 2 ? 1 : 2;
+    static constexpr int kGroups = 2 * HPC;            // 128-row groups per pair tile
+    static constexpr size_t smem() {
+        return 1024 + size_t(kSt) * (kATile + kPairBTile) + 8 * kXposeBytes + 256 + 8 * 260;
+    }
+};
 
+template <int HPC>
+__device__ __forceinline__ int pair_group(int m, int h, uint32_t rank) {
+    return HPC == 2 ? m * 4 + 2 * h + int(rank) : m * 2 + int(rank);
+}
+
+template <int HPC>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 moe_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sw,
                      const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
                      const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_b3,
                      const __grid_constant__ CUtensorMap tm_b4, GemmParams p) {
+    using C = PairCfg<HPC>;
     constexpr int kEpiWarps = 8;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + kPairSt * kPairATile;
-    uint8_t* sX = sB + kPairSt * kPairBTile;
+    uint8_t* sB = smem + C::kSt * C::kATile;
+    uint8_t* sX = sB + C::kSt * kPairBTile;
     uint64_t* full = reinterpret_cast<uint64_t*>(sX + kEpiWarps * kXposeBytes);
-    uint64_t* empty = full + kPairSt;
-    uint64_t* tfull = empty + kPairSt;
-    uint64_t* tempty = tfull + 1;
-    uint64_t* mma_done = tempty + 1;
+    uint64_t* empty = full + C::kSt;
+    uint64_t* tfull = empty + C::kSt;
+    uint64_t* tempty = tfull + C::kNBuf;
+    uint64_t* mma_done = tempty + C::kNBuf;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* ntile_off = const_cast<int*>(reinterpret_cast<volatile int*>(tmem_slot + 2));
@@ -321,12 +344,14 @@ moe_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
         s_off[i] = p.offsets[i];
     }
     if (tid == 0) {
-        for (int st = 0; st < kPairSt; ++st) {
+        for (int st = 0; st < C::kSt; ++st) {
             mbar_init(&full[st], 1);            // the leader's producer arrives (with all bytes expected)
             mbar_init(&empty[st], 1);           // the leader's MMA commit
         }
-        mbar_init(tfull, 1);
-        mbar_init(tempty, 2 * kEpiWarps);       // every epilogue warp of both CTAs
+        for (int b = 0; b < C::kNBuf; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 2 * kEpiWarps);   // every epilogue warp of both CTAs
+        }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -353,12 +378,12 @@ moe_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
             const CUtensorMap* bm[kNumBMaps] = {&tm_b0, &tm_b1, &tm_b2, &tm_b3, &tm_b4};
             int stage = 0;
             uint32_t phase = 0;
-            int issued[kPairSt];
-            uint32_t issued_par[kPairSt];
-            for (int st = 0; st < kPairSt; ++st) issued[st] = 0;
+            int issued[C::kSt];
+            uint32_t issued_par[C::kSt];
+            for (int st = 0; st < C::kSt; ++st) issued[st] = 0;
             bool ok = true;
             for (int t = cid; t < total && ok; t += ncl) {
-                const Tile tl = decode_tile<4>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+                const Tile tl = decode_tile<C::kGroups>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
                 const bool shared_grp = p.has_shared && tl.g == p.E;
                 const int nh = ((tl.nvalid + 15) & ~15) >> 1;   // token rows per CTA
                 int bi = 0;
@@ -368,25 +393,26 @@ moe_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                 const int e = shared_grp ? 0 : tl.g;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
-                    uint8_t* a = sA + stage * kPairATile;
+                    uint8_t* a = sA + stage * C::kATile;
                     uint8_t* b = sB + stage * kPairBTile;
                     const int k0 = kb * kBK;
                     const uint32_t bar = full_lead + uint32_t(stage) * 8u;
-                    if (rank == 0) mbar_expect_tx(&full[stage], 2u * (uint32_t(kPairATile) + bbytes));
-                    for (int h = 0; h < 2; ++h) {
-                        const int rg = tl.m * 4 + 2 * h + int(rank);
-                        tma_5d_pair(m, bar, a + h * kAHalfBytes, k0, 0, 0, rg * 4, e);
+                    if (rank == 0) mbar_expect_tx(&full[stage], 2u * (uint32_t(C::kATile) + bbytes));
+                    for (int h = 0; h < HPC; ++h) {
+                        const int rg = pair_group<HPC>(tl.m, h, rank);
+                        if (p.mode == 0) tma_5d_pair(m, bar, a + h * kAHalfBytes, k0, 0, 0, rg * 4, e);
+                        else tma_3d_pair(m, bar, a + h * kAHalfBytes, k0, rg * 128, e);
                     }
                     tma_2d_pair(bm[bi], bar, b, k0, tl.row0 + int(rank) * nh);
                     issued[stage] = 1;
                     issued_par[stage] = phase;
-                    if (++stage == kPairSt) { stage = 0; phase ^= 1; }
+                    if (++stage == C::kSt) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
             // drain: the leader sees its full barriers complete (both CTAs' bytes landed); the
             // peer sees its empty barriers released (the leader consumed what it copied)
-            for (int st = 0; st < kPairSt; ++st)
+            for (int st = 0; st < C::kSt; ++st)
                 if (issued[st]) {
                     if (rank == 0) mbar_wait(&full[st], issued_par[st], nullptr);
                     else mbar_wait(&empty[st], issued_par[st], nullptr);
@@ -396,32 +422,32 @@ moe_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
         // ------------------------------------------------ MMA issuer (leader only)
         if (lane == 0) {
             if (rank == 0) {
-                int stage = 0;
+                int stage = 0, buf = 0;
                 uint32_t phase = 0, acc_phase = 0;
                 bool ok = true;
                 for (int t = cid; t < total && ok; t += ncl) {
-                    const Tile tl = decode_tile<4>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+                    const Tile tl = decode_tile<C::kGroups>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
                     const int N = (tl.nvalid + 15) & ~15;
                     const uint32_t idesc = idesc_bf16(256, N);
-                    if (!mbar_wait_cluster(tempty, acc_phase ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
+                    if (!mbar_wait_cluster(&tempty[buf], acc_phase ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
                     tc_fence_after();
                     for (int kb = 0; kb < nk; ++kb) {
                         if (!mbar_wait(&full[stage], phase, abort_flag, p.wait_ns)) { ok = false; break; }
                         tc_fence_after();
                         const uint64_t bd = sdesc_sw128(su32(sB + stage * kPairBTile));
-                        for (int h = 0; h < 2; ++h) {
-                            const uint64_t ad = sdesc_sw128(su32(sA + stage * kPairATile + h * kAHalfBytes));
-                            const uint32_t dtm = tmem_base + uint32_t(h * kAccCols);
+                        for (int h = 0; h < HPC; ++h) {
+                            const uint64_t ad = sdesc_sw128(su32(sA + stage * C::kATile + h * kAHalfBytes));
+                            const uint32_t dtm = tmem_base + uint32_t((buf * HPC + h) * kAccCols);
 #pragma unroll
                             for (int kk = 0; kk < kBK / 16; ++kk)
                                 umma_bf16_pair(dtm, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
                         }
                         umma_commit_pair_both(&empty[stage]);
-                        if (++stage == kPairSt) { stage = 0; phase ^= 1; }
+                        if (++stage == C::kSt) { stage = 0; phase ^= 1; }
                     }
                     if (!ok) break;
-                    umma_commit_pair_both(tfull);
-                    acc_phase ^= 1;
+                    umma_commit_pair_both(&tfull[buf]);
+                    if (++buf == C::kNBuf) { buf = 0; acc_phase ^= 1; }
                 }
                 if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
                 umma_commit_pair_both(mma_done);     // completion of every MMA issued above, in both CTAs
@@ -434,18 +460,23 @@ moe_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
         const int part = (warp - 2) >> 2;
         constexpr int kParts = kEpiWarps / 4;
         uint16_t* xb = reinterpret_cast<uint16_t*>(sX + (warp - 2) * kXposeBytes);
+        int buf = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
         for (int t = cid; t < total; t += ncl) {
-            const Tile tl = decode_tile<4>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
-            if (!mbar_wait(tfull, acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
+            const Tile tl = decode_tile<C::kGroups>(t, ntile_off, G, s_off, p.m_tiles, p.m_rows);
+            if (!mbar_wait(&tfull[buf], acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
-            epilogue_tile<kParts>(p, tl, 2, tmem_base + (uint32_t(q * 32) << 16), tl.m * 4 + int(rank), 2, q, part,
-                                  lane, xb);
+            const int rg0 = pair_group<HPC>(tl.m, 0, rank);
+            // groups past the weight rows (odd group counts) were zero-filled: nothing to store
+            const int halves = HPC == 2 ? (rg0 + 2 < p.m_rows ? 2 : (rg0 < p.m_rows ? 1 : 0)) : (rg0 < p.m_rows ? 1 : 0);
+            if (halves)
+                epilogue_tile<kParts>(p, tl, halves, tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * HPC * kAccCols),
+                                      rg0, 2, q, part, lane, xb);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(tempty_lead);
-            acc_phase ^= 1;
+            if (lane == 0) mbar_arrive_cluster(tempty_lead + uint32_t(buf) * 8u);
+            if (++buf == C::kNBuf) { buf = 0; acc_phase ^= 1; }
         }
         if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
     }
@@ -480,6 +511,47 @@ static int launch_variant(int grid, cudaStream_t st, const CUtensorMap& tw, cons
         set = true;
     }
     moe_gemm_kernel<MX, HV><<<grid, 320, smem, st>>>(tw, tsw, tb[0], tb[1], tb[2], tb[3], tb[4], p);
+    return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
+
+template <int HPC>
+static int launch_pair(const GemmLaunch& L, const GemmParams& p, const CUtensorMap& tw, const CUtensorMap& tsw,
+                       cudaStream_t st) {
+    using C = PairCfg<HPC>;
+    const int K = p.K;
+    // each CTA loads half of a token tile, so the token boxes are 8 .. 128 rows
+    GemmParams pp = p;
+    pp.m_tiles = (p.m_rows + C::kGroups - 1) / C::kGroups;
+    CUtensorMap tbp[kNumBMaps]{};
+    const int rR8 = (L.R + 7) & ~7;
+    for (int i = 0; i < kNumBMaps; ++i) {
+        pp.b_rows[i] = (8 << i) < rR8 ? (8 << i) : rR8;
+        uint64_t dims[2] = {uint64_t(K), uint64_t(L.R)};
+        uint64_t str[1] = {uint64_t(K) * 2};
+        uint32_t box[2] = {kBK, uint32_t(pp.b_rows[i])};
+        if (!make_map(&tbp[i], L.act, 2, dims, str, box)) return 1;
+    }
+    static int max_clusters = 0;
+    constexpr size_t smem = C::smem();
+    if (!max_clusters) {
+        if (cudaFuncSetAttribute(moe_gemm_pair_kernel<HPC>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+            cudaSuccess)
+            return 2;
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(2 * (num_sms() / 2));
+        cfg.blockDim = dim3(320);
+        cfg.dynamicSmemBytes = smem;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, moe_gemm_pair_kernel<HPC>, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = num_sms() / 2;
+        }
+        max_clusters = n;
+    }
+    int clusters = max_clusters;
+    const int pair_tiles = L.max_tiles * pp.m_tiles;
+    if (pair_tiles < clusters) clusters = pair_tiles > 0 ? pair_tiles : 1;
+    moe_gemm_pair_kernel<HPC><<<2 * clusters, 320, smem, st>>>(tw, tsw, tbp[0], tbp[1], tbp[2], tbp[3], tbp[4], pp);
     return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
 
@@ -550,42 +622,10 @@ int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st) {
     p.swq = static_cast<const uint8_t*>(L.sw);
     p.sws = L.swscale;
     if (mx && mx_pair_eligible(L.mode, L.H, L.F)) return launch_moe_gemm_mx_pair(L, p, st);
-    if (!mx && L.mode == 0 && hv == 2 && p.m_rows % 4 == 0) {
-        // CTA pairs: each CTA loads half of a token tile, so the token boxes are 8 .. 128 rows
-        GemmParams pp = p;
-        pp.m_tiles = p.m_rows / 4;
-        CUtensorMap tbp[kNumBMaps]{};
-        const int rR8 = (L.R + 7) & ~7;
-        for (int i = 0; i < kNumBMaps; ++i) {
-            pp.b_rows[i] = (8 << i) < rR8 ? (8 << i) : rR8;
-            uint64_t dims[2] = {uint64_t(K), uint64_t(L.R)};
-            uint64_t str[1] = {uint64_t(K) * 2};
-            uint32_t box[2] = {kBK, uint32_t(pp.b_rows[i])};
-            if (!make_map(&tbp[i], L.act, 2, dims, str, box)) return 1;
-        }
-        static int max_clusters = 0;
-        const size_t smem = 1024 + size_t(kPairSt) * (kPairATile + kPairBTile) + 8 * kXposeBytes + 256 + 8 * 260;
-        if (!max_clusters) {
-            if (cudaFuncSetAttribute(moe_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-                cudaSuccess)
-                return 2;
-            cudaLaunchConfig_t cfg{};
-            cfg.gridDim = dim3(2 * (num_sms() / 2));
-            cfg.blockDim = dim3(320);
-            cfg.dynamicSmemBytes = smem;
-            int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, moe_gemm_pair_kernel, &cfg) != cudaSuccess || n <= 0) {
-                cudaGetLastError();
-                n = num_sms() / 2;
-            }
-            max_clusters = n;
-        }
-        int clusters = max_clusters;
-        const int pair_tiles = L.max_tiles * pp.m_tiles;
-        if (pair_tiles < clusters) clusters = pair_tiles > 0 ? pair_tiles : 1;
-        moe_gemm_pair_kernel<<<2 * clusters, 320, smem, st>>>(tw, tsw, tbp[0], tbp[1], tbp[2], tbp[3], tbp[4], pp);
-        return cudaGetLastError() == cudaSuccess ? 0 : 2;
-    }
+    // BF16 on CTA pairs: gate/up of long contractions in pair tiles of 512 weight rows (four
+    // 128-row groups), down in pair tiles of 256 rows with double-buffered accumulators
+    if (!mx && L.mode == 0 && hv == 2 && p.m_rows % 4 == 0) return launch_pair<2>(L, p, tw, tsw, st);
+    if (!mx && L.mode == 1 && p.m_rows % 2 == 0) return launch_pair<1>(L, p, tw, tsw, st);
     int grid = num_sms();
     const int max_tiles = L.max_tiles * p.m_tiles;
     if (max_tiles < grid) grid = max_tiles > 0 ? max_tiles : 1;

@@ -41,7 +41,7 @@ static __device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, vola
     const uint64_t t0 = gtimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try(b, parity)) return true;
-        if ((i & 31) == 0) {
+        if ((i & 31) == 0 || limit < kWaitNs) {   // a shortened bound is checked on every poll
             if (abort && *abort) return false;
             if (gtimer() - t0 > limit) return false;
         }
@@ -163,7 +163,7 @@ static __device__ __noinline__ bool mbar_wait_cluster(uint64_t* b, uint32_t pari
     const uint64_t t0 = gtimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_acq_cluster(b, parity)) return true;
-        if ((i & 31) == 0) {
+        if ((i & 31) == 0 || limit < kWaitNs) {   // a shortened bound is checked on every poll
             if (abort && *abort) return false;
             if (gtimer() - t0 > limit) return false;
         }
@@ -175,6 +175,11 @@ __device__ __forceinline__ void tma_2d_pair(const CUtensorMap* m, uint32_t bar_c
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
         ::"r"(su32(dst)), "l"(m), "r"(bar_cluster), "r"(c0), "r"(c1) : "memory");
+}
+__device__ __forceinline__ void tma_3d_pair(const CUtensorMap* m, uint32_t bar_cluster, void* dst, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(su32(dst)), "l"(m), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2) : "memory");
 }
 __device__ __forceinline__ void tma_5d_pair(const CUtensorMap* m, uint32_t bar_cluster, void* dst, int c0, int c1, int c2,
                                             int c3, int c4) {
