@@ -581,7 +581,8 @@ def measure_stack(torch, F, rank, hbm_gbs):
 def measure_hbm_ceiling(torch, sizes_mb=(8, 16, 32, 64, 76, 128, 256, 512, 1024, 2048), iters=20):
     """Streaming throughput a plain read (torch's float32 sum) and a device-to-device copy reach
     for transfers of a given size, rotating over enough buffers (>= 1 GiB together) that L2 never
-    holds the next one.  GB/s counts the bytes read (read) or read + written (copy)."""
+    holds the next one, replayed back to back from a CUDA graph.  GB/s counts the bytes read
+    (read) or read + written (copy)."""
     out = []
     for mb in sizes_mb:
         n = mb << 20
@@ -594,16 +595,26 @@ def measure_hbm_ceiling(torch, sizes_mb=(8, 16, 32, 64, 76, 128, 256, 512, 1024,
                 if kind == "read":
                     return bufs[i % k].sum()
                 return dst.copy_(bufs[i % k])
-            for i in range(3):
-                op(i)
+            # the timed reads are replayed from a CUDA graph, so host launch overhead is not counted
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                for i in range(3):
+                    op(i)
+            side.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                for i in range(iters):
+                    op(i)
+            g.replay()
             torch.cuda.synchronize()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            for i in range(iters):
-                op(i)
+            g.replay()
             e1.record()
             torch.cuda.synchronize()
             us = e0.elapsed_time(e1) * 1e3 / iters
+            del g
             moved = n if kind == "read" else 2 * n
             row[kind] = {"us": us, "gbs": moved / (us * 1e-6) / 1e9}
         out.append(row)

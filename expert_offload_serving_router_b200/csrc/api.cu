@@ -123,6 +123,7 @@ DecodeArgs decode_args(const ft_moe_shape* s, int T, const ft_moe_weights* w, co
     a.y = static_cast<uint16_t*>(y);
     a.o_sorted = static_cast<uint16_t*>(o_sorted);
     a.err = ws_at<uint32_t>(ws, L.err);
+    a.o_ws = ws_at<uint16_t>(ws, L.o_sorted);
     return a;
 }
 

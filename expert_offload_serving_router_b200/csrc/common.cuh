@@ -82,8 +82,10 @@ struct WsLayout {
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace header (cleared by ft_moe_workspace_init): word 0 device error flag, word 1 the
-// decode router's ticket (every launch leaves it at zero).
-constexpr size_t kWsHeaderBytes = 256;
+// decode router's ticket, words kWsDownTicket.. one ticket per 32 hidden rows for the
+// tensor-core decode's combine (every launch leaves the tickets at zero).
+constexpr size_t kWsHeaderBytes = 4096;
+constexpr int kWsDownTicket = 64;      // word index; 16384 / 32 = 512 tickets fit
 constexpr int kRouteTok = 128;          // tokens per router CTA
 constexpr int kRouteTargetCtas = 148;   // split K until the router grid covers about one wave
 constexpr int kRouteMaxSplit = 8;
@@ -109,7 +111,7 @@ inline WsLayout make_layout(const ft_moe_shape& s, int T) {
     if (L.C < 1) L.C = 1;
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t r = o; o = align256(o + bytes); return r; };
-    L.err = take(kWsHeaderBytes);   // first: [0] device error flag, [1] decode-router ticket
+    L.err = take(kWsHeaderBytes);   // first: [0] device error flag, [1] decode-router ticket, down tickets
     L.logits = take(sizeof(float) * size_t(T) * s.num_experts);
     L.topk_idx = take(sizeof(int32_t) * size_t(L.P));
     L.topk_w = take(sizeof(float) * size_t(L.P));

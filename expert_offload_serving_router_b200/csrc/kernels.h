@@ -38,6 +38,7 @@ struct DecodeArgs {
     uint16_t* y;                // [T, H] or NULL
     uint16_t* o_sorted;         // [R, H] when y == NULL
     uint32_t* err;              // workspace device error flag
+    uint16_t* o_ws;             // workspace [R, H] rows for the tensor-core decode's combine
 };
 
 struct GemmLaunch {
@@ -84,6 +85,9 @@ cudaError_t launch_permute(int T, int k, int E, int S, int H, const int32_t* idx
                            uint16_t* x_sorted, int32_t* chunk_cnt, int32_t* chunk_base, int32_t* local_rank,
                            const PermOut& out, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+// tensor-core decode (BF16, contiguous weights): false when the shape or weights do not qualify
+bool decode_mma_eligible(const DecodeArgs& a);
+cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st);
 int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st);
 // bound (ns without progress) on each pipeline wait of the grouped GEMMs (api.cu)
 unsigned long long gemm_wait_ns();

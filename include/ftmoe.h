@@ -149,8 +149,9 @@ uint64_t ft_set_pipeline_wait_limit_ns(uint64_t ns);
 size_t ft_moe_workspace_bytes(const ft_moe_shape* shape, int32_t max_tokens);
 
 /* Clears the device status words at the start of a freshly allocated
- * workspace (ws: device, 256-byte aligned, >= 256 bytes): the error flag and
- * the decode router's last-CTA ticket, which every call leaves at zero again.
+ * workspace (ws: device, 256-byte aligned, >= 4096 bytes): the error flag and
+ * the last-CTA tickets of the decode kernels, which every call leaves at zero
+ * again.
  * Call once per workspace before its first use; enqueued on `stream`. */
 ft_status ft_moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 

@@ -38,10 +38,11 @@ def full_check(L, x, n_rows=12, seed=0):
     return y, idx, lg, rel
 
 
-# decode batches whose token rows exceed 64 KB of x (qwen3_a3b T=32, dsv4_flash T=20,
-# gemma4_26b_a4b T=16) take the GEMV variant that stages each group's rows per batch
-CASES = [("tiny", 64), ("tiny", 1), ("tiny", 37),
-         ("qwen3_a3b", 1), ("qwen3_a3b", 4), ("qwen3_a3b", 16), ("qwen3_a3b", 32), ("qwen3_a3b", 4096),
+# decode batches: BF16 T >= 8 run on the tensor cores (qwen3_a3b 8/16/32, gemma4_26b_a4b 16,
+# tiny 8), smaller ones and MXFP4 on the GEMVs; MXFP4 batches whose token rows exceed 64 KB of x
+# (dsv4_flash T=20) take the GEMV variant that stages each group's rows per batch
+CASES = [("tiny", 64), ("tiny", 1), ("tiny", 37), ("tiny", 8),
+         ("qwen3_a3b", 1), ("qwen3_a3b", 4), ("qwen3_a3b", 8), ("qwen3_a3b", 16), ("qwen3_a3b", 32), ("qwen3_a3b", 4096),
          ("dsv4_flash", 1), ("dsv4_flash", 8), ("dsv4_flash", 20), ("dsv4_flash", 8192),
          ("gemma4_26b_a4b", 1), ("gemma4_26b_a4b", 16), ("gemma4_26b_a4b", 2048)]
 
@@ -190,7 +191,7 @@ def test_empty_batch_is_a_noop():
 
 
 @pytest.mark.parametrize("name,T", [("qwen3_a3b", 1), ("dsv4_flash", 1), ("gemma4_26b_a4b", 1), ("qwen3_a3b", 4),
-                                    ("tiny", 64)])
+                                    ("qwen3_a3b", 8), ("gemma4_26b_a4b", 16), ("tiny", 64)])
 def test_chained_layers_without_host_sync(name, T):
     """Layer calls back to back on one stream, each consuming the previous output: the
     dependent-launch overlap between calls must never let a kernel read an input before the
