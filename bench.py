@@ -53,21 +53,32 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def recorded_traffic(summary: str, source: str):
-    """DRAM bytes (read + write) per launch from a committed ncu summary under profiles/,
-    or None when the summary is missing or the kernel source changed since the capture."""
+def sources_sha1(sources) -> str:
+    """sha1 over the listed csrc files, in order (the sources a profiled kernel is built from)."""
     import hashlib
-    p = os.path.join(ROOT, "profiles", summary)
-    src = os.path.join(ROOT, "expert_offload_serving_router_b200", "csrc", source)
-    if not os.path.exists(p) or not os.path.exists(src):
-        return None
+    h = hashlib.sha1()
+    for src in sources:
+        h.update(open(os.path.join(ROOT, "expert_offload_serving_router_b200", "csrc", src), "rb").read())
+    return h.hexdigest()
+
+
+def recorded_traffic(summary: str, sources):
+    """DRAM bytes (read + write) per launch from a committed ncu summary under profiles/,
+    or None when the summary is missing or the kernel's sources changed since the capture."""
     import re
+    p = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(p):
+        return None
+    try:
+        sha = sources_sha1(sources)
+    except OSError:
+        return None
     fields = {}
     for line in open(p):
-        m = re.match(r"\s*-?\s*(dram_bytes_per_launch|kernel_source_sha1):\s*`?([0-9a-fA-F.]+)`?", line)
+        m = re.match(r"\s*-?\s*(dram_bytes_per_launch|kernel_sources_sha1):\s*`?([0-9a-fA-F.]+)`?", line)
         if m:
             fields[m.group(1)] = m.group(2)
-    if fields.get("kernel_source_sha1") != hashlib.sha1(open(src, "rb").read()).hexdigest():
+    if fields.get("kernel_sources_sha1") != sha:
         return None
     try:
         return float(fields["dram_bytes_per_launch"])
@@ -578,24 +589,26 @@ def measure_stack(torch, F, rank, hbm_gbs):
     return out
 
 
-def measure_hbm_ceiling(torch, sizes_mb=(8, 16, 32, 64, 76, 128, 256, 512, 1024, 2048), iters=20):
-    """Streaming throughput a plain read (torch's float32 sum) and a device-to-device copy reach
-    for transfers of a given size, rotating over enough buffers (>= 1 GiB together) that L2 never
-    holds the next one, replayed back to back from a CUDA graph.  GB/s counts the bytes read
-    (read) or read + written (copy)."""
+def measure_hbm_ceiling(torch, F, sizes_mb=(8, 16, 32, 64, 76, 128, 256, 512, 1024, 2048), iters=20):
+    """Streaming throughput of a plain read (the library's 16-byte-load probe kernel, best of 1,
+    2, 4 and 8 CTAs per SM) and of a device-to-device copy for transfers of a given size,
+    rotating over enough buffers (>= 1 GiB together) that L2 never holds the next one, replayed
+    back to back from a CUDA graph.  GB/s counts the bytes read (read) or read + written (copy)."""
     out = []
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
     for mb in sizes_mb:
         n = mb << 20
         k = max(4, -(-(1 << 30) // n))
         bufs = [torch.empty(n // 4, dtype=torch.float32, device="cuda").normal_() for _ in range(k)]
         dst = torch.empty(n // 4, dtype=torch.float32, device="cuda")
         row = {"mbytes": mb}
-        for kind in ("read", "copy"):
+        variants = [("read", c) for c in (1, 2, 4, 8)] + [("copy", 0)]
+        for kind, cps in variants:
             def op(i):
                 if kind == "read":
-                    return bufs[i % k].sum()
-                return dst.copy_(bufs[i % k])
-            # the timed reads are replayed from a CUDA graph, so host launch overhead is not counted
+                    F.ft_hbm_read_probe(bufs[i % k], n, sink, cps, torch.cuda.current_stream())
+                else:
+                    dst.copy_(bufs[i % k])
             side = torch.cuda.Stream()
             side.wait_stream(torch.cuda.current_stream())
             with torch.cuda.stream(side):
@@ -616,7 +629,13 @@ def measure_hbm_ceiling(torch, sizes_mb=(8, 16, 32, 64, 76, 128, 256, 512, 1024,
             us = e0.elapsed_time(e1) * 1e3 / iters
             del g
             moved = n if kind == "read" else 2 * n
-            row[kind] = {"us": us, "gbs": moved / (us * 1e-6) / 1e9}
+            res = {"us": us, "gbs": moved / (us * 1e-6) / 1e9}
+            if kind == "read":
+                res["ctas_per_sm"] = cps
+                if "read" not in row or res["gbs"] > row["read"]["gbs"]:
+                    row["read"] = res
+            else:
+                row["copy"] = res
         out.append(row)
         del bufs, dst
         torch.cuda.empty_cache()
@@ -625,7 +644,7 @@ def measure_hbm_ceiling(torch, sizes_mb=(8, 16, 32, 64, 76, 128, 256, 512, 1024,
 
 EXTRA_WORKLOADS = [("qwen3_a3b", [1, 4, 16]), ("gemma4_26b_a4b", [1]), ("tiny", [])]
 HEADLINE_DECODE = [1, 8]
-ROOFLINE_SUMMARY = ("moe_gemm_mxfp4_dsv4_flash_T8192.md", "gemm_mx_sm100.cu")
+ROOFLINE_SUMMARY = ("moe_gemm_mxfp4_dsv4_flash_T8192.md", ("gemm_mx_sm100.cu", "gemm_common.cuh", "sm100.cuh"))
 
 
 def main():
@@ -675,7 +694,7 @@ def main():
     if args.hbm_ceiling:
         if rank == 0:
             print(json.dumps({"mode": "hbm-ceiling", "peak_gbs": hbm_gbs, "peak_source": peak_src,
-                              "sizes": measure_hbm_ceiling(torch)}), flush=True)
+                              "sizes": measure_hbm_ceiling(torch, F)}), flush=True)
         return
 
     if args.decode_only:

@@ -151,12 +151,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const Tile& t
                 const int fl = lane & 15;
                 const bool lo = lane < 16;
 #pragma unroll
+                // token row t of the transpose buffer starts at xrow(t): rows 16..31 sit 32 bytes
+                // further on, so the two half-warps' 2-byte stores fall in different banks
+                auto xrow = [](int t) { return t * 16 + (t >= 16 ? 16 : 0); };
                 for (int i = 0; i < 16; ++i) {
                     const float send = lo ? v[u][16 + i] : v[u][i];
                     const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
                     const float gt = lo ? v[u][i] : recv;
                     const float up = lo ? recv : v[u][16 + i];
-                    xb[(lo ? i : 16 + i) * 16 + fl] = f2bf(silu_mul(gt, up));
+                    xb[xrow(lo ? i : 16 + i) + fl] = f2bf(silu_mul(gt, up));
                 }
                 __syncwarp();
                 const int fbase = rg * 64 + 16 * q;
@@ -166,7 +169,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const Tile& t
                     const int n = c * 32 + tok;
                     if (n < tl.nvalid)
                         *reinterpret_cast<uint4*>(p.out + size_t(tl.row0 + n) * p.out_ld + fbase + 8 * pp) =
-                            *reinterpret_cast<const uint4*>(xb + tok * 16 + 8 * pp);
+                            *reinterpret_cast<const uint4*>(xb + xrow(tok) + 8 * pp);
                 }
             } else {
 #pragma unroll

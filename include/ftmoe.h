@@ -378,6 +378,15 @@ ft_status ft_lru_step(int32_t E, int32_t n_slots, int32_t* content, int64_t* sta
 ft_status ft_lru_resize(int32_t E, int32_t n_old, int32_t n_new, int32_t* content, int64_t* stamp, int32_t* where,
                         int32_t* move_from, int32_t* move_to, int32_t* n_moves);
 
+/* Diagnostic: a plain streaming read of `bytes` (a multiple of 16) of device
+ * memory at `buf` (16-byte aligned) with 16-byte loads that bypass L1, four in
+ * flight per thread, ctas_per_sm (1..8) CTAs of 256 threads per SM; `sink` is
+ * one device word the kernel may write.  Enqueued on `stream`.  Time it with
+ * events to see the bandwidth a kernel that only reads reaches for a transfer
+ * of this size (decode layer calls move 50-650 MB, well below the sizes at
+ * which HBM reaches its copy peak). */
+ft_status ft_hbm_read_probe(const void* buf, size_t bytes, uint32_t* sink, int32_t ctas_per_sm, void* stream);
+
 /* Test hook for failure handling: make the n-th host->device expert copy
  * enqueue (counting from 1 after this call) report failure (n = 0 disables).
  * The failing decode step returns FT_ERR_CUDA and rolls the cache state of

@@ -226,3 +226,18 @@ def test_stream_calls_reject_a_null_handle_on_host():
         with pytest.raises(F.FtError) as ei:
             call()
         assert ei.value.status == F.FT_ERR_INVALID_ARG
+
+
+def test_pipeline_wait_limit_setter_round_trips():
+    prev = F.ft_set_pipeline_wait_limit_ns(12345)
+    assert prev == 4_000_000_000
+    assert F.ft_set_pipeline_wait_limit_ns(0) == 12345          # 0 restores the default
+    assert F.ft_set_pipeline_wait_limit_ns(prev) == 4_000_000_000
+
+
+def test_read_probe_rejects_bad_arguments_on_host():
+    for args in [(None, 1024, FAKE, 1), (FAKE + 4, 1024, FAKE, 1), (FAKE, 1000, FAKE, 1), (FAKE, 0, FAKE, 1),
+                 (FAKE, 1024, None, 1), (FAKE, 1024, FAKE, 0), (FAKE, 1024, FAKE, 9)]:
+        with pytest.raises(F.FtError) as ei:
+            F.ft_hbm_read_probe(*args, stream=0)
+        assert ei.value.status == F.FT_ERR_INVALID_ARG
