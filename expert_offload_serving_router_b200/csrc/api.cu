@@ -36,6 +36,9 @@ static int init_decode_max() {
 static int g_decode_max = init_decode_max();
 int decode_max() { return g_decode_max; }
 
+static bool g_block_scaled_decode = false;
+bool block_scaled_decode() { return g_block_scaled_decode; }
+
 static unsigned long long g_gemm_wait_ns = kWaitNs;
 unsigned long long gemm_wait_ns() { return g_gemm_wait_ns; }
 
@@ -124,6 +127,7 @@ DecodeArgs decode_args(const ft_moe_shape* s, int T, const ft_moe_weights* w, co
     a.o_sorted = static_cast<uint16_t*>(o_sorted);
     a.err = ws_at<uint32_t>(ws, L.err);
     a.o_ws = ws_at<uint16_t>(ws, L.o_sorted);
+    a.mx_ws = ws_at<uint8_t>(ws, L.mx_decode);
     return a;
 }
 
@@ -174,6 +178,12 @@ int32_t ft_set_decode_max_tokens(int32_t t) {
 }
 
 int32_t ft_get_decode_max_tokens(void) { return g_decode_max; }
+
+int32_t ft_set_block_scaled_decode(int32_t enable) {
+    const int32_t prev = g_block_scaled_decode ? 1 : 0;
+    g_block_scaled_decode = enable != 0;
+    return prev;
+}
 
 uint64_t ft_set_pipeline_wait_limit_ns(uint64_t ns) {
     const unsigned long long prev = g_gemm_wait_ns;

@@ -75,6 +75,7 @@ struct WsLayout {
     size_t x_sorted, h, o_sorted;
     size_t wr_planes;   // router weights as three bf16 planes (prefill-sized batches only)
     size_t route_part;  // partial logits of the prefill router, one slab per K split
+    size_t mx_decode;   // activation planes of the block-scaled MXFP4 decode (decode-sized batches)
     size_t total;
     int T, P, R, G, C;
 };
@@ -128,6 +129,10 @@ inline WsLayout make_layout(const ft_moe_shape& s, int T) {
     L.wr_planes = take(T > kSmallRoute ? size_t(3) * size_t((s.num_experts + 15) & ~15) * s.hidden * 2 : 0);
     L.route_part = take(T > kSmallRoute ? size_t(route_splits(T, s.hidden)) * ((T + kRouteTok - 1) / kRouteTok) *
                                               kRouteTok * ((s.num_experts + 15) & ~15) * sizeof(float) : 0);
+    // two E4M3 planes + E8M0 scales of x (32 rows) and of h (R rows): decode-sized MXFP4 batches
+    L.mx_decode = take(T <= kSmallRoute && s.wdtype == FT_W_MXFP4
+                           ? 2 * (32 * size_t(s.hidden) + size_t(s.hidden)) + 2 * (size_t(L.R) * s.ffn + size_t(L.R) * s.ffn / 32) + 2048
+                           : 0);
     L.total = o;
     return L;
 }

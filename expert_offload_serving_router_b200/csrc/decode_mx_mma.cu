@@ -1,0 +1,521 @@
+// Steps 3/4 (decode, MXFP4 weights) on the block-scaled tensor cores.
+//
+// The MXFP4 GEMVs are bound by decoding E2M1 codes on the ALUs.  Here the tensor core takes the
+// codes as they are: tcgen05.mma.kind::mxf8f6f4.block_scale multiplies E2M1 weights (A, with
+// their E8M0 scale per 32 elements) by E4M3 activations (B, with E8M0 scales).  A single E4M3
+// copy of the activations loses too much (the error study: 5.6e-2 of max|y| on the
+// DeepSeek-V4-Flash-shaped layer, over the 3e-2 tolerance), so each activation row is carried as
+// two planes -- hi = the OCP MX conversion of v, lo = the same conversion of v - hi, each with its
+// own E8M0 scale per 32 (1.2e-3 of max|y| in the study) -- and every K step issues one MMA per
+// plane into the same fp32 accumulator.
+//
+//   quant2_kernel:  bf16 rows -> E4M3 planes hi, lo [rows, K] + E8M0 scales [rows, K/32] each.
+//   decode_mx_mma_kernel<MODE>: items (active group, 128 weight rows), persistent CTAs, as the
+//       BF16 tensor-core decode; per 128-deep K step TMA brings 128 rows of codes unpacked to one
+//       byte per element (16U4_ALIGN16B, SW128) and the two activation planes; per item the
+//       epilogue warps lay the weight and activation scales out as tcgen05.cp source atoms (one
+//       per K step and operand, 32 rows x 16 bytes: byte 16 (m % 32) + 4 (m / 32) + j holds row
+//       m's scale of the j-th 32-block of the step) and at the item's start the MMA thread copies
+//       every atom into its own four TMEM columns (lane = row % 32 in every sub-partition, column =
+//       row / 32, byte = block), so no MMA waits on a copy mid-stream.
+// Weights and activation planes are read once; every wait is bounded.
+#include "gemm_common.cuh"
+#include "decode_common.cuh"
+
+namespace ftmoe {
+
+// ------------------------------------------------------------------ activation planes
+// One thread per (row, 32-element block): X1 = 2^(floor(log2 amax) - 8), hi = E4M3(v / X1)
+// (round to nearest even, saturating at 448), r = v - X1 * hi (exact), X2 from max|r|, lo =
+// E4M3(r / X2).  A block of zeros keeps the scale 2^0.  Rows >= rows_valid are written as zero.
+__device__ __forceinline__ uint32_t e8m0_of(float amax, float& X) {
+    if (!(amax > 0.f)) { X = 1.f; return 127u; }
+    int e = ilogbf(amax) - 8;
+    e = max(-127, min(127, e));
+    X = ldexpf(1.f, e);
+    return uint32_t(e + 127);
+}
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+    uint16_t lo, hi;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(lo) : "f"(a), "f"(b));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(hi) : "f"(c), "f"(d));
+    return uint32_t(lo) | (uint32_t(hi) << 16);
+}
+__device__ __forceinline__ void e4m3x4_dec(uint32_t q, float (&o)[4]) {
+    uint32_t h0, h1;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h0) : "h"(uint16_t(q & 0xFFFF)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(uint16_t(q >> 16)));
+    const __half2 a = *reinterpret_cast<const __half2*>(&h0), b = *reinterpret_cast<const __half2*>(&h1);
+    o[0] = __low2float(a); o[1] = __high2float(a); o[2] = __low2float(b); o[3] = __high2float(b);
+}
+
+__global__ void __launch_bounds__(256) quant2_kernel(const uint16_t* __restrict__ src, int rows_valid, int rows, int K,
+                                                     uint8_t* hi, uint8_t* lo, uint8_t* shi, uint8_t* slo) {
+    pdl_wait();
+    pdl_trigger();
+    const int nb = K / 32;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= rows * nb) return;
+    const int r = i / nb, b = i - r * nb;
+    float v[32];
+    if (r < rows_valid) {
+        const uint4* s = reinterpret_cast<const uint4*>(src + size_t(r) * K + 32 * b);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 u = __ldcg(s + q);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) { v[8 * q + 2 * j] = bf16lo(w[j]); v[8 * q + 2 * j + 1] = bf16hi(w[j]); }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    float X1, X2;
+    const uint32_t s1 = e8m0_of(amax, X1);
+    const float inv1 = 1.f / X1;                         // exact: a power of two
+    uint32_t qh[8];
+    float res[32];
+    float amax2 = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        qh[q] = e4m3x4(v[4 * q] * inv1, v[4 * q + 1] * inv1, v[4 * q + 2] * inv1, v[4 * q + 3] * inv1);
+        float d[4];
+        e4m3x4_dec(qh[q], d);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            res[4 * q + j] = v[4 * q + j] - d[j] * X1;   // exact: v has 8 significant bits
+            amax2 = fmaxf(amax2, fabsf(res[4 * q + j]));
+        }
+    }
+    const uint32_t s2 = e8m0_of(amax2, X2);
+    const float inv2 = 1.f / X2;
+    uint32_t ql[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+        ql[q] = e4m3x4(res[4 * q] * inv2, res[4 * q + 1] * inv2, res[4 * q + 2] * inv2, res[4 * q + 3] * inv2);
+    uint4* dh = reinterpret_cast<uint4*>(hi + size_t(r) * K + 32 * b);
+    uint4* dl = reinterpret_cast<uint4*>(lo + size_t(r) * K + 32 * b);
+    dh[0] = make_uint4(qh[0], qh[1], qh[2], qh[3]);
+    dh[1] = make_uint4(qh[4], qh[5], qh[6], qh[7]);
+    dl[0] = make_uint4(ql[0], ql[1], ql[2], ql[3]);
+    dl[1] = make_uint4(ql[4], ql[5], ql[6], ql[7]);
+    shi[size_t(r) * nb + b] = uint8_t(s1);
+    slo[size_t(r) * nb + b] = uint8_t(s2);
+}
+
+
+__device__ __forceinline__ int group_token_of(int flat, int P, int k) { return flat < P ? flat / k : flat - P; }
+
+// ------------------------------------------------------------------ block-scaled MMA
+constexpr int kDxSt = 7;                          // stages of one 128-deep K step
+constexpr int kDxATile = 128 * 128;               // 16 KB: 128 rows x 128 codes, one byte each
+constexpr int kDxBPlane = 32 * 128;               // 4 KB: up to 32 activation rows, one plane
+constexpr int kDxThreads = 192;
+constexpr int kDxMaxK = 4096;                     // largest contraction (scale atoms sized for it)
+constexpr int kDxSteps = kDxMaxK / 128;           // K steps per item at most
+constexpr int kDxAtomBuf = 3 * kDxSteps * 512;    // one item's weight, hi and lo scale atoms of every K step
+constexpr int kDxTmemCols = 512;                  // 2 x 32 accumulators + every step's three scale atoms
+constexpr int kDxColSf = 64;                      // kind k (weights, hi, lo), step c: columns 64 + 128 k + 4 c
+
+__host__ __device__ constexpr size_t dec_mx_smem() {
+    return 1024 + size_t(kDxSt) * (kDxATile + 2 * kDxBPlane) + size_t(kDxAtomBuf) + 512;
+}
+
+struct DecMxParams {
+    int T, k, E, H, F, G, NB, m_blocks, K;
+    const int32_t* offsets;
+    const int32_t* sorted_flat;
+    const int32_t* sched;
+    const int32_t* inv_pos;
+    const float* topk_w;
+    const uint8_t* wsc;               // weight scales [E, rows, K/32]
+    const uint8_t* bsc_hi;            // activation scales [rows, K/32], one per plane
+    const uint8_t* bsc_lo;
+    uint16_t* h;
+    uint16_t* o;
+    uint16_t* y;
+    uint32_t* ticket;
+    uint32_t* err;
+    unsigned long long wait_ns;
+};
+
+// kind::mxf8f6f4 block-scaled instruction descriptor: A E2M1, B E4M3, both K-major, E8M0
+// scales, M = 128; sf ids select the scale byte of the K block
+__device__ __forceinline__ uint32_t idesc_mx(int N, uint32_t sfa_id, uint32_t sfb_id) {
+    return (sfb_id << 4) | (5u << 7) | (0u << 10) | (uint32_t(N >> 3) << 17) | (1u << 23) | (uint32_t(128 >> 4) << 24) |
+           (sfa_id << 29);
+}
+__device__ __forceinline__ void umma_mx(uint32_t dtm, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t tsfa,
+                                        uint32_t tsfb, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(dtm), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(tsfa), "r"(tsfb));
+}
+// 32 rows x 16 bytes of shared memory (contiguous, no swizzle) -> TMEM lanes 0..31 of four
+// columns, repeated in every lane quarter
+__device__ __forceinline__ void tmem_cp_atom(uint32_t taddr, uint32_t saddr) {
+    uint64_t d = uint64_t((saddr >> 4) & 0x3FFFu);
+    d |= uint64_t(128 >> 4) << 16;      // leading byte offset
+    d |= uint64_t(128 >> 4) << 32;      // stride byte offset: next 8 rows
+    d |= uint64_t(1) << 46;
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kDxThreads, 1)
+decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_bh,
+                     const __grid_constant__ CUtensorMap tm_bl, DecMxParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + kDxSt * kDxATile;                       // [stage][plane] 4 KB each
+    uint8_t* sAtoms = sB + kDxSt * 2 * kDxBPlane;             // [kind][K step] 512-byte atoms of one item
+    uint64_t* full = reinterpret_cast<uint64_t*>(sAtoms + kDxAtomBuf);
+    uint64_t* empty = full + kDxSt;
+    uint64_t* tfull = empty + kDxSt;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* sf_full = tempty + 2;       // atoms of an item laid out
+    uint64_t* sf_free = sf_full + 1;      // atoms of an item copied to TMEM
+    uint64_t* mma_done = sf_free + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    pdl_wait();          // routing, the activation planes and h come from the preceding kernels
+    pdl_trigger();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_items = p.sched[1] * p.m_blocks;
+    if (int(blockIdx.x) >= n_items) return;
+    const int nk = p.K / 128;
+    if (tid == 0) {
+        for (int s = 0; s < kDxSt; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4); }
+        mbar_init(sf_full, 4);
+        mbar_init(sf_free, 1);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                     "r"(kDxTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int P = p.T * p.k;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer: codes + both activation planes
+        if (lane == 0) {
+            // the transaction count of the unpacking code copy is its packed size (4 bits per
+            // code), half of the 16 KB it fills in shared memory
+            const uint32_t bytes = uint32_t(kDxATile) / 2u + 2u * uint32_t(p.NB) * 128u;
+            int step = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+                const int slot = it / p.m_blocks, rg = it - slot * p.m_blocks;
+                const int g = p.sched[2 + (p.G + 1) + slot];
+                const int brow = MODE == 0 ? 0 : p.offsets[g];
+                for (int kb = 0; kb < nk; ++kb, ++step) {
+                    const int s = step % kDxSt;
+                    if (!mbar_wait(&empty[s], (uint32_t(step / kDxSt) & 1u) ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                    mbar_expect_tx(&full[s], bytes);
+                    if (MODE == 0) tma_5d(&tm_w, &full[s], sA + s * kDxATile, kb * 128, 0, 0, rg * 4, g);
+                    else tma_3d(&tm_w, &full[s], sA + s * kDxATile, kb * 128, rg * 128, g);
+                    tma_2d(&tm_bh, &full[s], sB + (2 * s) * kDxBPlane, kb * 128, brow);
+                    tma_2d(&tm_bl, &full[s], sB + (2 * s + 1) * kDxBPlane, kb * 128, brow);
+                }
+            }
+            if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+            for (int st = step - kDxSt > 0 ? step - kDxSt : 0; st < step; ++st)
+                mbar_wait(&full[st % kDxSt], uint32_t(st / kDxSt) & 1u, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer: an item's scales to TMEM, then two planes per K block
+        if (lane == 0) {
+            int step = 0, buf = 0, item = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++item) {
+                const uint8_t* atoms = sAtoms;
+                if (!mbar_wait(sf_full, uint32_t(item) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                if (!mbar_wait(&tempty[buf], acc_phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                tc_fence_after();
+                // every step's scales to their own TMEM columns first, so the MMAs below never wait
+                // on a copy (they execute after the copies: same issuing thread, issue order)
+                for (int kind = 0; kind < 3; ++kind)
+                    for (int c = 0; c < nk; ++c)
+                        tmem_cp_atom(tmem + uint32_t(kDxColSf + 128 * kind + 4 * c), su32(atoms + (kind * kDxSteps + c) * 512));
+                umma_commit(sf_free);          // the atoms may be rebuilt for the next item once copied
+                for (int kb = 0; kb < nk; ++kb, ++step) {
+                    const int s = step % kDxSt;
+                    if (!mbar_wait(&full[s], uint32_t(step / kDxSt) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t ad = sdesc_sw128(su32(sA + s * kDxATile));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {                 // 32-deep K blocks of this step
+                        const uint32_t tsfa = tmem + uint32_t(kDxColSf + 4 * kb) + (uint32_t(j) << 30);
+#pragma unroll
+                        for (int pl = 0; pl < 2; ++pl) {
+                            const uint64_t bd = sdesc_sw128(su32(sB + (2 * s + pl) * kDxBPlane));
+                            const uint32_t tsfb = tmem + uint32_t(kDxColSf + 128 * (1 + pl) + 4 * kb) + (uint32_t(j) << 30);
+                            umma_mx(tmem + uint32_t(32 * buf), ad + uint64_t(j * 2), bd + uint64_t(j * 2),
+                                    idesc_mx(p.NB, uint32_t(j), uint32_t(j)), tsfa, tsfb, (kb | j | pl) != 0);
+                        }
+                    }
+                    umma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&tfull[buf]);
+                if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+            }
+            if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+            umma_commit(mma_done);
+            mbar_wait(mma_done, 0, nullptr);
+        }
+    } else {
+        // ------------------------------------------------ scale atoms, then the epilogue
+        // Item i+1's atoms are laid out once item i's reached TMEM (the MMA thread copies them at
+        // the item's start), before item i's epilogue, so they are ready when item i ends.  Atom
+        // of K step c: byte 16 (m % 32) + 4 (m / 32) + j = scale of 32-block j of row m (weights:
+        // the A-tile row; activations: B row m < 32, the rest of the atom unused).
+        const int q = warp & 3, et = tid - 64;   // et: 0..127
+        const int nsb = p.K / 32;                // scale bytes per row
+        const size_t rows_e = MODE == 0 ? size_t(2) * p.F : size_t(p.H);
+        auto build_atoms = [&](int it2) {
+            uint8_t* atoms = sAtoms;
+            const int slot2 = it2 / p.m_blocks, rg2 = it2 - slot2 * p.m_blocks;
+            const int g2 = p.sched[2 + (p.G + 1) + slot2];
+            const int r02 = p.offsets[g2], n2 = p.offsets[g2 + 1] - r02;
+            int wrow;     // weight row of A-tile row et (gate/up: blocks of 16 gate rows then the 16 up rows)
+            if (MODE == 0) {
+                const int i = et >> 5, jj = et & 31, f = rg2 * 64 + 16 * i + (jj & 15);
+                wrow = jj < 16 ? f : p.F + f;
+            } else {
+                wrow = rg2 * 128 + et;
+            }
+            // a row's scales arrive as 16-byte vectors (four K steps each), all loads in flight
+            const uint4* ws = reinterpret_cast<const uint4*>(p.wsc + (size_t(g2) * rows_e + wrow) * nsb);
+            const int nv = nk / 4;
+            uint4 wv[kDxSteps / 4];
+#pragma unroll
+            for (int c4 = 0; c4 < kDxSteps / 4; ++c4)
+                if (c4 < nv) wv[c4] = __ldg(ws + c4);
+#pragma unroll
+            for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
+                if (c4 >= nv) break;
+                const uint32_t w4[4] = {wv[c4].x, wv[c4].y, wv[c4].z, wv[c4].w};
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+                    *reinterpret_cast<uint32_t*>(atoms + (4 * c4 + cc) * 512 + 16 * (et & 31) + 4 * (et >> 5)) = w4[cc];
+            }
+            if (et < 64) {
+                const int pl = et >> 5, nrow = et & 31;
+                const uint8_t* bsrc = pl ? p.bsc_lo : p.bsc_hi;
+                const int brow = MODE == 0 ? nrow : r02 + nrow;
+                const bool valid = MODE == 0 ? nrow < p.T : nrow < n2;
+                const uint4* bs = reinterpret_cast<const uint4*>(bsrc + size_t(brow) * nsb);
+#pragma unroll
+                for (int c4 = 0; c4 < kDxSteps / 4; ++c4)
+                    if (c4 < nv) wv[c4] = valid ? __ldcg(bs + c4) : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+#pragma unroll
+                for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
+                    if (c4 >= nv) break;
+                    const uint32_t b4[4] = {wv[c4].x, wv[c4].y, wv[c4].z, wv[c4].w};
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+                        *reinterpret_cast<uint32_t*>(atoms + ((1 + pl) * kDxSteps + 4 * c4 + cc) * 512 + 16 * nrow) = b4[cc];
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sf_full);
+        };
+        int buf = 0, item = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        build_atoms(blockIdx.x);
+        for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++item) {
+            const int slot = it / p.m_blocks, rg = it - slot * p.m_blocks;
+            const int g = p.sched[2 + (p.G + 1) + slot];
+            const int r0 = p.offsets[g], n = p.offsets[g + 1] - r0;
+            if (it + int(gridDim.x) < n_items) {
+                // the buffer is free once this item's atoms reached TMEM (at the item's start)
+                if (!mbar_wait(sf_free, uint32_t(item) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                build_atoms(it + gridDim.x);
+            }
+            // lane l < n stands for row r0 + l of the group; gate/up: its token
+            const int my_tok = (MODE == 0 && lane < n) ? group_token_of(p.sorted_flat[r0 + lane], P, p.k) : -1;
+            if (!mbar_wait(&tfull[buf], acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
+            tc_fence_after();
+            float v[32];
+            tmem_ld32_nowait(tmem + (uint32_t(q * 32) << 16) + uint32_t(32 * buf), v);
+            tmem_wait_16(v);
+            tmem_fence_regs(v + 16);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[buf]);
+            if (MODE == 0) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    if (c >= p.NB) break;
+                    const unsigned hit = __ballot_sync(0xffffffffu, my_tok == c);
+                    if (!hit) continue;
+                    const int r = r0 + __ffs(hit) - 1;
+                    const float other = __shfl_xor_sync(0xffffffffu, v[c], 16);
+                    const float hv = silu_mul(lane < 16 ? v[c] : other, lane < 16 ? other : v[c]);
+                    const uint32_t b = f2bf(hv);
+                    const uint32_t pair = b | (__shfl_down_sync(0xffffffffu, b, 1) << 16);
+                    if (lane < 16 && !(lane & 1))
+                        *reinterpret_cast<uint32_t*>(p.h + size_t(r) * p.F + 64 * rg + 16 * q + lane) = pair;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i < n) p.o[size_t(r0 + i) * p.H + 128 * rg + 32 * q + lane] = f2bf(v[i]);
+                if (p.y) {
+                    __threadfence();
+                    unsigned last = 0;
+                    if (lane == 0) last = atomicAdd(&p.ticket[4 * rg + q], 1u) == uint32_t(p.sched[1] - 1);
+                    last = __shfl_sync(0xffffffffu, last, 0);
+                    if (last) {
+                        __threadfence();
+                        const int hr = 128 * rg + 32 * q + lane;
+                        for (int t = 0; t < p.T; ++t) {
+                            float acc = 0.f;
+                            for (int j = 0; j < p.k; ++j)
+                                acc = fmaf(p.topk_w[t * p.k + j],
+                                           bf16f(__ldcg(p.o + size_t(p.inv_pos[t * p.k + j]) * p.H + hr)), acc);
+                            p.y[size_t(t) * p.H + hr] = f2bf(acc);
+                        }
+                        if (lane == 0) p.ticket[4 * rg + q] = 0;
+                    }
+                }
+            }
+            if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+        }
+        if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kDxTmemCols));
+    }
+}
+
+
+// ------------------------------------------------------------------ host side
+bool decode_mx_eligible(const DecodeArgs& a) {
+    return a.wdtype == FT_W_MXFP4 && !a.eptr && !a.S && a.T >= 1 && a.T <= 32 && a.H % 512 == 0 && a.F % 512 == 0 &&
+           a.H <= kDxMaxK && a.F <= kDxMaxK;
+}
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_dep(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+static bool plane_map(CUtensorMap* m, const void* base, int K, int rows, int NB) {
+    uint64_t d[2] = {uint64_t(K), uint64_t(rows)}, s[1] = {uint64_t(K)};
+    uint32_t b[2] = {128, uint32_t(NB)};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 2, d, s, b);
+}
+
+cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
+    const int T = a.T, H = a.H, F = a.F, E = a.E, k = a.k;
+    const int R = T * k, G = E;
+    const int na_max = R < G ? R : G;
+    const int NB = T <= 16 ? 16 : 32;
+    // scratch: x planes [32, H] x 2 + scales, h planes [R, F] x 2 + scales (256-byte aligned parts)
+    uint8_t* q = a.mx_ws;
+    auto take = [&](size_t bytes) { uint8_t* r = q; q += (bytes + 255) & ~size_t(255); return r; };
+    uint8_t* xh = take(32 * size_t(H));
+    uint8_t* xl = take(32 * size_t(H));
+    uint8_t* xsh = take(32 * size_t(H) / 32);
+    uint8_t* xsl = take(32 * size_t(H) / 32);
+    uint8_t* hh = take(size_t(R) * F);
+    uint8_t* hl = take(size_t(R) * F);
+    uint8_t* hsh = take(size_t(R) * F / 32);
+    uint8_t* hsl = take(size_t(R) * F / 32);
+
+    DecMxParams p{};
+    p.T = T; p.k = k; p.E = E; p.H = H; p.F = F; p.G = G; p.NB = NB;
+    p.offsets = a.offsets;
+    p.sorted_flat = a.sorted_flat;
+    p.sched = a.sched;
+    p.inv_pos = a.inv_pos;
+    p.topk_w = a.topk_w;
+    p.h = a.h;
+    p.o = a.y ? a.o_ws : a.o_sorted;
+    p.y = a.y;
+    p.ticket = a.err + kWsDownTicket;
+    p.err = a.err;
+    p.wait_ns = gemm_wait_ns();
+
+    CUtensorMap gw{}, dw{}, gbh{}, gbl{}, dbh{}, dbl{};
+    {   // codes unpacked to a byte per element by TMA; gate/up as (H, 16, 2, F/16, E) blocks of 16 gate + 16 up rows
+        uint64_t dims[5] = {uint64_t(H), 16, 2, uint64_t(F / 16), uint64_t(E)};
+        uint64_t str[4] = {uint64_t(H) / 2, uint64_t(F) * H / 2, uint64_t(16) * H / 2, uint64_t(2) * F * H / 2};
+        uint32_t box[5] = {128, 16, 2, 4, 1};
+        if (!make_map(&gw, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, a.w13, 5, dims, str, box)) return cudaErrorInvalidValue;
+        uint64_t d3[3] = {uint64_t(F), uint64_t(H), uint64_t(E)};
+        uint64_t s3[2] = {uint64_t(F) / 2, uint64_t(H) * F / 2};
+        uint32_t b3[3] = {128, 128, 1};
+        if (!make_map(&dw, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, a.w2, 3, d3, s3, b3)) return cudaErrorInvalidValue;
+    }
+    if (!plane_map(&gbh, xh, H, 32, NB) || !plane_map(&gbl, xl, H, 32, NB) || !plane_map(&dbh, hh, F, R, NB) ||
+        !plane_map(&dbl, hl, F, R, NB))
+        return cudaErrorInvalidValue;
+    constexpr size_t smem = dec_mx_smem();
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(decode_mx_mma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(decode_mx_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const int cap = num_sms();            // persistent: one CTA per SM (ring and scale atoms fill shared memory)
+    cudaError_t e = launch_dep(quant2_kernel, (32 * (H / 32) + 255) / 256, 256, 0, st, a.x, T, 32, H, xh, xl, xsh, xsl);
+    if (e != cudaSuccess) return e;
+    p.K = H;
+    p.m_blocks = F / 64;
+    p.wsc = a.w13s;
+    p.bsc_hi = xsh;
+    p.bsc_lo = xsl;
+    e = launch_dep(decode_mx_mma_kernel<0>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, kDxThreads, smem, st,
+                   gw, gbh, gbl, p);
+    if (e != cudaSuccess) return e;
+    e = launch_dep(quant2_kernel, (R * (F / 32) + 255) / 256, 256, 0, st, static_cast<const uint16_t*>(a.h), R, R, F, hh,
+                   hl, hsh, hsl);
+    if (e != cudaSuccess) return e;
+    p.K = F;
+    p.m_blocks = H / 128;
+    p.wsc = a.w2s;
+    p.bsc_hi = hsh;
+    p.bsc_lo = hsl;
+    e = launch_dep(decode_mx_mma_kernel<1>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, kDxThreads, smem, st,
+                   dw, dbh, dbl, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace ftmoe

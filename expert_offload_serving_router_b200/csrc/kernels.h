@@ -39,6 +39,7 @@ struct DecodeArgs {
     uint16_t* o_sorted;         // [R, H] when y == NULL
     uint32_t* err;              // workspace device error flag
     uint16_t* o_ws;             // workspace [R, H] rows for the tensor-core decode's combine
+    uint8_t* mx_ws;             // workspace scratch of the block-scaled MXFP4 decode (activation planes)
 };
 
 struct GemmLaunch {
@@ -88,6 +89,10 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 // tensor-core decode (BF16, contiguous weights): false when the shape or weights do not qualify
 bool decode_mma_eligible(const DecodeArgs& a);
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st);
+// block-scaled MXFP4 decode on the tensor cores (decode_mx_mma.cu)
+bool decode_mx_eligible(const DecodeArgs& a);
+cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st);
+bool block_scaled_decode();   // api.cu: ft_set_block_scaled_decode
 int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st);
 // bound (ns without progress) on each pipeline wait of the grouped GEMMs (api.cu)
 unsigned long long gemm_wait_ns();

@@ -58,6 +58,7 @@ _SIGS = {
     "ft_set_decode_max_tokens": (c_i32, [c_i32]),
     "ft_get_decode_max_tokens": (c_i32, []),
     "ft_set_pipeline_wait_limit_ns": (c_u64, [c_u64]),
+    "ft_set_block_scaled_decode": (c_i32, [c_i32]),
     "ft_hbm_read_probe": (c_i32, [c_vp, c_sz, c_vp, c_i32, c_vp]),
     "ft_moe_workspace_bytes": (c_sz, [ctypes.POINTER(ft_moe_shape), c_i32]),
     "ft_moe_workspace_init": (c_i32, [c_vp, c_sz, c_vp]),
@@ -174,6 +175,10 @@ def ft_get_decode_max_tokens() -> int:
 
 def ft_set_pipeline_wait_limit_ns(ns: int) -> int:
     return lib().ft_set_pipeline_wait_limit_ns(ns)
+
+
+def ft_set_block_scaled_decode(enable: int) -> int:
+    return lib().ft_set_block_scaled_decode(enable)
 
 
 def ft_hbm_read_probe(buf, nbytes: int, sink, ctas_per_sm: int, stream=None) -> None:

@@ -241,3 +241,11 @@ def test_read_probe_rejects_bad_arguments_on_host():
         with pytest.raises(F.FtError) as ei:
             F.ft_hbm_read_probe(*args, stream=0)
         assert ei.value.status == F.FT_ERR_INVALID_ARG
+
+
+def test_block_scaled_decode_switch_returns_previous_setting():
+    from expert_offload_serving_router_b200 import ftmoe as F
+    assert F.ft_set_block_scaled_decode(1) == 0
+    assert F.ft_set_block_scaled_decode(7) == 1
+    assert F.ft_set_block_scaled_decode(0) == 1
+    assert F.ft_set_block_scaled_decode(0) == 0

@@ -220,3 +220,50 @@ def test_chained_layers_without_host_sync(name, T):
     F.ft_moe_check(ws)
     for s in range(steps):
         assert np.array_equal(host(bufs[s + 1], np.uint16), ref[s]), f"step {s} differs"
+
+
+@pytest.fixture
+def block_scaled_decode():
+    prev = F.ft_set_block_scaled_decode(1)
+    try:
+        yield
+    finally:
+        assert F.ft_set_block_scaled_decode(prev) == 1
+
+
+@pytest.mark.parametrize("name,T,kw", [("dsv4_flash", 1, {}), ("dsv4_flash", 8, {}), ("dsv4_flash", 20, {}),
+                                       ("dsv4_flash", 32, {}),
+                                       ("custom", 13, dict(hidden=1024, ffn=512, num_experts=16, top_k=4,
+                                                           num_shared=0, wdtype=inputs.WDTYPE_MXFP4, config_id=83))])
+def test_block_scaled_mxfp4_decode_matches_oracle(block_scaled_decode, name, T, kw):
+    """MXFP4 decode on tcgen05.mma.kind::mxf8f6f4.block_scale (E2M1 weights with their E8M0
+    scales read as stored, activations as two E4M3 planes): every token checked against the
+    fp64 oracle within the MXFP4 tolerance, routing bit-exact."""
+    L = layer(name, **kw)
+    x = inputs.make_tokens(L.cfg, T, seed=5)
+    _, _, _, rel = full_check(L, x, n_rows=T)
+    assert rel < 1e-2, f"two-plane activations should stay well inside the MXFP4 bound, got {rel:.2e}"
+
+
+def test_block_scaled_decode_chained_is_deterministic(block_scaled_decode):
+    """Back-to-back block-scaled decode calls (ticketed combine, dependent launches) equal the
+    same chain run one call at a time."""
+    import torch
+    from gpu_util import dev, host, run_layer, workspace
+    L = layer("dsv4_flash")
+    T, H, k = 8, L.cfg.hidden, L.cfg.top_k
+    x0 = inputs.make_tokens(L.cfg, T, seed=12)
+    ref, x = [], x0
+    for _ in range(4):
+        y, _, _ = run_layer(L, x)
+        ref.append(y)
+        x = y
+    ws = workspace(L.shape, T)
+    bufs = [dev(x0)] + [torch.empty((T, H), dtype=torch.int16, device="cuda") for _ in range(4)]
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    for s in range(4):
+        F.ft_moe_layer_forward(L.shape, T, bufs[s], L.t["w_router"], L.t.get("bias"), L.weights, bufs[s + 1], idx,
+                               None, ws)
+    F.ft_moe_check(ws)
+    for s in range(4):
+        assert np.array_equal(host(bufs[s + 1], np.uint16), ref[s]), f"step {s} differs"
