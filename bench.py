@@ -316,13 +316,12 @@ def measure_prefill(torch, F, L, T, steps, warmup, stream, rank, clock_index=Non
                 clocks=clocks, ctx=dict(x=x, ws=ws, ws_bytes=ws_bytes, y=y))
 
 
-def measure_decode(torch, F, L, tokens, rank, hbm_gbs):
-    """Decode batches through the whole-layer call, rotating over 4 weight copies so no
+def measure_decode(torch, F, L, tokens, rank, hbm_gbs, nrot=4):
+    """Decode batches through the whole-layer call, rotating over nrot weight copies so no
     batch finds its experts in L2.  Timed as plain launches and as a replayed CUDA graph
-    of 4 calls (one per weight copy)."""
+    of nrot calls (one per weight copy)."""
     cfg = L.cfg
     H, E, k = cfg.hidden, cfg.num_experts, cfg.top_k
-    nrot = 4
     rot, keep = [L.weights], []
     for _ in range(1, nrot):
         wstruct, t = L.copy_weights(F)
@@ -665,6 +664,10 @@ def main():
                     help="time only prefill steps of this layer shape at its prefill size (for profiling)")
     ap.add_argument("--prefill-tokens", type=int, default=None,
                     help="with --prefill-only: the batch size (default: the shape's prefill size)")
+    ap.add_argument("--decode-rotations", type=int, default=4,
+                    help="with --decode-only: weight copies rotated between calls (1 for small ncu captures)")
+    ap.add_argument("--block-scaled-decode", action="store_true",
+                    help="run MXFP4 decode batches on the block-scaled tensor-core path")
     ap.add_argument("--hbm-ceiling", action="store_true",
                     help="only time plain streaming reads and copies of decode-sized transfers")
     args = ap.parse_args()
@@ -697,10 +700,14 @@ def main():
                               "sizes": measure_hbm_ceiling(torch, F)}), flush=True)
         return
 
+    if args.block_scaled_decode:
+        F.ft_set_block_scaled_decode(1)
+
     if args.decode_only:
         cfg = inputs.CONFIGS[args.decode_only]
         L = Layer(torch, F, cfg, inputs.make_layer(cfg, seed=0))
-        dec = measure_decode(torch, F, L, dec_tokens or list(cfg.decode_tokens), rank, hbm_gbs)
+        dec = measure_decode(torch, F, L, dec_tokens or list(cfg.decode_tokens), rank, hbm_gbs,
+                             nrot=args.decode_rotations)
         if rank == 0:
             print(json.dumps({"mode": "decode-only", "workload": f"{cfg.name} decode", "decode": dec}), flush=True)
         return

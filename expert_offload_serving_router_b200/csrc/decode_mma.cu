@@ -43,7 +43,7 @@ struct DecMmaParams {
 };
 
 __host__ __device__ constexpr size_t dec_mma_smem() {
-    return 1024 + size_t(kDmSt) * (kDmATile + kDmBTile) + 512;
+    return 1024 + size_t(kDmSt) * (kDmATile + kDmBTile) + 512 + kCombineTableBytes;
 }
 
 // token of the group's i-th row
@@ -84,6 +84,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
     uint64_t* mma_done = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_pos = reinterpret_cast<int*>(sB + kDmSt * kDmBTile + 512);
+    float* s_w = reinterpret_cast<float*>(s_pos + kCombinePosMax);
 
     pdl_wait();          // routing (offsets, schedule) and h come from the preceding kernels
     pdl_trigger();
@@ -102,6 +104,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)), "r"(64));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
+    if (MODE == 1 && p.y) load_combine_tables(p.inv_pos, p.topk_w, p.T, p.k, p.S, s_pos, s_w, tid, kDmThreads);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -207,15 +210,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
                     last = __shfl_sync(0xffffffffu, last, 0);
                     if (last) {
                         __threadfence();
-                        const int P = p.T * p.k, hr = 128 * d.rg + 32 * q + lane;
-                        for (int t = 0; t < p.T; ++t) {
-                            float acc = 0.f;
-                            for (int j = 0; j < p.k; ++j)
-                                acc = fmaf(p.topk_w[t * p.k + j],
-                                           bf16f(__ldcg(p.o + size_t(p.inv_pos[t * p.k + j]) * p.H + hr)), acc);
-                            if (p.S) acc += bf16f(__ldcg(p.o + size_t(p.inv_pos[P + t]) * p.H + hr));
-                            p.y[size_t(t) * p.H + hr] = f2bf(acc);
-                        }
+                        const int hr = 128 * d.rg + 32 * q + lane;
+                        combine_serial(p, p.S, s_pos, s_w, hr);
                         if (lane == 0) p.ticket[4 * d.rg + q] = 0;     // left at zero for the next call
                     }
                 }

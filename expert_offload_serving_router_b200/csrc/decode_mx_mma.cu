@@ -122,7 +122,7 @@ constexpr int kDxTmemCols = 512;                  // 2 x 32 accumulators + every
 constexpr int kDxColSf = 64;                      // kind k (weights, hi, lo), step c: columns 64 + 128 k + 4 c
 
 __host__ __device__ constexpr size_t dec_mx_smem() {
-    return 1024 + size_t(kDxSt) * (kDxATile + 2 * kDxBPlane) + size_t(kDxAtomBuf) + 512;
+    return 1024 + size_t(kDxSt) * (kDxATile + 2 * kDxBPlane) + size_t(kDxAtomBuf) + 512 + kCombineTableBytes;
 }
 
 struct DecMxParams {
@@ -184,6 +184,8 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
     uint64_t* mma_done = sf_free + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_pos = reinterpret_cast<int*>(sAtoms + kDxAtomBuf + 512);
+    float* s_w = reinterpret_cast<float*>(s_pos + kCombinePosMax);
 
     pdl_wait();          // routing, the activation planes and h come from the preceding kernels
     pdl_trigger();
@@ -205,6 +207,7 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                      "r"(kDxTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
+    if (MODE == 1 && p.y) load_combine_tables(p.inv_pos, p.topk_w, p.T, p.k, 0, s_pos, s_w, tid, kDxThreads);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -388,13 +391,7 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                     if (last) {
                         __threadfence();
                         const int hr = 128 * rg + 32 * q + lane;
-                        for (int t = 0; t < p.T; ++t) {
-                            float acc = 0.f;
-                            for (int j = 0; j < p.k; ++j)
-                                acc = fmaf(p.topk_w[t * p.k + j],
-                                           bf16f(__ldcg(p.o + size_t(p.inv_pos[t * p.k + j]) * p.H + hr)), acc);
-                            p.y[size_t(t) * p.H + hr] = f2bf(acc);
-                        }
+                        combine_serial(p, 0, s_pos, s_w, hr);
                         if (lane == 0) p.ticket[4 * rg + q] = 0;
                     }
                 }

@@ -150,10 +150,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const Tile& t
             if (p.mode == 0) {
                 const int fl = lane & 15;
                 const bool lo = lane < 16;
-#pragma unroll
                 // token row t of the transpose buffer starts at xrow(t): rows 16..31 sit 32 bytes
                 // further on, so the two half-warps' 2-byte stores fall in different banks
                 auto xrow = [](int t) { return t * 16 + (t >= 16 ? 16 : 0); };
+#pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float send = lo ? v[u][16 + i] : v[u][i];
                     const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
