@@ -9,12 +9,16 @@
 
 namespace ftmoe {
 
+// DEP: launched as a programmatic dependent of the expert kernel that writes o (decode
+// batches): the routing (inv_pos, gates; final before that kernel started) is read before
+// the wait, o after it, and the next kernel may be scheduled at once.
+template <bool DEP>
 __global__ void __launch_bounds__(256) combine_kernel(int T, int H, int k, int S, int R, const uint16_t* __restrict__ o,
                                                       const int32_t* __restrict__ inv_pos, const float* __restrict__ gw,
                                                       uint16_t* __restrict__ y) {
+    if (DEP) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int t = blockIdx.y;
     const int c = blockIdx.x * 256 + threadIdx.x;     // 16-byte column vector index
-    if (c * 8 >= H) return;
     const int P = T * k;
     int pos[kMaxTopK + 1];
     float wgt[kMaxTopK + 1];
@@ -24,6 +28,8 @@ __global__ void __launch_bounds__(256) combine_kernel(int T, int H, int k, int S
         if (j < k) { pos[nterm] = inv_pos[t * k + j]; wgt[nterm] = gw[t * k + j]; ++nterm; }
     }
     if (S) { pos[nterm] = inv_pos[P + t]; wgt[nterm] = 1.0f; ++nterm; }
+    if (DEP) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (c * 8 >= H) return;
     uint4 v[kMaxTopK + 1];
 #pragma unroll
     for (int j = 0; j < kMaxTopK + 1; ++j) {
@@ -54,8 +60,23 @@ cudaError_t launch_combine(int T, int H, int k, int S, int R, const uint16_t* o,
                            const float* gw, uint16_t* y, cudaStream_t st) {
     if (T <= 0) return cudaSuccess;
     dim3 grid((H / 8 + 255) / 256, T);
-    combine_kernel<<<grid, 256, 0, st>>>(T, H, k, S, R, o, inv_pos, gw, y);
+    combine_kernel<false><<<grid, 256, 0, st>>>(T, H, k, S, R, o, inv_pos, gw, y);
     return cudaGetLastError();
+}
+
+cudaError_t launch_combine_dependent(int T, int H, int k, int S, int R, const uint16_t* o, const int32_t* inv_pos,
+                                     const float* gw, uint16_t* y, cudaStream_t st) {
+    if (T <= 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((H / 8 + 255) / 256, T);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, combine_kernel<true>, T, H, k, S, R, o, inv_pos, gw, y);
 }
 
 __global__ void __launch_bounds__(256) unit_rms_kernel(int H, const uint16_t* in, uint16_t* out, float eps) {

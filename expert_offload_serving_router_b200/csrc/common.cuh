@@ -83,10 +83,8 @@ struct WsLayout {
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace header (cleared by ft_moe_workspace_init): word 0 device error flag, word 1 the
-// decode router's ticket, words kWsDownTicket.. one ticket per 32 hidden rows for the
-// tensor-core decode's combine (every launch leaves the tickets at zero).
+// decode router's ticket (left at zero by every launch); the rest is reserved.
 constexpr size_t kWsHeaderBytes = 4096;
-constexpr int kWsDownTicket = 64;      // word index; 16384 / 32 = 512 tickets fit
 constexpr int kRouteTok = 128;          // tokens per router CTA
 constexpr int kRouteTargetCtas = 148;   // split K until the router grid covers about one wave
 constexpr int kRouteMaxSplit = 8;

@@ -313,30 +313,4 @@ __device__ __forceinline__ void down_item4(const DecodeArgs& a, const uint8_t* c
     }
 }
 
-// ------------------------------------------------ ticketed combine of the tensor-core decode kernels
-// inv_pos [T*k + S*T] and topk_w [T*k] of the batch, staged in shared memory at kernel start
-constexpr int kCombinePosMax = 32 * (kMaxTopK + 1);
-constexpr int kCombineWMax = 32 * kMaxTopK;
-constexpr size_t kCombineTableBytes = 4 * size_t(kCombinePosMax + kCombineWMax);
-
-__device__ __forceinline__ void load_combine_tables(const int32_t* inv_pos, const float* topk_w, int T, int k, int S,
-                                                    int* s_pos, float* s_w, int tid, int nthreads) {
-    const int P = T * k;
-    for (int i = tid; i < P + (S ? T : 0); i += nthreads) s_pos[i] = inv_pos[i];
-    for (int i = tid; i < P; i += nthreads) s_w[i] = topk_w[i];
-}
-
-// y[t, hr] = sum_j g[t,j] o[pos(t,j), hr] (+ shared) in fp32, j order, one hidden row, token by
-// token (batching the row loads of several tokens measured slower)
-template <class Prm>
-__device__ __forceinline__ void combine_serial(const Prm& p, int S, const int* s_pos, const float* s_w, int hr) {
-    for (int t = 0; t < p.T; ++t) {
-        float acc = 0.f;
-        for (int j = 0; j < p.k; ++j)
-            acc = fmaf(s_w[t * p.k + j], bf16f(__ldcg(p.o + size_t(s_pos[t * p.k + j]) * p.H + hr)), acc);
-        if (S) acc += bf16f(__ldcg(p.o + size_t(s_pos[p.T * p.k + t]) * p.H + hr));
-        p.y[size_t(t) * p.H + hr] = f2bf(acc);
-    }
-}
-
 }  // namespace ftmoe

@@ -10,9 +10,9 @@
 //       gather of x, no x_sorted.
 //   down (MODE 1):    items (active group, 128 hidden rows).  B = the group's
 //       contiguous h rows [offsets[g], offsets[g+1]) (rows past the group belong to other
-//       groups and are ignored), o_sorted[row, hidden] -> bf16.  The last warp to finish a
-//       32-row slice of hidden rows (atomic ticket, no waiting) combines y[t] = sum_j g[t,j]
-//       o[pos(t,j)] (+ shared) in fp32, j order, for that slice: deterministic.
+//       groups and are ignored), o[row, hidden] -> bf16.  The gate-weighted combine back to
+//       token order follows as its own small kernel (programmatic dependent launch), so no
+//       CTA here waits on, or sums for, the others.
 // Persistent CTAs (two per SM) walk the items with one TMA ring; accumulators are double
 // buffered.  Warp roles: 0 TMA producer, 1 TMEM allocation + MMA issuer, 2-5 epilogue (TMEM
 // lane quarter warp & 3).  Every wait is bounded (the grouped GEMMs' limit).
@@ -32,18 +32,14 @@ struct DecMmaParams {
     const int32_t* offsets;
     const int32_t* sorted_flat;
     const int32_t* sched;              // [1] n_active, active groups at [2 + G + 1 ...]
-    const int32_t* inv_pos;
-    const float* topk_w;
     uint16_t* h;                       // [R, F]
     uint16_t* o;                       // [R, H]
-    uint16_t* y;                       // [T, H]
-    uint32_t* ticket;                  // [H/32] (one per 32 hidden rows), zero between calls
     uint32_t* err;
     unsigned long long wait_ns;
 };
 
 __host__ __device__ constexpr size_t dec_mma_smem() {
-    return 1024 + size_t(kDmSt) * (kDmATile + kDmBTile) + 512 + kCombineTableBytes;
+    return 1024 + size_t(kDmSt) * (kDmATile + kDmBTile) + 512;
 }
 
 // token of the group's i-th row
@@ -84,8 +80,6 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
     uint64_t* mma_done = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* s_pos = reinterpret_cast<int*>(sB + kDmSt * kDmBTile + 512);
-    float* s_w = reinterpret_cast<float*>(s_pos + kCombinePosMax);
 
     pdl_wait();          // routing (offsets, schedule) and h come from the preceding kernels
     pdl_trigger();
@@ -104,7 +98,6 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)), "r"(64));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    if (MODE == 1 && p.y) load_combine_tables(p.inv_pos, p.topk_w, p.T, p.k, p.S, s_pos, s_w, tid, kDmThreads);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -200,21 +193,6 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     if (i < d.n) p.o[size_t(d.r0 + i) * p.H + 128 * d.rg + 32 * q + lane] = f2bf(v[i]);
-                if (p.y) {
-                    // the last warp to finish these 32 hidden rows (one per item of the block:
-                    // atomic ticket, no waiting) combines y[t, rows] = sum_j g[t,j] o[pos(t,j), rows]
-                    // (+ shared) in j order, lane = hidden row
-                    __threadfence();
-                    unsigned last = 0;
-                    if (lane == 0) last = atomicAdd(&p.ticket[4 * d.rg + q], 1u) == uint32_t(p.sched[1] - 1);
-                    last = __shfl_sync(0xffffffffu, last, 0);
-                    if (last) {
-                        __threadfence();
-                        const int hr = 128 * d.rg + 32 * q + lane;
-                        combine_serial(p, p.S, s_pos, s_w, hr);
-                        if (lane == 0) p.ticket[4 * d.rg + q] = 0;     // left at zero for the next call
-                    }
-                }
             }
             if (++buf == 2) { buf = 0; acc_phase ^= 1; }
         }
@@ -258,12 +236,8 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st) {
     p.offsets = a.offsets;
     p.sorted_flat = a.sorted_flat;
     p.sched = a.sched;
-    p.inv_pos = a.inv_pos;
-    p.topk_w = a.topk_w;
     p.h = a.h;
     p.o = a.y ? a.o_ws : a.o_sorted;
-    p.y = a.y;
-    p.ticket = a.err + kWsDownTicket;
     p.err = a.err;
     p.wait_ns = gemm_wait_ns();
     CUtensorMap gw{}, gsw{}, gb{}, dw{}, dsw{}, db{};
@@ -308,6 +282,8 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st) {
     p.m_blocks = H / 128;
     e = launch_dependent(decode_mma_kernel<1>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, smem, st, dw,
                          dsw, db, p);
+    if (e != cudaSuccess) return e;
+    if (a.y) e = launch_combine_dependent(T, H, k, S, R, a.o_ws, a.inv_pos, a.topk_w, a.y, st);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -122,7 +122,7 @@ constexpr int kDxTmemCols = 512;                  // 2 x 32 accumulators + every
 constexpr int kDxColSf = 64;                      // kind k (weights, hi, lo), step c: columns 64 + 128 k + 4 c
 
 __host__ __device__ constexpr size_t dec_mx_smem() {
-    return 1024 + size_t(kDxSt) * (kDxATile + 2 * kDxBPlane) + size_t(kDxAtomBuf) + 512 + kCombineTableBytes;
+    return 1024 + size_t(kDxSt) * (kDxATile + 2 * kDxBPlane) + size_t(kDxAtomBuf) + 512;
 }
 
 struct DecMxParams {
@@ -130,15 +130,11 @@ struct DecMxParams {
     const int32_t* offsets;
     const int32_t* sorted_flat;
     const int32_t* sched;
-    const int32_t* inv_pos;
-    const float* topk_w;
     const uint8_t* wsc;               // weight scales [E, rows, K/32]
     const uint8_t* bsc_hi;            // activation scales [rows, K/32], one per plane
     const uint8_t* bsc_lo;
     uint16_t* h;
     uint16_t* o;
-    uint16_t* y;
-    uint32_t* ticket;
     uint32_t* err;
     unsigned long long wait_ns;
 };
@@ -184,8 +180,6 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
     uint64_t* mma_done = sf_free + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* s_pos = reinterpret_cast<int*>(sAtoms + kDxAtomBuf + 512);
-    float* s_w = reinterpret_cast<float*>(s_pos + kCombinePosMax);
 
     pdl_wait();          // routing, the activation planes and h come from the preceding kernels
     pdl_trigger();
@@ -207,7 +201,6 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                      "r"(kDxTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    if (MODE == 1 && p.y) load_combine_tables(p.inv_pos, p.topk_w, p.T, p.k, 0, s_pos, s_w, tid, kDxThreads);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -383,18 +376,6 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     if (i < n) p.o[size_t(r0 + i) * p.H + 128 * rg + 32 * q + lane] = f2bf(v[i]);
-                if (p.y) {
-                    __threadfence();
-                    unsigned last = 0;
-                    if (lane == 0) last = atomicAdd(&p.ticket[4 * rg + q], 1u) == uint32_t(p.sched[1] - 1);
-                    last = __shfl_sync(0xffffffffu, last, 0);
-                    if (last) {
-                        __threadfence();
-                        const int hr = 128 * rg + 32 * q + lane;
-                        combine_serial(p, 0, s_pos, s_w, hr);
-                        if (lane == 0) p.ticket[4 * rg + q] = 0;
-                    }
-                }
             }
             if (++buf == 2) { buf = 0; acc_phase ^= 1; }
         }
@@ -458,12 +439,8 @@ cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
     p.offsets = a.offsets;
     p.sorted_flat = a.sorted_flat;
     p.sched = a.sched;
-    p.inv_pos = a.inv_pos;
-    p.topk_w = a.topk_w;
     p.h = a.h;
     p.o = a.y ? a.o_ws : a.o_sorted;
-    p.y = a.y;
-    p.ticket = a.err + kWsDownTicket;
     p.err = a.err;
     p.wait_ns = gemm_wait_ns();
 
@@ -511,6 +488,8 @@ cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
     p.bsc_lo = hsl;
     e = launch_dep(decode_mx_mma_kernel<1>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, kDxThreads, smem, st,
                    dw, dbh, dbl, p);
+    if (e != cudaSuccess) return e;
+    if (a.y) e = launch_combine_dependent(T, H, k, 0, R, a.o_ws, a.inv_pos, a.topk_w, a.y, st);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -98,6 +98,8 @@ int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st);
 unsigned long long gemm_wait_ns();
 cudaError_t launch_combine(int T, int H, int k, int S, int R, const uint16_t* o, const int32_t* inv_pos,
                            const float* gw, uint16_t* y, cudaStream_t st);
+cudaError_t launch_combine_dependent(int T, int H, int k, int S, int R, const uint16_t* o, const int32_t* inv_pos,
+                           const float* gw, uint16_t* y, cudaStream_t st);   // PDL-launched after a decode expert kernel
 cudaError_t launch_unit_rms(int T, int H, const uint16_t* in, uint16_t* out, float eps, cudaStream_t st);
 
 }  // namespace ftmoe

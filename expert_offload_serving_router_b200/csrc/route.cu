@@ -95,16 +95,11 @@ __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteArgs a) {
     __syncthreads();
     if (!last) return;
     __threadfence();
-    // ---- last CTA: top-k for every token (+ permutation)
-    __shared__ float lrow[8][kMaxExperts];
+    // ---- last CTA: top-k for every token (+ permutation), a warp per token
     __shared__ int32_t sidx[kSmallRoute * kMaxTopK];
-    for (int t = warp; t < a.T; t += 8) {
-        for (int i = lane; i < a.E; i += 32) lrow[warp][i] = __ldcg(a.logits + size_t(t) * a.E + i);
-        __syncwarp();
-        warp_topk_row(lrow[warp], a.E, a.k, a.topk_idx + size_t(t) * a.k, a.topk_w + size_t(t) * a.k,
+    for (int t = warp; t < a.T; t += 8)
+        warp_topk_row(a.logits + size_t(t) * a.E, a.E, a.k, a.topk_idx + size_t(t) * a.k, a.topk_w + size_t(t) * a.k,
                       sidx + t * a.k);
-        __syncwarp();
-    }
     if (tid == 0) *a.ticket = 0u;
     __syncthreads();
     if (!a.do_permute) return;

@@ -2,10 +2,10 @@
 // experts ordered by logit descending, the lower index first on equal logits; gates =
 // softmax over the kept logits (fp32, summed in slot order).
 //
-// A Top8 list is kept sorted in registers.  Offering a candidate costs a fixed, branch-free
-// sequence (8 compares, 16 selects per array) so a warp of tokens never diverges on it; a
-// warp can also merge its 32 lists (one per lane) with a bitonic butterfly when one token's
-// experts are spread over the lanes.
+// The prefill router keeps a Top8 list sorted in registers per thread: offering a candidate
+// costs a fixed, branch-free sequence (8 compares, 16 selects per array) so a warp of tokens
+// never diverges on it, and a group of lanes merges its lists with a bitonic butterfly.  The
+// decode router's last CTA gives each token a warp and selects by warp reductions instead.
 #pragma once
 #include "common.cuh"
 
@@ -109,15 +109,42 @@ __device__ __forceinline__ void top_slot(const Top8& t, int k, int j, int32_t* e
     *w_out = expf(key_logit(kk) - l0) / den;
 }
 
-// Warp-wide top-k over the E logits of one token in `row` (shared memory): lane l offers
-// experts l, l+32, ... in order, then the lists are merged; lanes 0..k-1 write slot = lane.
+// Warp-wide top-k over the E <= 256 logits of one token, read from global memory `row` (L2:
+// another CTA wrote them) straight into registers.  Lane l holds the keys of experts l, l+32, ...; each of the k rounds takes the warp's largest key
+// (one max-reduction) and, among the lanes holding it, the lowest expert (one min-reduction),
+// then the owning lane drops it.  Same order as Top8 (logit desc, index asc; key 0 never
+// chosen) and the same gates; lanes 0..k-1 write slot = lane.
 __device__ inline void warp_topk_row(const float* row, int E, int k, int32_t* idx_out, float* w_out,
                                      int32_t* idx_smem) {
+    constexpr int kPer = kMaxExperts / 32;
     const int lane = threadIdx.x & 31;
+    uint32_t key[kPer];
+#pragma unroll
+    for (int s = 0; s < kPer; ++s) {
+        const int e = lane + 32 * s;
+        key[s] = e < E ? logit_key(__ldcg(row + e)) : 0u;
+    }
     Top8 t;
     t.init();
-    for (int e = lane; e < E; e += 32) t.offer(logit_key(row[e]), e);
-    group_merge_top8(t, 32);
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+        if (j >= k) break;
+        uint32_t bk = 0u, be = 0xffffffffu;        // this lane's best: experts ascend with s
+#pragma unroll
+        for (int s = 0; s < kPer; ++s) {
+            const bool better = key[s] > bk;
+            bk = better ? key[s] : bk;
+            be = better ? uint32_t(lane + 32 * s) : be;
+        }
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+        if (mk == 0u) break;                       // only key-0 experts left: slots stay (0, 0)
+        const uint32_t me = __reduce_min_sync(0xffffffffu, bk == mk ? be : 0xffffffffu);
+#pragma unroll
+        for (int s = 0; s < kPer; ++s)
+            if (uint32_t(lane + 32 * s) == me) key[s] = 0u;
+        t.key[j] = mk;
+        t.idx[j] = int32_t(me);
+    }
     if (lane < k) {
         int32_t ee;
         float ww;
