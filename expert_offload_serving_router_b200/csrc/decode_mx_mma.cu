@@ -110,19 +110,33 @@ __global__ void __launch_bounds__(256) quant2_kernel(const uint16_t* __restrict_
 
 __device__ __forceinline__ int group_token_of(int flat, int P, int k) { return flat < P ? flat / k : flat - P; }
 
+// Bring `bytes` (multiple of 16, 16-byte aligned) into L2 ahead of the TMA ring, 16 KB per request.
+__device__ __forceinline__ void l2_prefetch(const uint8_t* ptr, uint32_t bytes) {
+    for (uint32_t o = 0; o < bytes; o += 16384u) {
+        const uint32_t n = bytes - o < 16384u ? bytes - o : 16384u;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr + o), "r"(n) : "memory");
+    }
+}
+
 // ------------------------------------------------------------------ block-scaled MMA
-constexpr int kDxSt = 7;                          // stages of one 128-deep K step
-constexpr int kDxATile = 128 * 128;               // 16 KB: 128 rows x 128 codes, one byte each
-constexpr int kDxBPlane = 32 * 128;               // 4 KB: up to 32 activation rows, one plane
+// A stage is a 256-deep K step made of two 128-deep sub-tiles: one barrier wait and one commit per
+// eight MMAs (an mbarrier poll costs the issuing thread about as much as two small MMAs).
+constexpr int kDxSt = 4;                          // stages
+constexpr int kDxATile = 128 * 128;               // 16 KB: 128 rows x 128 codes, one byte each (one sub-tile)
+constexpr int kDxBPlane = 32 * 128;               // 4 KB: up to 32 activation rows of one plane and sub-tile
+constexpr int kDxAStage = 2 * kDxATile;           // 32 KB
+constexpr int kDxBSub = 2 * kDxBPlane;            // 8 KB: a sub-tile's B operand, hi rows then lo rows
+constexpr int kDxBStage = 2 * kDxBSub;            // 16 KB
 constexpr int kDxThreads = 192;
 constexpr int kDxMaxK = 4096;                     // largest contraction (scale atoms sized for it)
 constexpr int kDxSteps = kDxMaxK / 128;           // K steps per item at most
-constexpr int kDxAtomBuf = 3 * kDxSteps * 512;    // one item's weight, hi and lo scale atoms of every K step
-constexpr int kDxTmemCols = 512;                  // 2 x 32 accumulators + every step's three scale atoms
-constexpr int kDxColSf = 64;                      // kind k (weights, hi, lo), step c: columns 64 + 128 k + 4 c
+constexpr int kDxAtomBuf = 2 * kDxSteps * 512;    // one item's weight and activation scale atoms of every K step
+constexpr int kDxTmemCols = 512;                  // 2 x 64 accumulator columns + every step's two scale atoms
+constexpr int kDxAccCols = 64;                    // accumulator columns per buffer: N = 2 NB (hi rows, then lo rows)
+constexpr int kDxColSf = 128;                     // kind k (weights, activations), step c: columns 128 + 128 k + 4 c
 
 __host__ __device__ constexpr size_t dec_mx_smem() {
-    return 1024 + size_t(kDxSt) * (kDxATile + 2 * kDxBPlane) + size_t(kDxAtomBuf) + 512;
+    return 1024 + size_t(kDxSt) * (kDxAStage + kDxBStage) + size_t(kDxAtomBuf) + 512;
 }
 
 struct DecMxParams {
@@ -131,6 +145,7 @@ struct DecMxParams {
     const int32_t* sorted_flat;
     const int32_t* sched;
     const uint8_t* wsc;               // weight scales [E, rows, K/32]
+    const uint8_t* wcodes;            // packed codes: w13 [E][2F][H/2] (gate rows, then up rows) or w2 [E][H][F/2]
     const uint8_t* bsc_hi;            // activation scales [rows, K/32], one per plane
     const uint8_t* bsc_lo;
     uint16_t* h;
@@ -153,13 +168,22 @@ __device__ __forceinline__ void umma_mx(uint32_t dtm, uint64_t ad, uint64_t bd, 
         ::"r"(dtm), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(tsfa), "r"(tsfb));
 }
 // 32 rows x 16 bytes of shared memory (contiguous, no swizzle) -> TMEM lanes 0..31 of four
-// columns, repeated in every lane quarter
-__device__ __forceinline__ void tmem_cp_atom(uint32_t taddr, uint32_t saddr) {
+// columns, repeated in every lane quarter.  atom_desc gives the source descriptor of the atom at
+// saddr; the atom 512 bytes on is that descriptor + 32.
+__device__ __forceinline__ uint64_t atom_desc(uint32_t saddr) {
     uint64_t d = uint64_t((saddr >> 4) & 0x3FFFu);
     d |= uint64_t(128 >> 4) << 16;      // leading byte offset
     d |= uint64_t(128 >> 4) << 32;      // stride byte offset: next 8 rows
     d |= uint64_t(1) << 46;
+    return d;
+}
+__device__ __forceinline__ void tmem_cp_desc(uint32_t taddr, uint64_t d) {
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+}
+// the bounded wait, entered only when the phase is not already complete (the common case at
+// steady state costs one try_wait)
+__device__ __forceinline__ bool wait_fast(uint64_t* b, uint32_t parity, volatile int* abort, unsigned long long limit) {
+    return mbar_try(b, parity) || mbar_wait(b, parity, abort, limit);
 }
 
 template <int MODE>
@@ -169,8 +193,8 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = sA + kDxSt * kDxATile;                       // [stage][plane] 4 KB each
-    uint8_t* sAtoms = sB + kDxSt * 2 * kDxBPlane;             // [kind][K step] 512-byte atoms of one item
+    uint8_t* sB = sA + kDxSt * kDxAStage;                      // [stage][sub-tile] hi rows 0..NB-1, lo rows NB..2NB-1
+    uint8_t* sAtoms = sB + kDxSt * kDxBStage;                 // [kind][128-deep K step] 512-byte atoms of one item
     uint64_t* full = reinterpret_cast<uint64_t*>(sAtoms + kDxAtomBuf);
     uint64_t* empty = full + kDxSt;
     uint64_t* tfull = empty + kDxSt;
@@ -181,12 +205,33 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+    // an item's packed codes: gate/up 64 gate rows + the same 64 up rows; down 128 rows (contiguous)
+    auto prefetch_item = [&](int it) {
+        const int slot = it / p.m_blocks, rg = it - slot * p.m_blocks;
+        const int g = __ldcg(p.sched + 2 + (p.G + 1) + slot);
+        if (slot >= p.G || g < 0 || g >= p.E) return;       // only a hint: never an address outside w
+        if (MODE == 0) {
+            const size_t rb = size_t(p.H) / 2, base = size_t(g) * 2 * p.F * rb;
+            l2_prefetch(p.wcodes + base + size_t(64 * rg) * rb, uint32_t(64 * rb));
+            l2_prefetch(p.wcodes + base + size_t(p.F + 64 * rg) * rb, uint32_t(64 * rb));
+        } else {
+            const size_t rb = size_t(p.F) / 2;
+            l2_prefetch(p.wcodes + (size_t(g) * p.H + 128 * rg) * rb, uint32_t(128 * rb));
+        }
+    };
+    // The routing (schedule, offsets) was final before this grid could launch: the kernel ahead
+    // of it started its own dependents only after waiting for the kernels that wrote it.  So the
+    // first item's weights can stream into L2 while this grid waits for the activations.
+    if (threadIdx.x == 0) {
+        const int n0 = __ldcg(p.sched + 1) * p.m_blocks;
+        if (int(blockIdx.x) < n0) prefetch_item(blockIdx.x);
+    }
     pdl_wait();          // routing, the activation planes and h come from the preceding kernels
     pdl_trigger();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_items = p.sched[1] * p.m_blocks;
     if (int(blockIdx.x) >= n_items) return;
-    const int nk = p.K / 128;
+    const int nk = p.K / 128;                // 128-deep K steps (scale atoms); stages cover two
     if (tid == 0) {
         for (int s = 0; s < kDxSt; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4); }
@@ -212,21 +257,31 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
         if (lane == 0) {
             // the transaction count of the unpacking code copy is its packed size (4 bits per
             // code), half of the 16 KB it fills in shared memory
-            const uint32_t bytes = uint32_t(kDxATile) / 2u + 2u * uint32_t(p.NB) * 128u;
-            int step = 0;
+            const uint32_t bytes = 2u * (uint32_t(kDxATile) / 2u + 2u * uint32_t(p.NB) * 128u);
+            int step = 0, s = 0;
+            uint32_t phase = 0;
             bool ok = true;
             for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 const int slot = it / p.m_blocks, rg = it - slot * p.m_blocks;
                 const int g = p.sched[2 + (p.G + 1) + slot];
                 const int brow = MODE == 0 ? 0 : p.offsets[g];
-                for (int kb = 0; kb < nk; ++kb, ++step) {
-                    const int s = step % kDxSt;
-                    if (!mbar_wait(&empty[s], (uint32_t(step / kDxSt) & 1u) ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                if (it + int(gridDim.x) < n_items) prefetch_item(it + gridDim.x);   // the next item's weights
+                for (int kb = 0; kb < nk / 2; ++kb, ++step) {
+                    if (!wait_fast(&empty[s], phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
                     mbar_expect_tx(&full[s], bytes);
-                    if (MODE == 0) tma_5d(&tm_w, &full[s], sA + s * kDxATile, kb * 128, 0, 0, rg * 4, g);
-                    else tma_3d(&tm_w, &full[s], sA + s * kDxATile, kb * 128, rg * 128, g);
-                    tma_2d(&tm_bh, &full[s], sB + (2 * s) * kDxBPlane, kb * 128, brow);
-                    tma_2d(&tm_bl, &full[s], sB + (2 * s + 1) * kDxBPlane, kb * 128, brow);
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int k0 = (2 * kb + u) * 128;
+                        uint8_t* a = sA + s * kDxAStage + u * kDxATile;
+                        if (MODE == 0) tma_5d(&tm_w, &full[s], a, k0, 0, 0, rg * 4, g);
+                        else tma_3d(&tm_w, &full[s], a, k0, rg * 128, g);
+                        // one B operand of 2 NB rows: the lo plane's rows follow the hi plane's (NB x
+                        // 128 bytes later: a whole number of 1 KB swizzle atoms)
+                        uint8_t* b = sB + s * kDxBStage + u * kDxBSub;
+                        tma_2d(&tm_bh, &full[s], b, k0, brow);
+                        tma_2d(&tm_bl, &full[s], b + p.NB * 128, k0, brow);
+                    }
+                    if (++s == kDxSt) { s = 0; phase ^= 1u; }
                 }
             }
             if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
@@ -234,39 +289,49 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                 mbar_wait(&full[st % kDxSt], uint32_t(st / kDxSt) & 1u, nullptr);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer: an item's scales to TMEM, then two planes per K block
+        // ------------------------------------------------ MMA issuer: an item's scales to TMEM, then one MMA per K block
+        // At decode sizes this thread is the critical path (an MMA with N <= 64 occupies the tensor
+        // pipe for only ~56 cycles), so every operand but the stage is computed once per launch
+        // and the descriptors advance by adding (start address >> 4) offsets.
         if (lane == 0) {
-            int step = 0, buf = 0, item = 0;
-            uint32_t acc_phase = 0;
+            uint32_t idm[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) idm[j] = idesc_mx(2 * p.NB, uint32_t(j), uint32_t(j));
+            const uint64_t ad0 = sdesc_sw128(su32(sA)), bd0 = sdesc_sw128(su32(sB)), cp0 = atom_desc(su32(sAtoms));
+            int stage = 0, buf = 0, item = 0;
+            uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++item) {
-                const uint8_t* atoms = sAtoms;
-                if (!mbar_wait(sf_full, uint32_t(item) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
-                if (!mbar_wait(&tempty[buf], acc_phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                if (!wait_fast(sf_full, uint32_t(item) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                if (!wait_fast(&tempty[buf], acc_phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
                 tc_fence_after();
                 // every step's scales to their own TMEM columns first, so the MMAs below never wait
                 // on a copy (they execute after the copies: same issuing thread, issue order)
-                for (int kind = 0; kind < 3; ++kind)
-                    for (int c = 0; c < nk; ++c)
-                        tmem_cp_atom(tmem + uint32_t(kDxColSf + 128 * kind + 4 * c), su32(atoms + (kind * kDxSteps + c) * 512));
+                for (int c = 0; c < nk; ++c) {
+                    tmem_cp_desc(tmem + uint32_t(kDxColSf + 4 * c), cp0 + uint64_t(32 * c));
+                    tmem_cp_desc(tmem + uint32_t(kDxColSf + 128 + 4 * c), cp0 + uint64_t(32 * (kDxSteps + c)));
+                }
                 umma_commit(sf_free);          // the atoms may be rebuilt for the next item once copied
-                for (int kb = 0; kb < nk; ++kb, ++step) {
-                    const int s = step % kDxSt;
-                    if (!mbar_wait(&full[s], uint32_t(step / kDxSt) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint64_t ad = sdesc_sw128(su32(sA + s * kDxATile));
+                const uint32_t dacc = tmem + uint32_t(kDxAccCols * buf);
+                uint32_t sfa = tmem + uint32_t(kDxColSf), sfb = tmem + uint32_t(kDxColSf + 128);
+                for (int kb = 0; kb < nk / 2; ++kb) {
+                    // the stage's operands were all written by TMA (async proxy): its barrier's
+                    // completion orders them before these MMAs, no thread-sync fence needed
+                    if (!wait_fast(&full[stage], phase, abort_flag, p.wait_ns)) { ok = false; break; }
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {                 // 32-deep K blocks of this step
-                        const uint32_t tsfa = tmem + uint32_t(kDxColSf + 4 * kb) + (uint32_t(j) << 30);
-#pragma unroll
-                        for (int pl = 0; pl < 2; ++pl) {
-                            const uint64_t bd = sdesc_sw128(su32(sB + (2 * s + pl) * kDxBPlane));
-                            const uint32_t tsfb = tmem + uint32_t(kDxColSf + 128 * (1 + pl) + 4 * kb) + (uint32_t(j) << 30);
-                            umma_mx(tmem + uint32_t(32 * buf), ad + uint64_t(j * 2), bd + uint64_t(j * 2),
-                                    idesc_mx(p.NB, uint32_t(j), uint32_t(j)), tsfa, tsfb, (kb | j | pl) != 0);
-                        }
+                    for (int u = 0; u < 2; ++u) {
+                        const uint64_t ad = ad0 + uint64_t((stage * kDxAStage + u * kDxATile) >> 4);
+                        const uint64_t bd = bd0 + uint64_t((stage * kDxBStage + u * kDxBSub) >> 4);
+                        // the four 32-deep K blocks of the sub-tile (scale byte j of each row's step word)
+                        umma_mx(dacc, ad, bd, idm[0], sfa, sfb, (kb | u) != 0);
+                        umma_mx(dacc, ad + 2, bd + 2, idm[1], sfa + (1u << 30), sfb + (1u << 30), 1u);
+                        umma_mx(dacc, ad + 4, bd + 4, idm[2], sfa + (2u << 30), sfb + (2u << 30), 1u);
+                        umma_mx(dacc, ad + 6, bd + 6, idm[3], sfa + (3u << 30), sfb + (3u << 30), 1u);
+                        sfa += 4u;
+                        sfb += 4u;
                     }
-                    umma_commit(&empty[s]);
+                    umma_commit(&empty[stage]);
+                    if (++stage == kDxSt) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 umma_commit(&tfull[buf]);
@@ -281,7 +346,7 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
         // Item i+1's atoms are laid out once item i's reached TMEM (the MMA thread copies them at
         // the item's start), before item i's epilogue, so they are ready when item i ends.  Atom
         // of K step c: byte 16 (m % 32) + 4 (m / 32) + j = scale of 32-block j of row m (weights:
-        // the A-tile row; activations: B row m < 32, the rest of the atom unused).
+        // the A-tile row; activations: B row m < 2 NB -- the hi plane's rows, then the lo plane's).
         const int q = warp & 3, et = tid - 64;   // et: 0..127
         const int nsb = p.K / 32;                // scale bytes per row
         const size_t rows_e = MODE == 0 ? size_t(2) * p.F : size_t(p.H);
@@ -297,13 +362,13 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
             } else {
                 wrow = rg2 * 128 + et;
             }
-            // a row's scales arrive as 16-byte vectors (four K steps each), all loads in flight
+            // a row's scales arrive as 16-byte vectors (four K steps each), all loads in flight:
+            // issued unconditionally (vectors past the row's last re-read it) so none waits on a branch
             const uint4* ws = reinterpret_cast<const uint4*>(p.wsc + (size_t(g2) * rows_e + wrow) * nsb);
             const int nv = nk / 4;
             uint4 wv[kDxSteps / 4];
 #pragma unroll
-            for (int c4 = 0; c4 < kDxSteps / 4; ++c4)
-                if (c4 < nv) wv[c4] = __ldg(ws + c4);
+            for (int c4 = 0; c4 < kDxSteps / 4; ++c4) wv[c4] = __ldg(ws + min(c4, nv - 1));
 #pragma unroll
             for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
                 if (c4 >= nv) break;
@@ -312,22 +377,23 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                 for (int cc = 0; cc < 4; ++cc)
                     *reinterpret_cast<uint32_t*>(atoms + (4 * c4 + cc) * 512 + 16 * (et & 31) + 4 * (et >> 5)) = w4[cc];
             }
-            if (et < 64) {
-                const int pl = et >> 5, nrow = et & 31;
+            if (et < 64 && (et & 31) < p.NB) {
+                const int pl = et >> 5, nrow = et & 31, m = pl * p.NB + nrow;   // B row of the merged operand
                 const uint8_t* bsrc = pl ? p.bsc_lo : p.bsc_hi;
                 const int brow = MODE == 0 ? nrow : r02 + nrow;
                 const bool valid = MODE == 0 ? nrow < p.T : nrow < n2;
-                const uint4* bs = reinterpret_cast<const uint4*>(bsrc + size_t(brow) * nsb);
+                const uint4* bs = reinterpret_cast<const uint4*>(bsrc + size_t(valid ? brow : 0) * nsb);
 #pragma unroll
-                for (int c4 = 0; c4 < kDxSteps / 4; ++c4)
-                    if (c4 < nv) wv[c4] = valid ? __ldcg(bs + c4) : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+                for (int c4 = 0; c4 < kDxSteps / 4; ++c4) wv[c4] = __ldcg(bs + min(c4, nv - 1));
 #pragma unroll
                 for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
                     if (c4 >= nv) break;
-                    const uint32_t b4[4] = {wv[c4].x, wv[c4].y, wv[c4].z, wv[c4].w};
+                    const uint4 b = valid ? wv[c4] : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+                    const uint32_t b4[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc)
-                        *reinterpret_cast<uint32_t*>(atoms + ((1 + pl) * kDxSteps + 4 * c4 + cc) * 512 + 16 * nrow) = b4[cc];
+                        *reinterpret_cast<uint32_t*>(atoms + (kDxSteps + 4 * c4 + cc) * 512 + 16 * (m & 31) + 4 * (m >> 5)) =
+                            b4[cc];
                 }
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -352,9 +418,22 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
             if (!mbar_wait(&tfull[buf], acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             float v[32];
-            tmem_ld32_nowait(tmem + (uint32_t(q * 32) << 16) + uint32_t(32 * buf), v);
-            tmem_wait_16(v);
-            tmem_fence_regs(v + 16);
+            // column c of the hi rows plus column NB + c of the lo rows
+            const uint32_t tacc = tmem + (uint32_t(q * 32) << 16) + uint32_t(kDxAccCols * buf);
+            if (p.NB == 32) {
+                float w[32];
+                tmem_ld32_nowait(tacc, v);
+                tmem_ld32_nowait(tacc + 32u, w);
+                tmem_wait_ld(v, w);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) v[c] += w[c];
+            } else {
+                tmem_ld32_nowait(tacc, v);
+                tmem_wait_16(v);
+                tmem_fence_regs(v + 16);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) v[c] += v[16 + c];
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -473,6 +552,7 @@ cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
     p.K = H;
     p.m_blocks = F / 64;
     p.wsc = a.w13s;
+    p.wcodes = static_cast<const uint8_t*>(a.w13);
     p.bsc_hi = xsh;
     p.bsc_lo = xsl;
     e = launch_dep(decode_mx_mma_kernel<0>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, kDxThreads, smem, st,
@@ -484,6 +564,7 @@ cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
     p.K = F;
     p.m_blocks = H / 128;
     p.wsc = a.w2s;
+    p.wcodes = static_cast<const uint8_t*>(a.w2);
     p.bsc_hi = hsh;
     p.bsc_lo = hsl;
     e = launch_dep(decode_mx_mma_kernel<1>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, kDxThreads, smem, st,
