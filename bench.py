@@ -666,8 +666,8 @@ def main():
                     help="with --prefill-only: the batch size (default: the shape's prefill size)")
     ap.add_argument("--decode-rotations", type=int, default=4,
                     help="with --decode-only: weight copies rotated between calls (1 for small ncu captures)")
-    ap.add_argument("--block-scaled-decode", action="store_true",
-                    help="run MXFP4 decode batches on the block-scaled tensor-core path")
+    ap.add_argument("--block-scaled-decode", default=None, choices=["0", "1", "2"],
+                    help="MXFP4 decode on the block-scaled tensor cores: 0 never, 1 always, 2 from 4 tokens (default)")
     ap.add_argument("--hbm-ceiling", action="store_true",
                     help="only time plain streaming reads and copies of decode-sized transfers")
     args = ap.parse_args()
@@ -700,8 +700,8 @@ def main():
                               "sizes": measure_hbm_ceiling(torch, F)}), flush=True)
         return
 
-    if args.block_scaled_decode:
-        F.ft_set_block_scaled_decode(1)
+    if args.block_scaled_decode is not None:
+        F.ft_set_block_scaled_decode(int(args.block_scaled_decode))
 
     if args.decode_only:
         cfg = inputs.CONFIGS[args.decode_only]

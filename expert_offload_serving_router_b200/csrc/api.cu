@@ -36,8 +36,12 @@ static int init_decode_max() {
 static int g_decode_max = init_decode_max();
 int decode_max() { return g_decode_max; }
 
-static bool g_block_scaled_decode = false;
-bool block_scaled_decode() { return g_block_scaled_decode; }
+// 0 never, 1 every eligible decode batch, 2 (default) eligible batches of kBlockScaledMinT+ tokens
+static int g_block_scaled_decode = 2;
+constexpr int kBlockScaledMinT = 4;
+bool block_scaled_decode(int T) {
+    return g_block_scaled_decode == 1 || (g_block_scaled_decode == 2 && T >= kBlockScaledMinT);
+}
 
 static unsigned long long g_gemm_wait_ns = kWaitNs;
 unsigned long long gemm_wait_ns() { return g_gemm_wait_ns; }
@@ -179,9 +183,10 @@ int32_t ft_set_decode_max_tokens(int32_t t) {
 
 int32_t ft_get_decode_max_tokens(void) { return g_decode_max; }
 
-int32_t ft_set_block_scaled_decode(int32_t enable) {
-    const int32_t prev = g_block_scaled_decode ? 1 : 0;
-    g_block_scaled_decode = enable != 0;
+int32_t ft_set_block_scaled_decode(int32_t mode) {
+    if (mode < 0 || mode > 2) return -1;
+    const int32_t prev = g_block_scaled_decode;
+    g_block_scaled_decode = mode;
     return prev;
 }
 

@@ -261,13 +261,13 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 // BF16 decode batches of at least this many tokens run on the tensor cores (decode_mma.cu);
 // smaller ones stream through the SIMT GEMVs below, which measured faster at T <= 4
 constexpr int kDecodeMmaMinT = 8;
-// MXFP4 decode batches run on the block-scaled tensor cores only when selected
-// (ft_set_block_scaled_decode): measured slower than the GEMVs below so far
+// MXFP4 decode batches of 4+ tokens run on the block-scaled tensor cores (ft_set_block_scaled_decode
+// selects never / always / that default); smaller ones on the GEMVs below, faster there
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
     if (a.T >= kDecodeMmaMinT && decode_mma_eligible(a)) return launch_decode_mma(a, st);
-    if (block_scaled_decode() && decode_mx_eligible(a)) return launch_decode_mx(a, st);
+    if (block_scaled_decode(a.T) && decode_mx_eligible(a)) return launch_decode_mx(a, st);
     const int P = a.T * a.k, R = P + (a.S ? a.T : 0);
     const int G = a.E + (a.S ? 1 : 0);
     {

@@ -92,7 +92,7 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st);
 // block-scaled MXFP4 decode on the tensor cores (decode_mx_mma.cu)
 bool decode_mx_eligible(const DecodeArgs& a);
 cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st);
-bool block_scaled_decode();   // api.cu: ft_set_block_scaled_decode
+bool block_scaled_decode(int T);   // api.cu: ft_set_block_scaled_decode
 int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st);
 // bound (ns without progress) on each pipeline wait of the grouped GEMMs (api.cu)
 unsigned long long gemm_wait_ns();

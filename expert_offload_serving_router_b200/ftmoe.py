@@ -177,8 +177,8 @@ def ft_set_pipeline_wait_limit_ns(ns: int) -> int:
     return lib().ft_set_pipeline_wait_limit_ns(ns)
 
 
-def ft_set_block_scaled_decode(enable: int) -> int:
-    return lib().ft_set_block_scaled_decode(enable)
+def ft_set_block_scaled_decode(mode: int) -> int:
+    return lib().ft_set_block_scaled_decode(mode)
 
 
 def ft_hbm_read_probe(buf, nbytes: int, sink, ctas_per_sm: int, stream=None) -> None:

@@ -132,18 +132,20 @@ const char* ft_version(void);
 int32_t ft_set_decode_max_tokens(int32_t t);
 int32_t ft_get_decode_max_tokens(void);
 
-/* Block-scaled tensor-core decode for MXFP4 weights (process-wide, default off;
- * returns the previous setting).  When on, decode batches (T <= threshold) of
- * MXFP4 layers with contiguous weights, no shared expert, H and F multiples of
- * 512 and at most 4096 run the experts as tcgen05.mma.kind::mxf8f6f4.block_scale
- * MMAs: E2M1 weights with their E8M0 scales straight from HBM (no dequantisation)
- * times the activations carried as two E4M3 planes (high plane and the plane of
- * the remainder, each with its own E8M0 scale per 32 elements; x before gate/up,
- * h before down).  Accuracy: under 1e-2 of max|y| against the exact layer (a third
- * of the 3e-2 MXFP4 tolerance); the default GEMVs multiply the exactly decoded
- * weights in f16.  It needs the workspace of ft_moe_workspace_bytes (MXFP4 shapes reserve
- * room for the planes).  On the measured shapes it is slower than the GEMVs. */
-int32_t ft_set_block_scaled_decode(int32_t enable);
+/* Block-scaled tensor-core decode for MXFP4 weights.  mode 0: never; 1: every
+ * eligible decode batch; 2 (the default): eligible batches of 4 or more tokens
+ * (on the DeepSeek-V4-Flash shape it is faster than the GEMVs from 4 tokens on,
+ * slower for 1).  Process-wide; returns the previous mode, or -1 (and changes
+ * nothing) for a mode outside 0..2.  Eligible: MXFP4 layers with contiguous
+ * weights, no shared expert, H and F multiples of 512 and at most 4096.  The
+ * experts then run as tcgen05.mma.kind::mxf8f6f4.block_scale MMAs: E2M1 weights
+ * with their E8M0 scales straight from HBM (no dequantisation) times the
+ * activations carried as two E4M3 planes (high plane and the plane of the
+ * remainder, each with its own E8M0 scale per 32 elements; x before gate/up, h
+ * before down).  Accuracy: under 1e-2 of max|y| against the exact layer (a third
+ * of the 3e-2 MXFP4 tolerance); the GEMVs multiply the exactly decoded weights
+ * in f16.  ft_moe_workspace_bytes reserves room for the planes on MXFP4 shapes. */
+int32_t ft_set_block_scaled_decode(int32_t mode);
 
 /* Bound on every pipeline wait of the grouped-GEMM kernels (steps 3 and 4 when
  * T > decode threshold): the time, in ns, a role waits for a stage without

@@ -245,7 +245,7 @@ def test_read_probe_rejects_bad_arguments_on_host():
 
 def test_block_scaled_decode_switch_returns_previous_setting():
     from expert_offload_serving_router_b200 import ftmoe as F
-    assert F.ft_set_block_scaled_decode(1) == 0
-    assert F.ft_set_block_scaled_decode(7) == 1
+    assert F.ft_set_block_scaled_decode(1) == 2          # default: from 4 tokens on
+    assert F.ft_set_block_scaled_decode(7) == -1         # rejected, nothing changes
     assert F.ft_set_block_scaled_decode(0) == 1
-    assert F.ft_set_block_scaled_decode(0) == 0
+    assert F.ft_set_block_scaled_decode(2) == 0

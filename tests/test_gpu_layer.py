@@ -39,8 +39,8 @@ def full_check(L, x, n_rows=12, seed=0):
 
 
 # decode batches: BF16 T >= 8 run on the tensor cores (qwen3_a3b 8/16/32, gemma4_26b_a4b 16,
-# tiny 8), smaller ones and MXFP4 on the GEMVs; MXFP4 batches whose token rows exceed 64 KB of x
-# (dsv4_flash T=20) take the GEMV variant that stages each group's rows per batch
+# tiny 8), smaller ones on the GEMVs; MXFP4 (dsv4_flash) T >= 4 on the block-scaled tensor cores,
+# T = 1 on the GEMVs (the GEMV variants for larger batches: test_mxfp4_gemv_decode below)
 CASES = [("tiny", 64), ("tiny", 1), ("tiny", 37), ("tiny", 8),
          ("qwen3_a3b", 1), ("qwen3_a3b", 4), ("qwen3_a3b", 8), ("qwen3_a3b", 16), ("qwen3_a3b", 32), ("qwen3_a3b", 4096),
          ("dsv4_flash", 1), ("dsv4_flash", 8), ("dsv4_flash", 20), ("dsv4_flash", 8192),
@@ -267,3 +267,17 @@ def test_block_scaled_decode_chained_is_deterministic(block_scaled_decode):
     F.ft_moe_check(ws)
     for s in range(4):
         assert np.array_equal(host(bufs[s + 1], np.uint16), ref[s]), f"step {s} differs"
+
+
+@pytest.mark.parametrize("T", [4, 8, 20, 32])
+def test_mxfp4_gemv_decode_matches_oracle(T):
+    """The MXFP4 GEMV decode kept for batches the block-scaled path does not take (block-scaled
+    decode switched off): T = 20 and 32 exceed 64 KB of x rows and take the variant that stages
+    each group's rows per batch."""
+    prev = F.ft_set_block_scaled_decode(0)
+    try:
+        L = layer("dsv4_flash")
+        x = inputs.make_tokens(L.cfg, T, seed=6)
+        full_check(L, x, n_rows=T)
+    finally:
+        assert F.ft_set_block_scaled_decode(prev) == 0
