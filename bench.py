@@ -588,6 +588,36 @@ def measure_stack(torch, F, rank, hbm_gbs):
     return out
 
 
+def measure_tma_reads(torch, F, reps=5):
+    """Rate of TMA loads of 128-byte rows into a shared-memory ring (the library's TMA read probe,
+    one CTA per SM): whole 128-row tiles against tile::gather4 loads of the same rows, and gather4
+    loads of hashed rows inside a 64 MiB region (permuted token rows as a grouped GEMM would read
+    them in place; the region fits in L2), with tile loads of that region for reference.  GB/s
+    counts the bytes landed in shared memory; median of `reps` launches."""
+    gib, region = 1 << 30, 64 << 20
+    buf = torch.empty(gib // 4, dtype=torch.float32, device="cuda").normal_()
+    small = buf[: region // 4]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    cases = [("tiles, 1 GiB", 0, buf, gib, 0), ("gather4 consecutive rows, 1 GiB", 1, buf, gib, 0),
+             ("gather4 hashed rows in 64 MiB", 2, buf, gib, region), ("tiles, 64 MiB", 0, small, region, 0)]
+    out = []
+    for name, mode, b, nbytes, reg in cases:
+        landed = (nbytes // 128 // 128 // nsm) * nsm * 128 * 128
+        times = []
+        for _ in range(reps + 1):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            F.ft_tma_read_probe(mode, b, nbytes, reg, status, torch.cuda.current_stream())
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e3)
+        st = int(status.item())
+        us = float(np.median(times[1:]))
+        out.append({"case": name, "us": us, "gbs": landed / (us * 1e-6) / 1e9, "status": st})
+    return out
+
+
 def measure_hbm_ceiling(torch, F, sizes_mb=(8, 16, 32, 64, 76, 128, 256, 512, 1024, 2048), iters=20):
     """Streaming throughput of a plain read (the library's 16-byte-load probe kernel, best of 1,
     2, 4 and 8 CTAs per SM) and of a device-to-device copy for transfers of a given size,
@@ -668,6 +698,8 @@ def main():
                     help="with --decode-only: weight copies rotated between calls (1 for small ncu captures)")
     ap.add_argument("--block-scaled-decode", default=None, choices=["0", "1", "2"],
                     help="MXFP4 decode on the block-scaled tensor cores: 0 never, 1 always, 2 from 4 tokens (default)")
+    ap.add_argument("--tma-probe", action="store_true",
+                    help="only time TMA tile loads against tile::gather4 row gathers")
     ap.add_argument("--hbm-ceiling", action="store_true",
                     help="only time plain streaming reads and copies of decode-sized transfers")
     args = ap.parse_args()
@@ -693,6 +725,11 @@ def main():
         ftbuild.build()
     F.lib()
     hbm_gbs, tc_burst, tc_sus, peak_src = peaks()
+
+    if args.tma_probe:
+        if rank == 0:
+            print(json.dumps({"mode": "tma-probe", "reads": measure_tma_reads(torch, F)}), flush=True)
+        return
 
     if args.hbm_ceiling:
         if rank == 0:

@@ -60,6 +60,7 @@ _SIGS = {
     "ft_set_pipeline_wait_limit_ns": (c_u64, [c_u64]),
     "ft_set_block_scaled_decode": (c_i32, [c_i32]),
     "ft_hbm_read_probe": (c_i32, [c_vp, c_sz, c_vp, c_i32, c_vp]),
+    "ft_tma_read_probe": (c_i32, [c_i32, c_vp, c_sz, c_sz, c_vp, c_vp]),
     "ft_moe_workspace_bytes": (c_sz, [ctypes.POINTER(ft_moe_shape), c_i32]),
     "ft_moe_workspace_init": (c_i32, [c_vp, c_sz, c_vp]),
     "ft_moe_check": (c_i32, [c_vp, c_vp]),
@@ -183,6 +184,10 @@ def ft_set_block_scaled_decode(mode: int) -> int:
 
 def ft_hbm_read_probe(buf, nbytes: int, sink, ctas_per_sm: int, stream=None) -> None:
     _check(lib().ft_hbm_read_probe(_p(buf), nbytes, _p(sink), ctas_per_sm, _s(stream)))
+
+
+def ft_tma_read_probe(mode: int, buf, nbytes: int, region_bytes: int, status, stream=None) -> None:
+    _check(lib().ft_tma_read_probe(mode, _p(buf), nbytes, region_bytes, _p(status), _s(stream)))
 
 
 def ft_moe_workspace_bytes(shape: ft_moe_shape, max_tokens: int) -> int:

@@ -402,6 +402,16 @@ ft_status ft_lru_resize(int32_t E, int32_t n_old, int32_t n_new, int32_t* conten
  * which HBM reaches its copy peak). */
 ft_status ft_hbm_read_probe(const void* buf, size_t bytes, uint32_t* sink, int32_t ctas_per_sm, void* stream);
 
+/* Diagnostic: TMA loads of 128-byte rows of `buf` into a 6-stage shared-memory ring, one CTA
+ * per SM, nothing computed: mode 0 loads 128-row tiles; mode 1 the same rows as tile::gather4
+ * loads (four rows per load); mode 2 gather4 loads of hashed rows inside the first
+ * region_bytes (how a grouped GEMM would read permuted token rows in place).  Each CTA
+ * streams bytes / (128 x 128 x SMs) tiles.  buf: device, 16-byte aligned, bytes >= 128 x 128
+ * x SMs.  *status (device word, set to zero by the caller): 2 or 3 if a bounded wait ran out
+ * (no fault is raised).  Time it with events on `stream`; returns after the launch. */
+ft_status ft_tma_read_probe(int32_t mode, const void* buf, size_t bytes, size_t region_bytes, uint32_t* status,
+                            void* stream);
+
 /* Test hook for failure handling: make the n-th host->device expert copy
  * enqueue (counting from 1 after this call) report failure (n = 0 disables).
  * The failing decode step returns FT_ERR_CUDA and rolls the cache state of

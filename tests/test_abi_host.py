@@ -249,3 +249,13 @@ def test_block_scaled_decode_switch_returns_previous_setting():
     assert F.ft_set_block_scaled_decode(7) == -1         # rejected, nothing changes
     assert F.ft_set_block_scaled_decode(0) == 1
     assert F.ft_set_block_scaled_decode(2) == 0
+
+
+def test_tma_probe_rejects_bad_arguments_on_host():
+    from expert_offload_serving_router_b200 import ftmoe as F
+    for args in [(3, 4096, 1 << 30, 0, 4096), (0, 0, 1 << 30, 0, 4096), (0, 4096, 1 << 30, 0, 0), (0, 4104, 1 << 30, 0, 4096),
+                 (0, 4096, 128, 0, 4096), (2, 4096, 1 << 30, 2 << 30, 4096)]:
+        mode, buf, n, region, status = args
+        with pytest.raises(F.FtError) as ei:
+            F.ft_tma_read_probe(mode, buf, n, region, status, stream=0)
+        assert ei.value.status == F.FT_ERR_INVALID_ARG
