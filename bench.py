@@ -671,8 +671,8 @@ def measure_hbm_ceiling(torch, F, sizes_mb=(8, 16, 32, 64, 76, 128, 256, 512, 10
     return out
 
 
-EXTRA_WORKLOADS = [("qwen3_a3b", [1, 4, 16]), ("gemma4_26b_a4b", [1]), ("tiny", [])]
-HEADLINE_DECODE = [1, 8]
+EXTRA_WORKLOADS = [("qwen3_a3b", [1, 4, 8, 16, 32]), ("gemma4_26b_a4b", [1, 4, 8, 16, 32]), ("tiny", [])]
+HEADLINE_DECODE = [1, 4, 8, 16, 32]
 ROOFLINE_SUMMARY = ("moe_gemm_mxfp4_dsv4_flash_T8192.md", ("gemm_mx_sm100.cu", "gemm_common.cuh", "sm100.cuh"))
 
 
