@@ -1,7 +1,7 @@
 // Steps 3/4 (decode, BF16 weights) on the tensor cores.  A decode batch (T <= 32 tokens) is a
 // stream over the routed experts' weights; with several tokens per expert the SIMT GEMV spends
 // as long on its FMAs and shared-memory reads of x as on the stream.  Here every MMA has the
-// weights as A (M = 128 rows, TMA-fed through a four-stage ring) and the tokens as B (N =
+// weights as A (M = 128 rows, TMA-fed through a three-stage ring) and the tokens as B (N =
 // T rounded up to 16), so the arithmetic is the tensor cores' and each CTA is a weight stream.
 //
 //   gate/up (MODE 0): items (active group, 128 interleaved gate/up rows = 64 f).
@@ -13,7 +13,7 @@
 //       groups and are ignored), o[row, hidden] -> bf16.  The gate-weighted combine back to
 //       token order follows as its own small kernel (programmatic dependent launch), so no
 //       CTA here waits on, or sums for, the others.
-// Persistent CTAs (two per SM) walk the items with one TMA ring; accumulators are double
+// Persistent CTAs (three per SM) walk the items with one TMA ring; accumulators are double
 // buffered.  Warp roles: 0 TMA producer, 1 TMEM allocation + MMA issuer, 2-5 epilogue (TMEM
 // lane quarter warp & 3).  Every wait is bounded (the grouped GEMMs' limit).
 #include "gemm_common.cuh"
@@ -21,7 +21,7 @@
 
 namespace ftmoe {
 
-constexpr int kDmSt = 4;                           // stages of one 64-deep K step
+constexpr int kDmSt = 3;                           // stages of one 64-deep K step (three CTAs per SM)
 constexpr int kDmATile = 128 * kBK * 2;            // 16 KB
 constexpr int kDmBTile = 32 * kBK * 2;             // 4 KB: up to 32 token rows
 constexpr int kDmThreads = 192;
@@ -66,7 +66,7 @@ __device__ __forceinline__ DmItem dm_item(const DecMmaParams& p, int it) {
 // ring runs across items and the accumulators are double buffered (2 x 32 TMEM columns), so
 // an item's epilogue (and combine) overlaps the next item's weight stream.
 template <int MODE>
-__global__ void __launch_bounds__(kDmThreads, 2)
+__global__ void __launch_bounds__(kDmThreads, 3)
 decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sw,
                   const __grid_constant__ CUtensorMap tm_b, DecMmaParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -273,8 +273,11 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    // persistent grids: up to two CTAs per SM, never more than the items a batch can have
-    const int cap = 2 * num_sms();
+    // persistent grids: up to three CTAs per SM (3-stage rings), never more than the items a batch
+    // can have.  Three shallower rings per SM beat two deeper ones whenever a batch's items fit in
+    // one wave of 3 x SMs (qwen3_a3b T = 8: 64.8 -> 57.0 us) and lose a little when a second wave
+    // runs on few CTAs (T = 32: 100.2 -> 105.5 us)
+    const int cap = 3 * num_sms();
     p.m_blocks = F / 64;
     cudaError_t e = launch_dependent(decode_mma_kernel<0>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, smem,
                                      st, gw, gsw, gb, p);
