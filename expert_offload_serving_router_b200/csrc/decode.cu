@@ -259,14 +259,18 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 // BF16 decode batches of at least this many tokens run on the tensor cores (decode_mma.cu);
-// smaller ones stream through the SIMT GEMVs below, which measured faster at T <= 4
-constexpr int kDecodeMmaMinT = 8;
+// smaller ones stream through the SIMT GEMVs below.  With a shared expert one group always holds
+// every token, and the tensor cores win from two tokens on (gemma4_26b_a4b T = 2 / 4: 55.3 ->
+// 50.5 / 84.2 -> 69.9 us); without one from four (qwen3_a3b T = 3: 39.9 vs 42.3, T = 4 even,
+// T = 6: 56.9 -> 49.4 us)
+constexpr int kDecodeMmaMinT = 4;
+constexpr int kDecodeMmaMinTShared = 2;
 // MXFP4 decode batches of 4+ tokens run on the block-scaled tensor cores (ft_set_block_scaled_decode
 // selects never / always / that default); smaller ones on the GEMVs below, faster there
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
-    if (a.T >= kDecodeMmaMinT && decode_mma_eligible(a)) return launch_decode_mma(a, st);
+    if (a.T >= (a.S ? kDecodeMmaMinTShared : kDecodeMmaMinT) && decode_mma_eligible(a)) return launch_decode_mma(a, st);
     if (block_scaled_decode(a.T) && decode_mx_eligible(a)) return launch_decode_mx(a, st);
     const int P = a.T * a.k, R = P + (a.S ? a.T : 0);
     const int G = a.E + (a.S ? 1 : 0);

@@ -38,13 +38,15 @@ def full_check(L, x, n_rows=12, seed=0):
     return y, idx, lg, rel
 
 
-# decode batches: BF16 T >= 8 run on the tensor cores (qwen3_a3b 8/16/32, gemma4_26b_a4b 16,
-# tiny 8), smaller ones on the GEMVs; MXFP4 (dsv4_flash) T >= 4 on the block-scaled tensor cores,
-# T = 1 on the GEMVs (the GEMV variants for larger batches: test_mxfp4_gemv_decode below)
-CASES = [("tiny", 64), ("tiny", 1), ("tiny", 37), ("tiny", 8),
-         ("qwen3_a3b", 1), ("qwen3_a3b", 4), ("qwen3_a3b", 8), ("qwen3_a3b", 16), ("qwen3_a3b", 32), ("qwen3_a3b", 4096),
+# decode batches (T <= 32): BF16 T >= 4, or T >= 2 with a shared expert, run on the tensor cores
+# (qwen3_a3b 4/8/16/32, gemma4_26b_a4b 2/16, tiny 8), smaller ones on the GEMVs (qwen3_a3b 1/3,
+# gemma4_26b_a4b 1, tiny 1/3); MXFP4 (dsv4_flash) T >= 4 on the block-scaled tensor cores, T = 1 on
+# the GEMVs (the GEMV variants for larger batches: test_mxfp4_gemv_decode below); larger T on the
+# grouped GEMMs
+CASES = [("tiny", 64), ("tiny", 1), ("tiny", 37), ("tiny", 8), ("tiny", 3),
+         ("qwen3_a3b", 1), ("qwen3_a3b", 3), ("qwen3_a3b", 4), ("qwen3_a3b", 8), ("qwen3_a3b", 16), ("qwen3_a3b", 32), ("qwen3_a3b", 4096),
          ("dsv4_flash", 1), ("dsv4_flash", 8), ("dsv4_flash", 20), ("dsv4_flash", 8192),
-         ("gemma4_26b_a4b", 1), ("gemma4_26b_a4b", 16), ("gemma4_26b_a4b", 2048)]
+         ("gemma4_26b_a4b", 1), ("gemma4_26b_a4b", 2), ("gemma4_26b_a4b", 16), ("gemma4_26b_a4b", 2048)]
 
 
 @pytest.mark.parametrize("name,T", CASES)
