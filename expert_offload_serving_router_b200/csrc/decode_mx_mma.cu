@@ -110,14 +110,6 @@ __global__ void __launch_bounds__(256) quant2_kernel(const uint16_t* __restrict_
 
 __device__ __forceinline__ int group_token_of(int flat, int P, int k) { return flat < P ? flat / k : flat - P; }
 
-// Bring `bytes` (multiple of 16, 16-byte aligned) into L2 ahead of the TMA ring, 16 KB per request.
-__device__ __forceinline__ void l2_prefetch(const uint8_t* ptr, uint32_t bytes) {
-    for (uint32_t o = 0; o < bytes; o += 16384u) {
-        const uint32_t n = bytes - o < 16384u ? bytes - o : 16384u;
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr + o), "r"(n) : "memory");
-    }
-}
-
 // ------------------------------------------------------------------ block-scaled MMA
 // A stage is a 256-deep K step made of two 128-deep sub-tiles: one barrier wait and one commit per
 // eight MMAs (an mbarrier poll costs the issuing thread about as much as two small MMAs).
@@ -145,7 +137,6 @@ struct DecMxParams {
     const int32_t* sorted_flat;
     const int32_t* sched;
     const uint8_t* wsc;               // weight scales [E, rows, K/32]
-    const uint8_t* wcodes;            // packed codes: w13 [E][2F][H/2] (gate rows, then up rows) or w2 [E][H][F/2]
     const uint8_t* bsc_hi;            // activation scales [rows, K/32], one per plane
     const uint8_t* bsc_lo;
     uint16_t* h;
@@ -205,27 +196,6 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    // an item's packed codes: gate/up 64 gate rows + the same 64 up rows; down 128 rows (contiguous)
-    auto prefetch_item = [&](int it) {
-        const int slot = it / p.m_blocks, rg = it - slot * p.m_blocks;
-        const int g = __ldcg(p.sched + 2 + (p.G + 1) + slot);
-        if (slot >= p.G || g < 0 || g >= p.E) return;       // only a hint: never an address outside w
-        if (MODE == 0) {
-            const size_t rb = size_t(p.H) / 2, base = size_t(g) * 2 * p.F * rb;
-            l2_prefetch(p.wcodes + base + size_t(64 * rg) * rb, uint32_t(64 * rb));
-            l2_prefetch(p.wcodes + base + size_t(p.F + 64 * rg) * rb, uint32_t(64 * rb));
-        } else {
-            const size_t rb = size_t(p.F) / 2;
-            l2_prefetch(p.wcodes + (size_t(g) * p.H + 128 * rg) * rb, uint32_t(128 * rb));
-        }
-    };
-    // The routing (schedule, offsets) was final before this grid could launch: the kernel ahead
-    // of it started its own dependents only after waiting for the kernels that wrote it.  So the
-    // first item's weights can stream into L2 while this grid waits for the activations.
-    if (threadIdx.x == 0) {
-        const int n0 = __ldcg(p.sched + 1) * p.m_blocks;
-        if (int(blockIdx.x) < n0) prefetch_item(blockIdx.x);
-    }
     pdl_wait();          // routing, the activation planes and h come from the preceding kernels
     pdl_trigger();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -265,7 +235,6 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                 const int slot = it / p.m_blocks, rg = it - slot * p.m_blocks;
                 const int g = p.sched[2 + (p.G + 1) + slot];
                 const int brow = MODE == 0 ? 0 : p.offsets[g];
-                if (it + int(gridDim.x) < n_items) prefetch_item(it + gridDim.x);   // the next item's weights
                 for (int kb = 0; kb < nk / 2; ++kb, ++step) {
                     if (!wait_fast(&empty[s], phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
                     mbar_expect_tx(&full[s], bytes);
@@ -552,7 +521,6 @@ cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
     p.K = H;
     p.m_blocks = F / 64;
     p.wsc = a.w13s;
-    p.wcodes = static_cast<const uint8_t*>(a.w13);
     p.bsc_hi = xsh;
     p.bsc_lo = xsl;
     e = launch_dep(decode_mx_mma_kernel<0>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, kDxThreads, smem, st,
@@ -564,7 +532,6 @@ cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
     p.K = F;
     p.m_blocks = H / 128;
     p.wsc = a.w2s;
-    p.wcodes = static_cast<const uint8_t*>(a.w2);
     p.bsc_hi = hsh;
     p.bsc_lo = hsl;
     e = launch_dep(decode_mx_mma_kernel<1>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, kDxThreads, smem, st,
