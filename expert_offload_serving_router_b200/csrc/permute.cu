@@ -107,6 +107,42 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(PermArgs a, int C) {
 // One CTA per 128 pairs (8 warps x 16): scatter the permutation, then gather the x rows.
 constexpr int kScatterItems = 128;
 
+// A warp copies rows q, q + 1 (q = 2 warp, 2 warp + 16, ...) of the CTA's pairs from x into
+// x_sorted, every 16-byte vector of both rows loaded before the first store (NV per lane and
+// row: rows of up to 32 NV vectors).  Rows whose pair is dropped (pos < 0) are skipped; the
+// loads of a missing second row re-read the first (in range) and are not stored.
+template <int NV>
+__device__ __forceinline__ void gather_two_rows(const PermArgs& a, const int* spos, const int* stok, int n, int nv,
+                                                int warp, int lane) {
+    for (int q = 2 * warp; q < n; q += 16) {
+        const int pos0 = spos[q], pos1 = q + 1 < n ? spos[q + 1] : -1;
+        const uint4* src0 = reinterpret_cast<const uint4*>(a.x + size_t(stok[q]) * a.H);
+        const uint4* src1 = reinterpret_cast<const uint4*>(a.x + size_t(q + 1 < n ? stok[q + 1] : stok[q]) * a.H);
+        uint4* dst0 = reinterpret_cast<uint4*>(a.x_sorted + size_t(pos0 < 0 ? 0 : pos0) * a.H);
+        uint4* dst1 = reinterpret_cast<uint4*>(a.x_sorted + size_t(pos1 < 0 ? 0 : pos1) * a.H);
+        uint4 u0[NV], u1[NV];
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int v = lane + 32 * j;
+            if (v < nv) {
+                if (pos0 >= 0) u0[j] = __ldg(src0 + v);
+                if (pos1 >= 0) u1[j] = __ldg(src1 + v);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int v = lane + 32 * j;
+            if (v < nv) {
+                if (pos0 >= 0) dst0[v] = u0[j];
+                if (pos1 >= 0) dst1[v] = u1[j];
+            }
+        }
+    }
+}
+
+// GV: the gather form, chosen on the host from H: 8 / 12 = two rows per warp with GV vectors per
+// lane and row (rows of up to 256 / 384 vectors), 0 = one row per warp, 4 vectors in flight.
+template <int GV>
 __global__ void __launch_bounds__(256) perm_scatter_kernel(PermArgs a) {
     __shared__ int spos[kScatterItems];
     __shared__ int stok[kScatterItems];
@@ -129,36 +165,13 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(PermArgs a) {
     }
     if (!a.x_sorted) return;
     __syncthreads();
-    // gather, 16-byte vectors.  Rows of up to 4 KB: one warp moves two rows at once with all
-    // their vectors in flight (16 per lane); longer rows: one warp per row, 4 vectors in flight
-    // per lane (measured best for each at H = 2048 and H = 4096).
+    // gather, 16-byte vectors.  Rows of up to 4 KB (6 KB): one warp moves two rows at once with
+    // all their vectors in flight (8 / 12 per lane and row); longer rows: one warp per row, 4
+    // vectors in flight per lane (measured best for each at H = 2048, 2816 and 4096).
     const int lane = tid & 31, warp = tid >> 5;
     const int nv = a.H / 8;
-    if (nv <= 256) {
-        for (int q = 2 * warp; q < n; q += 16) {
-            const int pos0 = spos[q], pos1 = q + 1 < n ? spos[q + 1] : -1;
-            const uint4* src0 = reinterpret_cast<const uint4*>(a.x + size_t(stok[q]) * a.H);
-            const uint4* src1 = reinterpret_cast<const uint4*>(a.x + size_t(q + 1 < n ? stok[q + 1] : stok[q]) * a.H);
-            uint4* dst0 = reinterpret_cast<uint4*>(a.x_sorted + size_t(pos0 < 0 ? 0 : pos0) * a.H);
-            uint4* dst1 = reinterpret_cast<uint4*>(a.x_sorted + size_t(pos1 < 0 ? 0 : pos1) * a.H);
-            uint4 u0[8], u1[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int v = lane + 32 * j;
-                if (v < nv) {
-                    if (pos0 >= 0) u0[j] = __ldg(src0 + v);
-                    if (pos1 >= 0) u1[j] = __ldg(src1 + v);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int v = lane + 32 * j;
-                if (v < nv) {
-                    if (pos0 >= 0) dst0[v] = u0[j];
-                    if (pos1 >= 0) dst1[v] = u1[j];
-                }
-            }
-        }
+    if constexpr (GV > 0) {
+        gather_two_rows<GV>(a, spos, stok, n, nv, warp, lane);
         return;
     }
     for (int q = warp; q < n; q += 8) {
@@ -213,7 +226,10 @@ cudaError_t launch_permute(int T, int k, int E, int S, int H, const int32_t* idx
         PermArgs a{T, k, E, S, H, idx, x, x_sorted, chunk_cnt, chunk_base, local_rank, out};
         perm_count_kernel<<<C, 256, 0, st>>>(a);
         perm_scan_kernel<<<1, 1024, 0, st>>>(a, C);
-        perm_scatter_kernel<<<(R + kScatterItems - 1) / kScatterItems, 256, 0, st>>>(a);
+        const int grid = (R + kScatterItems - 1) / kScatterItems, nv = H / 8;
+        if (!x_sorted || nv <= 256) perm_scatter_kernel<8><<<grid, 256, 0, st>>>(a);
+        else if (nv <= 384) perm_scatter_kernel<12><<<grid, 256, 0, st>>>(a);
+        else perm_scatter_kernel<0><<<grid, 256, 0, st>>>(a);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
