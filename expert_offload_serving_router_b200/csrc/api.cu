@@ -263,7 +263,8 @@ ft_status ft_moe_permute(const ft_moe_shape* shape, int32_t T, const int32_t* to
     WsLayout L;
     if ((s = check_ws(shape, T, ws, ws_bytes, &L))) return s;
     if ((s = cuda_state())) return s;
-    PermOut po{offsets, sorted_flat, inv_pos, ws_at<int32_t>(ws, L.sched), ws_at<uint32_t>(ws, L.err)};
+    PermOut po{offsets, sorted_flat, inv_pos, ws_at<int32_t>(ws, L.sched), ws_at<uint32_t>(ws, L.err),
+               ws_at<uint32_t>(ws, L.err) + kWsReady};
     return cuda_ok(launch_permute(T, shape->top_k, shape->num_experts, shape->num_shared, shape->hidden, topk_idx,
                                   static_cast<const uint16_t*>(x), static_cast<uint16_t*>(x_sorted),
                                   ws_at<int32_t>(ws, L.chunk_cnt), ws_at<int32_t>(ws, L.chunk_base),
@@ -368,7 +369,7 @@ ft_status ft_moe_layer_forward(const ft_moe_shape* shape, int32_t T, const void*
     int32_t* offsets = ws_at<int32_t>(ws, L.offsets);
     int32_t* sorted_flat = ws_at<int32_t>(ws, L.sorted_flat);
     int32_t* inv_pos = ws_at<int32_t>(ws, L.inv_pos);
-    PermOut po{offsets, sorted_flat, inv_pos, ws_at<int32_t>(ws, L.sched), err};
+    PermOut po{offsets, sorted_flat, inv_pos, ws_at<int32_t>(ws, L.sched), err, err + kWsReady};
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     if (decode) {
         // route + top-k + permutation in one launch, then two weight-streaming kernels

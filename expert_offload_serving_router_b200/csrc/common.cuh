@@ -83,8 +83,11 @@ struct WsLayout {
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace header (cleared by ft_moe_workspace_init): word 0 device error flag, word 1 the
-// decode router's ticket (left at zero by every launch); the rest is reserved.
+// decode router's ticket (left at zero by every launch), words kWsReady.. the tensor-core
+// decode's per-group counters (2 x (E + S) words, left at zero by every launch and zeroed by
+// the decode permutation); the rest is reserved.
 constexpr size_t kWsHeaderBytes = 4096;
+constexpr int kWsReady = 64;            // word index; 2 x 257 counters fit
 constexpr int kRouteTok = 128;          // tokens per router CTA
 constexpr int kRouteTargetCtas = 148;   // split K until the router grid covers about one wave
 constexpr int kRouteMaxSplit = 8;

@@ -4,18 +4,24 @@
 // weights as A (M = 128 rows, TMA-fed through a three-stage ring) and the tokens as B (N =
 // T rounded up to 16), so the arithmetic is the tensor cores' and each CTA is a weight stream.
 //
-//   gate/up (MODE 0): items (active group, 128 interleaved gate/up rows = 64 f).
-//       B = x itself ([T, H], every token): the MMA computes all T columns and the epilogue
-//       keeps the columns of the group's tokens, h[row, f] = silu(gate) * up -> bf16.  No
-//       gather of x, no x_sorted.
-//   down (MODE 1):    items (active group, 128 hidden rows).  B = the group's
-//       contiguous h rows [offsets[g], offsets[g+1]) (rows past the group belong to other
-//       groups and are ignored), o[row, hidden] -> bf16.  The gate-weighted combine back to
-//       token order follows as its own small kernel (programmatic dependent launch), so no
-//       CTA here waits on, or sums for, the others.
-// Persistent CTAs (three per SM) walk the items with one TMA ring; accumulators are double
-// buffered.  Warp roles: 0 TMA producer, 1 TMEM allocation + MMA issuer, 2-5 epilogue (TMEM
-// lane quarter warp & 3).  Every wait is bounded (the grouped GEMMs' limit).
+// One persistent launch does both projections.  Its items are all gate/up items, then all down
+// items:
+//   gate/up: (active group, 128 interleaved gate/up rows = 64 f).  B = x itself ([T, H], every
+//       token): the MMA computes all T columns and the epilogue keeps the columns of the group's
+//       tokens, h[row, f] = silu(gate) * up -> bf16.  No gather of x, no x_sorted.  Each epilogue
+//       warp then raises the group's readiness counter (after a fence).
+//   down:    (active group, 128 hidden rows).  B = the group's contiguous h rows
+//       [offsets[g], offsets[g+1]) (rows past the group belong to other groups and are
+//       ignored), o[row, hidden] -> bf16.  Its producer waits (bounded) until every gate/up
+//       item of the group has raised the counter before it loads h; the weights need no wait.
+//       The last down item of a group to pass that wait returns the group's counters to zero.
+// So a group's down items start as soon as its own h is written, while other groups' gate/up
+// items are still streaming, and there is no second launch.  The gate-weighted combine back to
+// token order follows as its own small kernel (programmatic dependent launch).
+// Persistent CTAs (three per SM, never more than fit at once, so every gate/up item a down
+// item waits for is running or done) walk the items with one TMA ring; accumulators are double
+// buffered.  Warp roles: 0 TMA producer, 1 TMEM allocation + MMA issuer, 2-5 epilogue (TMEM lane
+// quarter warp & 3).  Every wait is bounded (the grouped GEMMs' limit).
 #include "gemm_common.cuh"
 #include "decode_common.cuh"
 
@@ -28,12 +34,14 @@ constexpr int kDmThreads = 192;
 
 struct DecMmaParams {
     int T, k, E, S, H, F, G, NB;      // NB = MMA N (T rounded up to 16)
-    int m_blocks;                      // 128-row weight blocks per expert (gate/up: F/64, down: H/128)
+    int gu_blocks;                     // 128-row gate/up blocks per expert (F / 64)
+    int dn_blocks;                     // 128-row down blocks per expert (H / 128)
     const int32_t* offsets;
     const int32_t* sorted_flat;
     const int32_t* sched;              // [1] n_active, active groups at [2 + G + 1 ...]
     uint16_t* h;                       // [R, F]
     uint16_t* o;                       // [R, H]
+    uint32_t* ready;                   // [G] gate/up epilogue warps done per group, [G .. 2G) down items past the wait
     uint32_t* err;
     unsigned long long wait_ns;
 };
@@ -49,11 +57,14 @@ __device__ __forceinline__ int group_token(const DecMmaParams& p, int g, int i) 
     return fl < P ? fl / p.k : fl - P;
 }
 
-struct DmItem { int g, e, rg, r0, n; bool shared; };
-__device__ __forceinline__ DmItem dm_item(const DecMmaParams& p, int it) {
+struct DmItem { int g, e, rg, r0, n; bool shared, down; };
+__device__ __forceinline__ DmItem dm_item(const DecMmaParams& p, int it, int n_gu) {
     DmItem d;
-    const int slot = it / p.m_blocks;
-    d.rg = it - slot * p.m_blocks;
+    d.down = it >= n_gu;
+    const int blocks = d.down ? p.dn_blocks : p.gu_blocks;
+    const int j = d.down ? it - n_gu : it;
+    const int slot = j / blocks;
+    d.rg = j - slot * blocks;
     d.g = p.sched[2 + (p.G + 1) + slot];
     d.r0 = p.offsets[d.g];
     d.n = p.offsets[d.g + 1] - d.r0;
@@ -62,13 +73,20 @@ __device__ __forceinline__ DmItem dm_item(const DecMmaParams& p, int it) {
     return d;
 }
 
-// Persistent: CTA b takes items b, b + gridDim.x, ... of (active group, 128-row block); one TMA
-// ring runs across items and the accumulators are double buffered (2 x 32 TMEM columns), so
-// an item's epilogue (and combine) overlaps the next item's weight stream.
-template <int MODE>
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* a) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+    return v;
+}
+
+// Persistent: CTA b takes items b, b + gridDim.x, ... (gate/up items first); one TMA ring runs
+// across items and the accumulators are double buffered (2 x 32 TMEM columns), so an item's
+// epilogue overlaps the next item's weight stream.
 __global__ void __launch_bounds__(kDmThreads, 3)
-decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sw,
-                  const __grid_constant__ CUtensorMap tm_b, DecMmaParams p) {
+decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w13, const __grid_constant__ CUtensorMap tm_sw13,
+                  const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w2,
+                  const __grid_constant__ CUtensorMap tm_sw2, const __grid_constant__ CUtensorMap tm_h,
+                  DecMmaParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
@@ -81,12 +99,14 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    pdl_wait();          // routing (offsets, schedule) and h come from the preceding kernels
+    pdl_wait();          // routing (offsets, schedule) comes from the preceding kernels
     pdl_trigger();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_items = p.sched[1] * p.m_blocks;
+    const int n_active = p.sched[1];
+    const int n_gu = n_active * p.gu_blocks;
+    const int n_items = n_gu + n_active * p.dn_blocks;
     if (int(blockIdx.x) >= n_items) return;            // uniform across the CTA
-    const int nk = (MODE == 0 ? p.H : p.F) / kBK;
+    const int nk_gu = p.H / kBK, nk_dn = p.F / kBK;
     if (tid == 0) {
         for (int s = 0; s < kDmSt; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4); }
@@ -107,18 +127,38 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint32_t bbytes = uint32_t(p.NB) * kBK * 2;
+            const uint32_t h_target = 4u * uint32_t(p.gu_blocks);     // four epilogue warps per gate/up item
             int step = 0;
             bool ok = true;
             for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-                const DmItem d = dm_item(p, it);
-                const CUtensorMap* ma = d.shared ? &tm_sw : &tm_w;
+                const DmItem d = dm_item(p, it, n_gu);
+                if (d.down) {
+                    // the group's h rows must all be written before the first B load
+                    const unsigned long long t0 = gtimer();
+                    while (ld_acquire_u32(p.ready + d.g) < h_target) {
+                        if (*abort_flag || gtimer() - t0 > p.wait_ns) { ok = false; break; }
+                        __nanosleep(64);
+                    }
+                    if (!ok) break;
+                    asm volatile("fence.proxy.async.global;" ::: "memory");   // h (generic writes) -> TMA reads
+                    // the last down item of the group past this point leaves both counters at zero
+                    if (atomicAdd(p.ready + p.G + d.g, 1u) == uint32_t(p.dn_blocks - 1)) {
+                        p.ready[d.g] = 0u;
+                        p.ready[p.G + d.g] = 0u;
+                    }
+                }
+                const int nk = d.down ? nk_dn : nk_gu;
                 for (int kb = 0; kb < nk; ++kb, ++step) {
                     const int s = step % kDmSt;
                     if (!mbar_wait(&empty[s], (uint32_t(step / kDmSt) & 1u) ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
                     mbar_expect_tx(&full[s], uint32_t(kDmATile) + bbytes);
-                    if (MODE == 0) tma_5d(ma, &full[s], sA + s * kDmATile, kb * kBK, 0, 0, d.rg * 4, d.e);
-                    else tma_3d(ma, &full[s], sA + s * kDmATile, kb * kBK, d.rg * 128, d.e);
-                    tma_2d(&tm_b, &full[s], sB + s * kDmBTile, kb * kBK, MODE == 0 ? 0 : d.r0);
+                    if (!d.down) {
+                        tma_5d(d.shared ? &tm_sw13 : &tm_w13, &full[s], sA + s * kDmATile, kb * kBK, 0, 0, d.rg * 4, d.e);
+                        tma_2d(&tm_x, &full[s], sB + s * kDmBTile, kb * kBK, 0);
+                    } else {
+                        tma_3d(d.shared ? &tm_sw2 : &tm_w2, &full[s], sA + s * kDmATile, kb * kBK, d.rg * 128, d.e);
+                        tma_2d(&tm_h, &full[s], sB + s * kDmBTile, kb * kBK, d.r0);
+                    }
                 }
             }
             if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
@@ -133,6 +173,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+                const int nk = it >= n_gu ? nk_dn : nk_gu;
                 if (!mbar_wait(&tempty[buf], acc_phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
                 tc_fence_after();
                 for (int kb = 0; kb < nk; ++kb, ++step) {
@@ -162,9 +203,9 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
         uint32_t acc_phase = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-            const DmItem d = dm_item(p, it);
+            const DmItem d = dm_item(p, it, n_gu);
             // lane l < n stands for row r0 + l of the group; gate/up: its token
-            const int my_tok = (MODE == 0 && lane < d.n) ? group_token(p, d.g, lane) : -1;
+            const int my_tok = (!d.down && lane < d.n) ? group_token(p, d.g, lane) : -1;
             if (!mbar_wait(&tfull[buf], acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             float v[32];
@@ -174,7 +215,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[buf]);          // the accumulator is free for the item after next
-            if (MODE == 0) {
+            if (!d.down) {
                 // rows 32q..32q+15: gate of f = 64 rg + 16 q + (lane & 15); rows +16: up of the same f
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
@@ -189,6 +230,10 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
                     if (lane < 16 && !(lane & 1))
                         *reinterpret_cast<uint32_t*>(p.h + size_t(r) * p.F + 64 * d.rg + 16 * q + lane) = pair;
                 }
+                // these h columns are written: one count towards the group's down items
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicAdd(p.ready + d.g, 1u);
             } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
@@ -211,21 +256,6 @@ bool decode_mma_eligible(const DecodeArgs& a) {
     return a.wdtype == FT_W_BF16 && !a.eptr && a.T >= 1 && a.T <= 32 && a.H % 128 == 0 && a.F % 64 == 0;
 }
 
-template <typename... KArgs, typename... Args>
-static cudaError_t launch_dependent(void (*kern)(KArgs...), int grid, size_t smem, cudaStream_t st, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kDmThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args...);
-}
-
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st) {
     const int T = a.T, H = a.H, F = a.F, E = a.E, k = a.k, S = a.S;
     const int P = T * k, R = P + (S ? T : 0), G = E + (S ? 1 : 0);
@@ -233,11 +263,14 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st) {
     const int NB = T <= 16 ? 16 : 32;
     DecMmaParams p{};
     p.T = T; p.k = k; p.E = E; p.S = S; p.H = H; p.F = F; p.G = G; p.NB = NB;
+    p.gu_blocks = F / 64;
+    p.dn_blocks = H / 128;
     p.offsets = a.offsets;
     p.sorted_flat = a.sorted_flat;
     p.sched = a.sched;
     p.h = a.h;
     p.o = a.y ? a.o_ws : a.o_sorted;
+    p.ready = a.err + kWsReady;
     p.err = a.err;
     p.wait_ns = gemm_wait_ns();
     CUtensorMap gw{}, gsw{}, gb{}, dw{}, dsw{}, db{};
@@ -265,26 +298,33 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st) {
     }
     if (!S) { gsw = gw; dsw = dw; }
     constexpr size_t smem = dec_mma_smem();
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(decode_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    // Down items wait for gate/up items of other CTAs, so every CTA must be resident at once: the
+    // grid is three per SM (what fits at this shared-memory size: 3 x 62 KB; all of them enter
+    // within a few microseconds, measured) and never more than the items a batch can have.  Were
+    // a CTA ever kept from running by other work, a waiting down item gives up after the bounded
+    // wait and the call reports a timeout.
+    static bool attrs_set = false;
+    if (!attrs_set) {
+        cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e == cudaSuccess)   // the whole unified L1 / shared array as shared memory
+            e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     int(cudaSharedmemCarveoutMaxShared));
         if (e != cudaSuccess) return e;
-        attr = true;
+        attrs_set = true;
     }
-    // persistent grids: up to three CTAs per SM (3-stage rings), never more than the items a batch
-    // can have.  Three shallower rings per SM beat two deeper ones whenever a batch's items fit in
-    // one wave of 3 x SMs (qwen3_a3b T = 8: 64.8 -> 57.0 us) and lose a little when a second wave
-    // runs on few CTAs (T = 32: 100.2 -> 105.5 us)
     const int cap = 3 * num_sms();
-    p.m_blocks = F / 64;
-    cudaError_t e = launch_dependent(decode_mma_kernel<0>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, smem,
-                                     st, gw, gsw, gb, p);
-    if (e != cudaSuccess) return e;
-    p.m_blocks = H / 128;
-    e = launch_dependent(decode_mma_kernel<1>, na_max * p.m_blocks < cap ? na_max * p.m_blocks : cap, smem, st, dw,
-                         dsw, db, p);
+    const int max_items = na_max * (p.gu_blocks + p.dn_blocks);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(max_items < cap ? max_items : cap);
+    cfg.blockDim = dim3(kDmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_mma_kernel, gw, gsw, gb, dw, dsw, db, p);
     if (e != cudaSuccess) return e;
     if (a.y) e = launch_combine_dependent(T, H, k, S, R, a.o_ws, a.inv_pos, a.topk_w, a.y, st);
     if (e != cudaSuccess) return e;

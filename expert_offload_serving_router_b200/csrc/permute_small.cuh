@@ -55,6 +55,7 @@ struct PermOut {
     int32_t* inv_pos;      // [R]
     int32_t* sched;        // [2 + 2*(G+1)]: total tiles (BN rows), n_active, ntile_off[G+1], active[G]
     uint32_t* err;         // device error flag
+    uint32_t* ready;       // [2G] the tensor-core decode's per-group counters, zeroed here (may be null)
 };
 
 // Single-warp counting sort for decode-sized batches (R <= a few hundred pairs): no block
@@ -67,6 +68,8 @@ __device__ inline void warp_permute_small(const int32_t* idx_smem, int T, int k,
     const int R = P + (S ? T : 0);
     const int G = E + (S ? 1 : 0);
     for (int g = lane; g <= G; g += 32) cnt[g] = 0;
+    if (out.ready)
+        for (int g = lane; g < 2 * G; g += 32) out.ready[g] = 0u;
     __syncwarp();
     for (int i = lane; i < R; i += 32) {
         const int g = i < P ? idx_smem[i] : E;
