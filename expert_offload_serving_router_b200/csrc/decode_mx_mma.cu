@@ -10,14 +10,15 @@
 // plane into the same fp32 accumulator.
 //
 //   quant2_kernel:  bf16 rows -> E4M3 planes hi, lo [rows, K] + E8M0 scales [rows, K/32] each.
-//   decode_mx_mma_kernel<MODE>: items (active group, 128 weight rows), persistent CTAs, as the
-//       BF16 tensor-core decode; per 128-deep K step TMA brings 128 rows of codes unpacked to one
-//       byte per element (16U4_ALIGN16B, SW128) and the two activation planes; per item the
-//       epilogue warps lay the weight and activation scales out as tcgen05.cp source atoms (one
-//       per K step and operand, 32 rows x 16 bytes: byte 16 (m % 32) + 4 (m / 32) + j holds row
-//       m's scale of the j-th 32-block of the step) and at the item's start the MMA thread copies
-//       every atom into its own four TMEM columns (lane = row % 32 in every sub-partition, column =
-//       row / 32, byte = block), so no MMA waits on a copy mid-stream.
+//   decode_mx_mma_kernel<MODE>: items (active group, 128 weight rows), a contiguous run of them per
+//       persistent CTA; per 256-deep K stage TMA brings 128 rows of codes unpacked to one byte per
+//       element (16U4_ALIGN16B, SW128) and the two activation planes.  The MMA thread issues only
+//       MMAs and commits.  The epilogue warps lay each item's weight scales (and, when they change,
+//       the activation scales: once per launch for gate/up, once per group for down) out as
+//       tcgen05.cp source atoms (32 rows x 16 bytes per K step: byte 16 (m % 32) + 4 (m / 32) + j
+//       holds row m's scale of the step's j-th 32-block), and a copier warp moves them into
+//       double-buffered TMEM columns (lane = row % 32 in every sub-partition, column = row / 32,
+//       byte = block) an item ahead of the MMAs, ordered by mbarriers both ways.
 // Weights and activation planes are read once; every wait is bounded.
 #include "gemm_common.cuh"
 #include "decode_common.cuh"
@@ -119,13 +120,12 @@ constexpr int kDxBPlane = 32 * 128;               // 4 KB: up to 32 activation r
 constexpr int kDxAStage = 2 * kDxATile;           // 32 KB
 constexpr int kDxBSub = 2 * kDxBPlane;            // 8 KB: a sub-tile's B operand, hi rows then lo rows
 constexpr int kDxBStage = 2 * kDxBSub;            // 16 KB
-constexpr int kDxThreads = 192;
+constexpr int kDxThreads = 224;                   // producer, MMA issuer, four epilogue / atom warps, scale copier
 constexpr int kDxMaxK = 4096;                     // largest contraction (scale atoms sized for it)
 constexpr int kDxSteps = kDxMaxK / 128;           // K steps per item at most
-constexpr int kDxAtomBuf = 2 * kDxSteps * 512;    // one item's weight and activation scale atoms of every K step
-constexpr int kDxTmemCols = 512;                  // 2 x 64 accumulator columns + every step's two scale atoms
+constexpr int kDxAtomBuf = 2 * kDxSteps * 512;    // 32 KB of scale atoms: weight buffers and activation atoms
+constexpr int kDxTmemCols = 512;
 constexpr int kDxAccCols = 64;                    // accumulator columns per buffer: N = 2 NB (hi rows, then lo rows)
-constexpr int kDxColSf = 128;                     // kind k (weights, activations), step c: columns 128 + 128 k + 4 c
 
 __host__ __device__ constexpr size_t dec_mx_smem() {
     return 1024 + size_t(kDxSt) * (kDxAStage + kDxBStage) + size_t(kDxAtomBuf) + 512;
@@ -177,6 +177,34 @@ __device__ __forceinline__ bool wait_fast(uint64_t* b, uint32_t parity, volatile
     return mbar_try(b, parity) || mbar_wait(b, parity, abort, limit);
 }
 
+// Where an item's scale factors live.  TMEM columns: [0, 128) the two accumulator buffers, then
+// nact activation-scale buffers and two weight-scale buffers of 4 columns per 128-deep K step
+// (step c of a buffer at column base + 4 c).  Shared memory (the 32 KB atom area): gate/up --
+// weight atom buffers 0 and 1 at 0 and nk x 512 bytes, the activation atoms (built once) first
+// in buffer 1's place; down -- the activation atoms of the current group at 0, then nwb weight
+// atom buffers.
+struct DxScaleLayout {
+    int nk, nact, nwb;
+    __device__ int act_col(int run) const { return 128 + 4 * nk * (run % nact); }
+    __device__ int w_col(int j) const { return 128 + 4 * nk * (nact + (j & 1)); }
+};
+template <int MODE>
+__device__ __forceinline__ DxScaleLayout dx_layout(int nk) {
+    DxScaleLayout L;
+    L.nk = nk;
+    L.nact = MODE == 0 ? 1 : (128 + 16 * nk <= kDxTmemCols ? 2 : 1);
+    const int atom = nk * 512;
+    L.nwb = MODE == 0 ? 2 : min(2, (kDxAtomBuf - atom) / atom);
+    return L;
+}
+
+// The activation operand an item reads: gate/up -- x, the same for every item; down -- its group's
+// rows of h.  A change of key means new activation scales.
+template <int MODE>
+__device__ __forceinline__ int dx_act_key(const DecMxParams& p, int it) {
+    return MODE == 0 ? 0 : p.sched[2 + (p.G + 1) + it / p.m_blocks];
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kDxThreads, 1)
 decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_bh,
@@ -185,29 +213,42 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + kDxSt * kDxAStage;                      // [stage][sub-tile] hi rows 0..NB-1, lo rows NB..2NB-1
-    uint8_t* sAtoms = sB + kDxSt * kDxBStage;                 // [kind][128-deep K step] 512-byte atoms of one item
+    uint8_t* sAtoms = sB + kDxSt * kDxBStage;                 // scale atoms (DxScaleLayout)
     uint64_t* full = reinterpret_cast<uint64_t*>(sAtoms + kDxAtomBuf);
     uint64_t* empty = full + kDxSt;
     uint64_t* tfull = empty + kDxSt;
     uint64_t* tempty = tfull + 2;
-    uint64_t* sf_full = tempty + 2;       // atoms of an item laid out
-    uint64_t* sf_free = sf_full + 1;      // atoms of an item copied to TMEM
-    uint64_t* mma_done = sf_free + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* atoms_full = tempty + 2;    // [weight atom buffer] an item's atoms laid out
+    uint64_t* atoms_free = atoms_full + 2;// [weight atom buffer] an item's atoms copied to TMEM
+    uint64_t* sf_ready = atoms_free + 2;  // [TMEM weight-scale buffer] an item's scales in TMEM
+    uint64_t* mma_done = sf_ready + 2;
+    uint64_t* cp_done = mma_done + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     pdl_wait();          // routing, the activation planes and h come from the preceding kernels
     pdl_trigger();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_items = p.sched[1] * p.m_blocks;
-    if (int(blockIdx.x) >= n_items) return;
+    // a contiguous run of items per CTA: consecutive items mostly share their group, so down items
+    // reuse the activation scales already in TMEM
+    const int i0 = int((long long)blockIdx.x * n_items / gridDim.x);
+    const int i1 = int((long long)(blockIdx.x + 1) * n_items / gridDim.x);
+    const int n_my = i1 - i0;
+    if (n_my <= 0) return;
     const int nk = p.K / 128;                // 128-deep K steps (scale atoms); stages cover two
+    const DxScaleLayout SL = dx_layout<MODE>(nk);
     if (tid == 0) {
         for (int s = 0; s < kDxSt; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4); }
-        mbar_init(sf_full, 4);
-        mbar_init(sf_free, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+            mbar_init(&atoms_full[b], 4);
+            mbar_init(&atoms_free[b], 1);
+            mbar_init(&sf_ready[b], 1);
+        }
         mbar_init(mma_done, 1);
+        mbar_init(cp_done, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -231,7 +272,7 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
             int step = 0, s = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            for (int it = i0; it < i1 && ok; ++it) {
                 const int slot = it / p.m_blocks, rg = it - slot * p.m_blocks;
                 const int g = p.sched[2 + (p.G + 1) + slot];
                 const int brow = MODE == 0 ? 0 : p.offsets[g];
@@ -258,31 +299,30 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                 mbar_wait(&full[st % kDxSt], uint32_t(st / kDxSt) & 1u, nullptr);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer: an item's scales to TMEM, then one MMA per K block
+        // ------------------------------------------------ MMA issuer: one MMA per 32-deep K block
         // At decode sizes this thread is the critical path (an MMA with N <= 64 occupies the tensor
-        // pipe for only ~56 cycles), so every operand but the stage is computed once per launch
-        // and the descriptors advance by adding (start address >> 4) offsets.
+        // pipe for only ~56 cycles), so it issues nothing but MMAs and commits: the scale factors
+        // reach TMEM through the copier warp, every descriptor is computed once per launch and the
+        // descriptors advance by adding (start address >> 4) offsets.
         if (lane == 0) {
             uint32_t idm[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) idm[j] = idesc_mx(2 * p.NB, uint32_t(j), uint32_t(j));
-            const uint64_t ad0 = sdesc_sw128(su32(sA)), bd0 = sdesc_sw128(su32(sB)), cp0 = atom_desc(su32(sAtoms));
-            int stage = 0, buf = 0, item = 0;
-            uint32_t phase = 0, acc_phase = 0;
+            const uint64_t ad0 = sdesc_sw128(su32(sA)), bd0 = sdesc_sw128(su32(sB));
+            int stage = 0, run = -1, prev_key = -1;
+            uint32_t phase = 0;
             bool ok = true;
-            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++item) {
-                if (!wait_fast(sf_full, uint32_t(item) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
-                if (!wait_fast(&tempty[buf], acc_phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+            for (int j = 0; j < n_my && ok; ++j) {
+                const int key = dx_act_key<MODE>(p, i0 + j);
+                if (j == 0 || key != prev_key) ++run;
+                prev_key = key;
+                const int buf = j & 1;
+                const uint32_t par = uint32_t(j >> 1) & 1u;
+                if (!wait_fast(&sf_ready[buf], par, abort_flag, p.wait_ns)) { ok = false; break; }
+                if (!wait_fast(&tempty[buf], par ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
                 tc_fence_after();
-                // every step's scales to their own TMEM columns first, so the MMAs below never wait
-                // on a copy (they execute after the copies: same issuing thread, issue order)
-                for (int c = 0; c < nk; ++c) {
-                    tmem_cp_desc(tmem + uint32_t(kDxColSf + 4 * c), cp0 + uint64_t(32 * c));
-                    tmem_cp_desc(tmem + uint32_t(kDxColSf + 128 + 4 * c), cp0 + uint64_t(32 * (kDxSteps + c)));
-                }
-                umma_commit(sf_free);          // the atoms may be rebuilt for the next item once copied
                 const uint32_t dacc = tmem + uint32_t(kDxAccCols * buf);
-                uint32_t sfa = tmem + uint32_t(kDxColSf), sfb = tmem + uint32_t(kDxColSf + 128);
+                uint32_t sfa = tmem + uint32_t(SL.w_col(j)), sfb = tmem + uint32_t(SL.act_col(run));
                 for (int kb = 0; kb < nk / 2; ++kb) {
                     // the stage's operands were all written by TMA (async proxy): its barrier's
                     // completion orders them before these MMAs, no thread-sync fence needed
@@ -304,26 +344,62 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                 }
                 if (!ok) break;
                 umma_commit(&tfull[buf]);
-                if (++buf == 2) { buf = 0; acc_phase ^= 1; }
             }
             if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
             umma_commit(mma_done);
             mbar_wait(mma_done, 0, nullptr);
         }
+    } else if (warp == 6) {
+        // ------------------------------------------------ scale copier: atoms -> TMEM, ahead of the MMAs
+        // Item j's weight scales go to TMEM buffer j & 1 once item j - 2 (the buffer's last reader)
+        // has completed; new activation scales go to their buffer once no issued item still reads it.
+        if (lane == 0) {
+            const uint64_t cp0 = atom_desc(su32(sAtoms));
+            const int atom_steps = nk;                 // one 512-byte atom per step: descriptor + 32 each
+            int run = -1, prev_key = -1;
+            bool ok = true;
+            for (int j = 0; j < n_my; ++j) {
+                const int key = dx_act_key<MODE>(p, i0 + j);
+                const bool act_new = j == 0 || key != prev_key;
+                if (act_new) ++run;
+                prev_key = key;
+                const int wb = j % SL.nwb;
+                if (!wait_fast(&atoms_full[wb], uint32_t(j / SL.nwb) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                if (j >= 2 && !wait_fast(&tfull[j & 1], uint32_t((j - 2) >> 1) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                if (act_new && SL.nact == 1 && j >= 1 &&
+                    !wait_fast(&tfull[(j - 1) & 1], uint32_t((j - 1) >> 1) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                tc_fence_after();
+                if (act_new) {
+                    const uint64_t a0 = cp0 + uint64_t(MODE == 0 ? 32 * atom_steps : 0);
+                    for (int c = 0; c < nk; ++c) tmem_cp_desc(tmem + uint32_t(SL.act_col(run) + 4 * c), a0 + uint64_t(32 * c));
+                }
+                const uint64_t w0 = cp0 + uint64_t(32 * atom_steps * (MODE == 0 ? wb : 1 + wb));
+                for (int c = 0; c < nk; ++c) tmem_cp_desc(tmem + uint32_t(SL.w_col(j) + 4 * c), w0 + uint64_t(32 * c));
+                umma_commit(&sf_ready[j & 1]);
+                umma_commit(&atoms_free[wb]);
+            }
+            if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+            umma_commit(cp_done);
+            mbar_wait(cp_done, 0, nullptr);
+        }
     } else {
         // ------------------------------------------------ scale atoms, then the epilogue
-        // Item i+1's atoms are laid out once item i's reached TMEM (the MMA thread copies them at
-        // the item's start), before item i's epilogue, so they are ready when item i ends.  Atom
-        // of K step c: byte 16 (m % 32) + 4 (m / 32) + j = scale of 32-block j of row m (weights:
-        // the A-tile row; activations: B row m < 2 NB -- the hi plane's rows, then the lo plane's).
+        // Item j + 1's atoms are laid out as soon as its atom buffer is free, before item j's
+        // epilogue.  Atom of K step c: byte 16 (m % 32) + 4 (m / 32) + jb = scale of 32-block jb of
+        // row m (weights: the A-tile row; activations: B row m < 2 NB -- the hi plane's rows, then
+        // the lo plane's).
         const int q = warp & 3, et = tid - 64;   // et: 0..127
         const int nsb = p.K / 32;                // scale bytes per row
         const size_t rows_e = MODE == 0 ? size_t(2) * p.F : size_t(p.H);
-        auto build_atoms = [&](int it2) {
-            uint8_t* atoms = sAtoms;
+        const int atom = nk * 512;
+        auto build_atoms = [&](int j, bool act_new) {
+            const int it2 = i0 + j;
             const int slot2 = it2 / p.m_blocks, rg2 = it2 - slot2 * p.m_blocks;
             const int g2 = p.sched[2 + (p.G + 1) + slot2];
             const int r02 = p.offsets[g2], n2 = p.offsets[g2 + 1] - r02;
+            const int wb = j % SL.nwb;
+            uint8_t* wdst = sAtoms + (MODE == 0 ? wb : 1 + wb) * atom;
+            uint8_t* adst = sAtoms + (MODE == 0 ? atom : 0);
             int wrow;     // weight row of A-tile row et (gate/up: blocks of 16 gate rows then the 16 up rows)
             if (MODE == 0) {
                 const int i = et >> 5, jj = et & 31, f = rg2 * 64 + 16 * i + (jj & 15);
@@ -344,9 +420,9 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                 const uint32_t w4[4] = {wv[c4].x, wv[c4].y, wv[c4].z, wv[c4].w};
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc)
-                    *reinterpret_cast<uint32_t*>(atoms + (4 * c4 + cc) * 512 + 16 * (et & 31) + 4 * (et >> 5)) = w4[cc];
+                    *reinterpret_cast<uint32_t*>(wdst + (4 * c4 + cc) * 512 + 16 * (et & 31) + 4 * (et >> 5)) = w4[cc];
             }
-            if (et < 64 && (et & 31) < p.NB) {
+            if (act_new && et < 64 && (et & 31) < p.NB) {
                 const int pl = et >> 5, nrow = et & 31, m = pl * p.NB + nrow;   // B row of the merged operand
                 const uint8_t* bsrc = pl ? p.bsc_lo : p.bsc_hi;
                 const int brow = MODE == 0 ? nrow : r02 + nrow;
@@ -361,30 +437,36 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                     const uint32_t b4[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc)
-                        *reinterpret_cast<uint32_t*>(atoms + (kDxSteps + 4 * c4 + cc) * 512 + 16 * (m & 31) + 4 * (m >> 5)) =
-                            b4[cc];
+                        *reinterpret_cast<uint32_t*>(adst + (4 * c4 + cc) * 512 + 16 * (m & 31) + 4 * (m >> 5)) = b4[cc];
                 }
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
-            if (lane == 0) mbar_arrive(sf_full);
+            if (lane == 0) mbar_arrive(&atoms_full[wb]);
         };
-        int buf = 0, item = 0;
-        uint32_t acc_phase = 0;
+        // the wait for item x's atoms to have been copied (its buffer's phase x / nwb)
+        auto copied = [&](int x) {
+            return wait_fast(&atoms_free[x % SL.nwb], uint32_t(x / SL.nwb) & 1u, abort_flag, p.wait_ns);
+        };
         bool ok = true;
-        build_atoms(blockIdx.x);
-        for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++item) {
+        build_atoms(0, true);
+        for (int j = 0; j < n_my; ++j) {
+            const int it = i0 + j;
             const int slot = it / p.m_blocks, rg = it - slot * p.m_blocks;
             const int g = p.sched[2 + (p.G + 1) + slot];
             const int r0 = p.offsets[g], n = p.offsets[g + 1] - r0;
-            if (it + int(gridDim.x) < n_items) {
-                // the buffer is free once this item's atoms reached TMEM (at the item's start)
-                if (!mbar_wait(sf_free, uint32_t(item) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
-                build_atoms(it + gridDim.x);
+            if (j + 1 < n_my) {
+                const bool act_new = MODE == 1 && dx_act_key<MODE>(p, it + 1) != dx_act_key<MODE>(p, it);
+                // the weight buffer's previous item, the activation atoms' last copy (item j), and
+                // for gate/up item 1 the activation atoms that shared buffer 1 (copied with item 0)
+                if (j + 1 >= SL.nwb && !copied(j + 1 - SL.nwb)) { ok = false; break; }
+                if ((act_new || (MODE == 0 && j == 0)) && !copied(j)) { ok = false; break; }
+                build_atoms(j + 1, act_new);
             }
             // lane l < n stands for row r0 + l of the group; gate/up: its token
             const int my_tok = (MODE == 0 && lane < n) ? group_token_of(p.sorted_flat[r0 + lane], P, p.k) : -1;
-            if (!mbar_wait(&tfull[buf], acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
+            const int buf = j & 1;
+            if (!mbar_wait(&tfull[buf], uint32_t(j >> 1) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             float v[32];
             // column c of the hi rows plus column NB + c of the lo rows
@@ -425,7 +507,6 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                 for (int i = 0; i < 32; ++i)
                     if (i < n) p.o[size_t(r0 + i) * p.H + 128 * rg + 32 * q + lane] = f2bf(v[i]);
             }
-            if (++buf == 2) { buf = 0; acc_phase ^= 1; }
         }
         if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
     }

@@ -236,7 +236,11 @@ def block_scaled_decode():
 @pytest.mark.parametrize("name,T,kw", [("dsv4_flash", 1, {}), ("dsv4_flash", 8, {}), ("dsv4_flash", 20, {}),
                                        ("dsv4_flash", 32, {}),
                                        ("custom", 13, dict(hidden=1024, ffn=512, num_experts=16, top_k=4,
-                                                           num_shared=0, wdtype=inputs.WDTYPE_MXFP4, config_id=83))])
+                                                           num_shared=0, wdtype=inputs.WDTYPE_MXFP4, config_id=83)),
+                                       # FFN 4096: one activation-scale buffer in TMEM for down, a
+                                       # single weight-atom buffer, and runs of items that cross groups
+                                       ("custom", 12, dict(hidden=1024, ffn=4096, num_experts=24, top_k=4,
+                                                           num_shared=0, wdtype=inputs.WDTYPE_MXFP4, config_id=91))])
 def test_block_scaled_mxfp4_decode_matches_oracle(block_scaled_decode, name, T, kw):
     """MXFP4 decode on tcgen05.mma.kind::mxf8f6f4.block_scale (E2M1 weights with their E8M0
     scales read as stored, activations as two E4M3 planes): every token checked against the
