@@ -7,6 +7,13 @@
 
 namespace ftmoe {
 
+// gpu-scope acquire load of a cross-CTA counter (the tensor-core decodes' per-group readiness)
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* a) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+    return v;
+}
+
 struct EW { const uint8_t *w13, *w13s, *w2, *w2s; };
 
 // Programmatic dependent launch: a kernel launched with the programmatic-serialization

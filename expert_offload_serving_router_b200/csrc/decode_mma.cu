@@ -73,12 +73,6 @@ __device__ __forceinline__ DmItem dm_item(const DecMmaParams& p, int it, int n_g
     return d;
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* a) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
-    return v;
-}
-
 // Persistent: CTA b takes items b, b + gridDim.x, ... (gate/up items first); one TMA ring runs
 // across items and the accumulators are double buffered (2 x 32 TMEM columns), so an item's
 // epilogue overlaps the next item's weight stream.

@@ -19,6 +19,9 @@
 //       holds row m's scale of the step's j-th 32-block), and a copier warp moves them into
 //       double-buffered TMEM columns (lane = row % 32 in every sub-partition, column = row / 32,
 //       byte = block) an item ahead of the MMAs, ordered by mbarriers both ways.
+//   decode_mx_fused_kernel: batches of up to 16 tokens with FFN <= 2048 -- gate/up and down items
+//       in one persistent launch; the gate/up epilogue writes h as its two planes and raises a
+//       per-group counter that down items wait for; the scale atoms get four warps of their own.
 // Weights and activation planes are read once; every wait is bounded.
 #include "gemm_common.cuh"
 #include "decode_common.cuh"
@@ -175,6 +178,14 @@ __device__ __forceinline__ void tmem_cp_desc(uint32_t taddr, uint64_t d) {
 // steady state costs one try_wait)
 __device__ __forceinline__ bool wait_fast(uint64_t* b, uint32_t parity, volatile int* abort, unsigned long long limit) {
     return mbar_try(b, parity) || mbar_wait(b, parity, abort, limit);
+}
+// a bounded mbarrier wait taken by lane 0 for the whole warp (warp-uniform outcome)
+__device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, volatile int* abort, unsigned long long limit) {
+    int r = 0;
+    if ((threadIdx.x & 31) == 0) r = wait_fast(b, parity, abort, limit) ? 1 : 0;
+    r = __shfl_sync(0xffffffffu, r, 0);
+    __syncwarp();
+    return r != 0;
 }
 
 // Where an item's scale factors live.  TMEM columns: [0, 128) the two accumulator buffers, then
@@ -446,7 +457,7 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
         };
         // the wait for item x's atoms to have been copied (its buffer's phase x / nwb)
         auto copied = [&](int x) {
-            return wait_fast(&atoms_free[x % SL.nwb], uint32_t(x / SL.nwb) & 1u, abort_flag, p.wait_ns);
+            return warp_wait(&atoms_free[x % SL.nwb], uint32_t(x / SL.nwb) & 1u, abort_flag, p.wait_ns);
         };
         bool ok = true;
         build_atoms(0, true);
@@ -466,7 +477,7 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
             // lane l < n stands for row r0 + l of the group; gate/up: its token
             const int my_tok = (MODE == 0 && lane < n) ? group_token_of(p.sorted_flat[r0 + lane], P, p.k) : -1;
             const int buf = j & 1;
-            if (!mbar_wait(&tfull[buf], uint32_t(j >> 1) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+            if (!warp_wait(&tfull[buf], uint32_t(j >> 1) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             float v[32];
             // column c of the hi rows plus column NB + c of the lo rows
@@ -506,6 +517,459 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     if (i < n) p.o[size_t(r0 + i) * p.H + 128 * rg + 32 * q + lane] = f2bf(v[i]);
+            }
+        }
+        if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kDxTmemCols));
+    }
+}
+
+
+// ------------------------------------------------------------------ gate/up and down in one launch
+// For FFN widths up to 2048 both GEMVs run as one persistent launch: CTA b takes items b,
+// b + gridDim.x, ... of the list [gate/up items | down items].  The gate/up epilogue writes h
+// straight as the two E4M3 planes with their E8M0 scales (the steps of quant2_kernel on the
+// bf16-rounded h; the two warps that hold a 32-column block exchange their partial maxima through
+// shared memory) and then raises its group's counter.  A down item's producer waits for all the
+// group's gate/up epilogues before its TMA reads h, and the warps that lay out its activation
+// scales wait too before they load them.  Each down item is read twice (producer, copier once its
+// atoms exist): the last of the 2 x dn_blocks reads of a group leaves both counters at zero.
+constexpr int kFxMaxKDn = 2048;            // largest down contraction (F) of the fused plan
+// Batches of up to 16 tokens: the one launch saves the second launch's ramp and fills the
+// gate/up tail (dsv4_flash T = 4 / 8: 93 -> 87 / 153 -> 146 us); at 32 tokens the strided down
+// items (new activation scales for every one) and two-row gate/up epilogues cost what it saves.
+constexpr int kFxMaxT = 16;
+constexpr int kFxWBuf = kDxAtomBuf / 2;    // 16 KB weight-atom buffers at 0 and 16 KB
+constexpr int kFxDnAct = kFxWBuf / 2;      // down items' activation atoms at 8 KB (<= 16 steps)
+constexpr int kFxThreads = 352;            // producer, MMA issuer, four epilogue warps, copier, four atom builders
+
+__host__ __device__ constexpr size_t dec_mx_fused_smem() { return dec_mx_smem() + 1024; }
+
+struct DecMxFusedParams {
+    int T, k, E, H, F, G, NB, gu_blocks, dn_blocks;
+    const int32_t* offsets;
+    const int32_t* sorted_flat;
+    const int32_t* sched;
+    const uint8_t* wsc13;        // gate/up weight scales [E, 2F, H/32]
+    const uint8_t* wsc2;         // down weight scales [E, H, F/32]
+    const uint8_t* xsh;          // x plane scales [32, H/32]
+    const uint8_t* xsl;
+    uint8_t* hh;                 // h planes [R, F] and their scales [R, F/32]
+    uint8_t* hl;
+    uint8_t* hsh;
+    uint8_t* hsl;
+    uint16_t* o;
+    uint32_t* ready;             // [2G]: gate/up epilogue warps done per group, then down reads
+    uint32_t* err;
+    unsigned long long wait_ns;
+};
+
+struct FxItem {
+    int g, rg, r0, n;
+    bool down;
+};
+__device__ __forceinline__ FxItem fx_item(const DecMxFusedParams& p, int it, int n_gu) {
+    FxItem d;
+    d.down = it >= n_gu;
+    const int li = d.down ? it - n_gu : it;
+    const int nb = d.down ? p.dn_blocks : p.gu_blocks;
+    const int slot = li / nb;
+    d.rg = li - slot * nb;
+    d.g = p.sched[2 + (p.G + 1) + slot];
+    d.r0 = p.offsets[d.g];
+    d.n = p.offsets[d.g + 1] - d.r0;
+    return d;
+}
+__device__ __forceinline__ int fx_act_key(const FxItem& d) { return d.down ? d.g : -1; }
+// one of a down item's two reads of its group's counter is done
+__device__ __forceinline__ void fx_read_done(const DecMxFusedParams& p, int g) {
+    if (atomicAdd(p.ready + p.G + g, 1u) == uint32_t(2 * p.dn_blocks - 1)) {
+        p.ready[g] = 0u;
+        p.ready[p.G + g] = 0u;
+    }
+}
+// one thread's bounded wait for all the group's gate/up epilogue warps
+__device__ __forceinline__ bool fx_group_wait(const DecMxFusedParams& p, int g, volatile int* abort_flag) {
+    const uint32_t target = 4u * uint32_t(p.gu_blocks);     // four epilogue warps per gate/up item
+    const unsigned long long t0 = gtimer();
+    while (ld_acquire_u32(p.ready + g) < target) {
+        if (*abort_flag || gtimer() - t0 > p.wait_ns) return false;
+        __nanosleep(64);
+    }
+    return true;
+}
+// the same wait by a whole warp (every lane acquires; the outcome is warp-uniform)
+__device__ __forceinline__ bool fx_group_wait_warp(const DecMxFusedParams& p, int g, volatile int* abort_flag) {
+    const uint32_t target = 4u * uint32_t(p.gu_blocks);
+    const unsigned long long t0 = gtimer();
+    for (;;) {
+        if (__all_sync(0xffffffffu, ld_acquire_u32(p.ready + g) >= target)) return true;
+        if (__any_sync(0xffffffffu, *abort_flag != 0 || gtimer() - t0 > p.wait_ns)) return false;
+        __nanosleep(64);
+    }
+}
+__device__ __forceinline__ float warp_max(float m) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    return m;
+}
+
+__global__ void __launch_bounds__(kFxThreads, 1)
+decode_mx_fused_kernel(const __grid_constant__ CUtensorMap tm_w13, const __grid_constant__ CUtensorMap tm_w2,
+                       const __grid_constant__ CUtensorMap tm_xh, const __grid_constant__ CUtensorMap tm_xl,
+                       const __grid_constant__ CUtensorMap tm_hh, const __grid_constant__ CUtensorMap tm_hl,
+                       DecMxFusedParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + kDxSt * kDxAStage;
+    uint8_t* sAtoms = sB + kDxSt * kDxBStage;  // weight atoms [0, 16K) and [16K, 32K); x atoms at 16K; down activation atoms at 8K
+    uint64_t* full = reinterpret_cast<uint64_t*>(sAtoms + kDxAtomBuf);
+    uint64_t* empty = full + kDxSt;
+    uint64_t* tfull = empty + kDxSt;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* atoms_full = tempty + 2;
+    uint64_t* atoms_free = atoms_full + 2;
+    uint64_t* sf_ready = atoms_free + 2;
+    uint64_t* mma_done = sf_ready + 2;
+    uint64_t* cp_done = mma_done + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    uint64_t* pair_bar = reinterpret_cast<uint64_t*>(tmem_slot + 2);     // [pair of epilogue warps]
+    float* xch = reinterpret_cast<float*>(sAtoms + kDxAtomBuf + 512);   // [pair][round][half][32 rows] partial maxima
+
+    pdl_wait();          // routing and the x planes come from the preceding kernels
+    pdl_trigger();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_gu = p.sched[1] * p.gu_blocks;
+    const int n_items = n_gu + p.sched[1] * p.dn_blocks;
+    if (int(blockIdx.x) >= n_items) return;
+    const int n_my = (n_items - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x);
+    const int nk_gu = p.H / 128, nk_dn = p.F / 128, nk_max = max(nk_gu, nk_dn);
+    // TMEM: accumulators [0, 128); x scales at 128 or the two down activation-scale buffers at
+    // 128 + 4 nk_dn a; weight-scale buffers at wbase + 4 nk_max b
+    const int wbase = 128 + 4 * max(nk_gu, 2 * nk_dn);
+    if (tid == 0) {
+        for (int s = 0; s < kDxSt; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+            mbar_init(&atoms_full[b], 4);
+            mbar_init(&atoms_free[b], 1);
+            mbar_init(&sf_ready[b], 1);
+        }
+        mbar_init(mma_done, 1);
+        mbar_init(cp_done, 1);
+        mbar_init(&pair_bar[0], 2);
+        mbar_init(&pair_bar[1], 2);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                     "r"(kDxTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int P = p.T * p.k;
+    auto item = [&](int j) { return fx_item(p, int(blockIdx.x) + j * int(gridDim.x), n_gu); };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer: codes + both activation planes
+        if (lane == 0) {
+            const uint32_t bytes = 2u * (uint32_t(kDxATile) / 2u + 2u * uint32_t(p.NB) * 128u);
+            int s = 0;
+            long step = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int j = 0; j < n_my && ok; ++j) {
+                const FxItem d = item(j);
+                if (d.down) {
+                    // every h row of the group written before the first B load
+                    if (!fx_group_wait(p, d.g, abort_flag)) { ok = false; break; }
+                    asm volatile("fence.proxy.async.global;" ::: "memory");   // h (generic writes) -> TMA reads
+                    fx_read_done(p, d.g);
+                }
+                const int nk = d.down ? nk_dn : nk_gu;
+                const int brow = d.down ? d.r0 : 0;
+                for (int kb = 0; kb < nk / 2; ++kb, ++step) {
+                    if (!wait_fast(&empty[s], phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                    mbar_expect_tx(&full[s], bytes);
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int k0 = (2 * kb + u) * 128;
+                        uint8_t* a = sA + s * kDxAStage + u * kDxATile;
+                        if (d.down) tma_3d(&tm_w2, &full[s], a, k0, d.rg * 128, d.g);
+                        else tma_5d(&tm_w13, &full[s], a, k0, 0, 0, d.rg * 4, d.g);
+                        uint8_t* b = sB + s * kDxBStage + u * kDxBSub;
+                        tma_2d(d.down ? &tm_hh : &tm_xh, &full[s], b, k0, brow);
+                        tma_2d(d.down ? &tm_hl : &tm_xl, &full[s], b + p.NB * 128, k0, brow);
+                    }
+                    if (++s == kDxSt) { s = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+            for (long st = step - kDxSt > 0 ? step - kDxSt : 0; st < step; ++st)
+                mbar_wait(&full[st % kDxSt], uint32_t(st / kDxSt) & 1u, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer: MMAs and commits only
+        if (lane == 0) {
+            uint32_t idm[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) idm[j] = idesc_mx(2 * p.NB, uint32_t(j), uint32_t(j));
+            const uint64_t ad0 = sdesc_sw128(su32(sA)), bd0 = sdesc_sw128(su32(sB));
+            int stage = 0, drun = -1, prev_key = -2;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int j = 0; j < n_my && ok; ++j) {
+                const FxItem d = item(j);
+                const int key = fx_act_key(d);
+                if (d.down && key != prev_key) ++drun;
+                prev_key = key;
+                const int buf = j & 1;
+                const uint32_t par = uint32_t(j >> 1) & 1u;
+                if (!wait_fast(&sf_ready[buf], par, abort_flag, p.wait_ns)) { ok = false; break; }
+                if (!wait_fast(&tempty[buf], par ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t dacc = tmem + uint32_t(kDxAccCols * buf);
+                uint32_t sfa = tmem + uint32_t(wbase + 4 * nk_max * buf);
+                uint32_t sfb = tmem + uint32_t(d.down ? 128 + 4 * nk_dn * (drun & 1) : 128);
+                const int nk = d.down ? nk_dn : nk_gu;
+                for (int kb = 0; kb < nk / 2; ++kb) {
+                    if (!wait_fast(&full[stage], phase, abort_flag, p.wait_ns)) { ok = false; break; }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const uint64_t ad = ad0 + uint64_t((stage * kDxAStage + u * kDxATile) >> 4);
+                        const uint64_t bd = bd0 + uint64_t((stage * kDxBStage + u * kDxBSub) >> 4);
+                        umma_mx(dacc, ad, bd, idm[0], sfa, sfb, (kb | u) != 0);
+                        umma_mx(dacc, ad + 2, bd + 2, idm[1], sfa + (1u << 30), sfb + (1u << 30), 1u);
+                        umma_mx(dacc, ad + 4, bd + 4, idm[2], sfa + (2u << 30), sfb + (2u << 30), 1u);
+                        umma_mx(dacc, ad + 6, bd + 6, idm[3], sfa + (3u << 30), sfb + (3u << 30), 1u);
+                        sfa += 4u;
+                        sfb += 4u;
+                    }
+                    umma_commit(&empty[stage]);
+                    if (++stage == kDxSt) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[buf]);
+            }
+            if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+            umma_commit(mma_done);
+            mbar_wait(mma_done, 0, nullptr);
+        }
+    } else if (warp == 6) {
+        // ------------------------------------------------ scale copier
+        // Weight scales to buffer j & 1 once item j - 2 completed; activation scales when they
+        // change -- the down buffers overlap the x scales, so the first down item waits for the
+        // item before it.
+        if (lane == 0) {
+            const uint64_t cp0 = atom_desc(su32(sAtoms));
+            int drun = -1, prev_key = -2;
+            bool ok = true;
+            for (int j = 0; j < n_my; ++j) {
+                const FxItem d = item(j);
+                const int key = fx_act_key(d);
+                const bool act_new = key != prev_key;
+                const bool first_down = d.down && j > 0 && prev_key == -1;
+                if (d.down && act_new) ++drun;
+                prev_key = key;
+                const int wb = j & 1;
+                if (!wait_fast(&atoms_full[wb], uint32_t(j >> 1) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                if (d.down) fx_read_done(p, d.g);    // the item's activation scales (if any) are loaded
+                if (j >= 2 && !wait_fast(&tfull[wb], uint32_t((j - 2) >> 1) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+                if (first_down && !wait_fast(&tfull[(j - 1) & 1], uint32_t((j - 1) >> 1) & 1u, abort_flag, p.wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int nk = d.down ? nk_dn : nk_gu;
+                if (act_new) {
+                    const uint32_t acol = d.down ? uint32_t(128 + 4 * nk_dn * (drun & 1)) : 128u;
+                    const uint64_t a0 = cp0 + uint64_t((d.down ? kFxDnAct : kFxWBuf) >> 4);
+                    for (int c = 0; c < nk; ++c) tmem_cp_desc(tmem + acol + uint32_t(4 * c), a0 + uint64_t(32 * c));
+                }
+                const uint64_t w0 = cp0 + uint64_t((wb * kFxWBuf) >> 4);
+                const uint32_t wcol = uint32_t(wbase + 4 * nk_max * wb);
+                for (int c = 0; c < nk; ++c) tmem_cp_desc(tmem + wcol + uint32_t(4 * c), w0 + uint64_t(32 * c));
+                umma_commit(&sf_ready[wb]);
+                umma_commit(&atoms_free[wb]);
+            }
+            if (!ok) { *abort_flag = 1; atomicExch(p.err, kDevErrTimeout); }
+            umma_commit(cp_done);
+            mbar_wait(cp_done, 0, nullptr);
+        }
+    } else if (warp >= 7) {
+        // ------------------------------------------------ scale atoms (thread et: A-tile row et)
+        // Item j's atoms go to buffer j & 1 once item j - 2's were copied (item 1: once item 0's,
+        // whose x atoms sat in buffer 1; new down activation atoms: once item j - 1's).  These
+        // warps run ahead of the epilogues, so a down item's wait for its group's h never holds
+        // up the gate/up epilogues that produce it.
+        const int et = tid - 224;                // 0..127
+        const bool act_warp = et < 64;           // these load activation scales
+        auto copied = [&](int x) { return warp_wait(&atoms_free[x & 1], uint32_t(x >> 1) & 1u, abort_flag, p.wait_ns); };
+        bool ok = true;
+        int prev_key = -2;
+        for (int j = 0; j < n_my; ++j) {
+            const FxItem d = item(j);
+            const int key = fx_act_key(d);
+            const bool act_new = key != prev_key;
+            prev_key = key;
+            if (j >= 2 && !copied(j - 2)) { ok = false; break; }
+            if (j == 1 && !item(0).down && !copied(0)) { ok = false; break; }
+            if (j >= 1 && act_new && d.down && !copied(j - 1)) { ok = false; break; }
+            if (act_new && d.down && act_warp && !fx_group_wait_warp(p, d.g, abort_flag)) { ok = false; break; }
+            const int nk = d.down ? nk_dn : nk_gu;
+            const int nsb = 4 * nk;              // scale bytes per row
+            uint8_t* wdst = sAtoms + (j & 1) * kFxWBuf;
+            uint8_t* adst = sAtoms + (d.down ? kFxDnAct : kFxWBuf);
+            int wrow;
+            if (!d.down) {
+                const int i = et >> 5, jj = et & 31, fr = d.rg * 64 + 16 * i + (jj & 15);
+                wrow = jj < 16 ? fr : p.F + fr;
+            } else {
+                wrow = d.rg * 128 + et;
+            }
+            const uint8_t* wsc = d.down ? p.wsc2 + (size_t(d.g) * p.H + wrow) * nsb
+                                        : p.wsc13 + (size_t(d.g) * 2 * p.F + wrow) * nsb;
+            // a row's scales arrive as 16-byte vectors (four K steps each), all loads in flight:
+            // issued unconditionally (vectors past the row's last re-read it) so none waits on a branch
+            const uint4* ws = reinterpret_cast<const uint4*>(wsc);
+            const int nv = nk / 4;
+            uint4 wv[kDxSteps / 4];
+#pragma unroll
+            for (int c4 = 0; c4 < kDxSteps / 4; ++c4) wv[c4] = __ldg(ws + min(c4, nv - 1));
+#pragma unroll
+            for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
+                if (c4 >= nv) break;
+                const uint32_t w4[4] = {wv[c4].x, wv[c4].y, wv[c4].z, wv[c4].w};
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+                    *reinterpret_cast<uint32_t*>(wdst + (4 * c4 + cc) * 512 + 16 * (et & 31) + 4 * (et >> 5)) = w4[cc];
+            }
+            if (act_new && act_warp && (et & 31) < p.NB) {
+                const int pl = et >> 5, nrow = et & 31, m = pl * p.NB + nrow;   // B row of the merged operand
+                const uint8_t* bsrc = d.down ? (pl ? p.hsl : p.hsh) : (pl ? p.xsl : p.xsh);
+                const int brow = d.down ? d.r0 + nrow : nrow;
+                const bool valid = d.down ? nrow < d.n : nrow < p.T;
+                const uint4* bs = reinterpret_cast<const uint4*>(bsrc + size_t(valid ? brow : 0) * nsb);
+#pragma unroll
+                for (int c4 = 0; c4 < kDxSteps / 4; ++c4) wv[c4] = __ldcg(bs + min(c4, nv - 1));
+#pragma unroll
+                for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
+                    if (c4 >= nv) break;
+                    const uint4 b = valid ? wv[c4] : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+                    const uint32_t b4[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+                        *reinterpret_cast<uint32_t*>(adst + (4 * c4 + cc) * 512 + 16 * (m & 31) + 4 * (m >> 5)) = b4[cc];
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&atoms_full[j & 1]);
+        }
+        if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
+    } else {
+        // ------------------------------------------------ epilogue warps 2..5 (TMEM lane quarter q)
+        const int q = warp & 3;
+        // the two warps of a 32-column h block meet on their pair's barrier (two arrivals a phase)
+        const int pr = q >> 1, hf = q & 1;
+        int ps = 0;
+        auto pair_sync = [&]() {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pair_bar[pr]);
+            const bool r = warp_wait(&pair_bar[pr], uint32_t(ps & 1), abort_flag, p.wait_ns);
+            ++ps;
+            return r;
+        };
+        bool ok = true;
+        for (int j = 0; j < n_my && ok; ++j) {
+            const FxItem d = item(j);
+            const int my_tok = (!d.down && lane < d.n) ? group_token_of(p.sorted_flat[d.r0 + lane], P, p.k) : -1;
+            const int buf = j & 1;
+            if (!warp_wait(&tfull[buf], uint32_t(j >> 1) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t tacc = tmem + (uint32_t(q * 32) << 16) + uint32_t(kDxAccCols * buf);
+            if (d.down) {
+                // column c of the hi rows plus column NB + c of the lo rows
+                float v[32];
+                if (p.NB == 32) {
+                    float w[32];
+                    tmem_ld32_nowait(tacc, v);
+                    tmem_ld32_nowait(tacc + 32u, w);
+                    tmem_wait_ld(v, w);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) v[c] += w[c];
+                } else {
+                    tmem_ld32_nowait(tacc, v);
+                    tmem_wait_16(v);
+                    tmem_fence_regs(v + 16);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) v[c] += v[16 + c];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i < d.n) p.o[size_t(d.r0 + i) * p.H + 128 * d.rg + 32 * q + lane] = f2bf(v[i]);
+            } else {
+                // One group row (token) at a time: its accumulator column read straight from TMEM.
+                // Lanes < 16: h at column f = 64 rg + 16 q + lane (gate row lane, up row lane + 16);
+                // warps q = 2 pr, 2 pr + 1 hold 32-column block pr.  Each writes its partial max|h|,
+                // meets its partner, forms the block's first scale and plane, writes its partial
+                // max|h - hi|, meets again, and stores both planes (slot rl of each array is this
+                // row's; the next item writes them only after both warps passed the last meeting).
+                float* x1 = xch + pr * 128;        // [half][row] partial max|h|
+                float* x2 = x1 + 64;               // [half][row] partial max|h - hi|
+                const int f = 64 * d.rg + 16 * q + lane;
+                for (int rl = 0; rl < d.n; ++rl) {
+                    const int c = __shfl_sync(0xffffffffu, my_tok, rl);
+                    float ah, al;
+                    tmem_ld1x2(tacc + uint32_t(c), tacc + uint32_t(p.NB + c), ah, al);
+                    const float acc = ah + al;
+                    const float other = __shfl_xor_sync(0xffffffffu, acc, 16);
+                    const float hv = lane < 16 ? bf16lo(uint32_t(f2bf(silu_mul(acc, other)))) : 0.f;
+                    const float m1 = warp_max(fabsf(hv));
+                    if (lane == 0) x1[hf * 32 + rl] = m1;
+                    if (!pair_sync()) { ok = false; break; }
+                    float X1, X2, d4[4];
+                    const uint32_t s1 = e8m0_of(fmaxf(x1[rl], x1[32 + rl]), X1);
+                    const uint32_t hi = e4m3x4(hv * (1.f / X1), 0.f, 0.f, 0.f) & 0xFFu;
+                    e4m3x4_dec(hi, d4);
+                    const float res = hv - d4[0] * X1;
+                    const float m2 = warp_max(lane < 16 ? fabsf(res) : 0.f);
+                    if (lane == 0) x2[hf * 32 + rl] = m2;
+                    if (!pair_sync()) { ok = false; break; }
+                    const uint32_t s2 = e8m0_of(fmaxf(x2[rl], x2[32 + rl]), X2);
+                    const uint32_t lo = e4m3x4(res * (1.f / X2), 0.f, 0.f, 0.f) & 0xFFu;
+                    const int r = d.r0 + rl;
+                    if (lane < 16) {
+                        p.hh[size_t(r) * p.F + f] = uint8_t(hi);
+                        p.hl[size_t(r) * p.F + f] = uint8_t(lo);
+                    }
+                    if (hf == 0 && lane == 0) {
+                        p.hsh[size_t(r) * (p.F / 32) + 2 * d.rg + pr] = uint8_t(s1);
+                        p.hsl[size_t(r) * (p.F / 32) + 2 * d.rg + pr] = uint8_t(s2);
+                    }
+                }
+                if (!ok) break;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicAdd(p.ready + d.g, 1u);
             }
         }
         if (!ok) { *abort_flag = 1; if (lane == 0) atomicExch(p.err, kDevErrTimeout); }
@@ -587,6 +1051,41 @@ cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
     if (!plane_map(&gbh, xh, H, 32, NB) || !plane_map(&gbl, xl, H, 32, NB) || !plane_map(&dbh, hh, F, R, NB) ||
         !plane_map(&dbl, hl, F, R, NB))
         return cudaErrorInvalidValue;
+    if (F <= kFxMaxKDn && T <= kFxMaxT) {
+        // x planes, then gate/up and down in one persistent launch (h planes written by its epilogue)
+        constexpr size_t fsmem = dec_mx_fused_smem();
+        static bool fattr = false;
+        if (!fattr) {
+            cudaError_t e = cudaFuncSetAttribute(decode_mx_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 int(fsmem));
+            if (e != cudaSuccess) return e;
+            fattr = true;
+        }
+        DecMxFusedParams f{};
+        f.T = T; f.k = k; f.E = E; f.H = H; f.F = F; f.G = G; f.NB = NB;
+        f.gu_blocks = F / 64;
+        f.dn_blocks = H / 128;
+        f.offsets = a.offsets;
+        f.sorted_flat = a.sorted_flat;
+        f.sched = a.sched;
+        f.wsc13 = a.w13s;
+        f.wsc2 = a.w2s;
+        f.xsh = xsh; f.xsl = xsl;
+        f.hh = hh; f.hl = hl; f.hsh = hsh; f.hsl = hsl;
+        f.o = p.o;
+        f.ready = a.err + kWsReady;
+        f.err = a.err;
+        f.wait_ns = p.wait_ns;
+        const int items = na_max * (f.gu_blocks + f.dn_blocks);
+        cudaError_t e = launch_dep(quant2_kernel, (32 * (H / 32) + 255) / 256, 256, 0, st, a.x, T, 32, H, xh, xl, xsh, xsl);
+        if (e != cudaSuccess) return e;
+        e = launch_dep(decode_mx_fused_kernel, items < num_sms() ? items : num_sms(), kFxThreads, fsmem, st, gw, dw, gbh,
+                       gbl, dbh, dbl, f);
+        if (e != cudaSuccess) return e;
+        if (a.y) e = launch_combine_dependent(T, H, k, 0, R, a.o_ws, a.inv_pos, a.topk_w, a.y, st);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
     constexpr size_t smem = dec_mx_smem();
     static bool attr = false;
     if (!attr) {

@@ -113,6 +113,16 @@ __device__ __forceinline__ void tmem_fence_regs(float* v) {   // no-op that pins
     asm volatile("" : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
                  "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]));
 }
+// one column at each of two TMEM addresses (warp-uniform) for this thread's lane, waited for
+__device__ __forceinline__ void tmem_ld1x2(uint32_t ta, uint32_t tb, float& a, float& b) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%2];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%1}, [%3];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=f"(a), "=f"(b)
+        : "r"(ta), "r"(tb)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld(float (&a)[32], float (&b)[32]) {
     tmem_wait_16(a);
     tmem_fence_regs(a + 16);

@@ -233,8 +233,12 @@ def block_scaled_decode():
         assert F.ft_set_block_scaled_decode(prev) == 1
 
 
-@pytest.mark.parametrize("name,T,kw", [("dsv4_flash", 1, {}), ("dsv4_flash", 8, {}), ("dsv4_flash", 20, {}),
-                                       ("dsv4_flash", 32, {}),
+@pytest.mark.parametrize("name,T,kw", [("dsv4_flash", 1, {}), ("dsv4_flash", 8, {}), ("dsv4_flash", 16, {}),
+                                       ("dsv4_flash", 20, {}), ("dsv4_flash", 32, {}),
+                                       # few gate/up items: some CTAs start on down items and wait
+                                       # for other CTAs' gate/up epilogues
+                                       ("custom", 4, dict(hidden=512, ffn=512, num_experts=4, top_k=1,
+                                                          num_shared=0, wdtype=inputs.WDTYPE_MXFP4, config_id=92)),
                                        ("custom", 13, dict(hidden=1024, ffn=512, num_experts=16, top_k=4,
                                                            num_shared=0, wdtype=inputs.WDTYPE_MXFP4, config_id=83)),
                                        # FFN 4096: one activation-scale buffer in TMEM for down, a
