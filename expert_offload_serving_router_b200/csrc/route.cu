@@ -28,6 +28,10 @@ struct SmallRouteArgs {
     PermOut perm;
 };
 
+// TOK tokens per pass, NI float4s of the router row per thread and pass of the row: every x load
+// of a pass is issued before any is used (TOK x NI 8-byte loads in flight per thread), so a pass
+// costs one L2 round trip rather than one per token.
+template <int TOK, int NI>
 __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteArgs a) {
     __shared__ float red[kSmallRoute][8];
     __shared__ int last;
@@ -36,10 +40,10 @@ __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteArgs a) {
     const float* wrow = a.wr + size_t(e) * a.H;
     for (int t = tid; t < kSmallRoute * 8; t += 256) (&red[0][0])[t] = 0.f;
     __syncthreads();
-    for (int base = 0; base < nq; base += 256 * 4) {
-        float4 w[4];
+    for (int base = 0; base < nq; base += 256 * NI) {
+        float4 w[NI];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < NI; ++i) {
             int q = base + tid + 256 * i;
             w[i] = q < nq ? __ldg(reinterpret_cast<const float4*>(wrow) + q) : make_float4(0, 0, 0, 0);
         }
@@ -50,35 +54,53 @@ __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteArgs a) {
             asm volatile("griddepcontrol.wait;" ::: "memory");
             asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         }
-        // eight tokens per pass: all their x loads in flight together, then one transpose-
-        // reduce leaves token t0 + 4*bit4(lane) + 2*bit3(lane) + bit2(lane) on lane
-        for (int t0 = 0; t0 < a.T; t0 += 8) {
-            float s[8];
+        for (int t0 = 0; t0 < a.T; t0 += TOK) {
+            // loads with clamped indices (rows past T re-read the last token, vectors past the
+            // row's end its last vector): no branch between them; both kinds are dropped below
+            uint2 u[TOK][NI];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < TOK; ++j) {
+                const uint2* xr = reinterpret_cast<const uint2*>(a.x + size_t(min(t0 + j, a.T - 1)) * a.H);
+#pragma unroll
+                for (int i = 0; i < NI; ++i) u[j][i] = __ldg(xr + min(base + tid + 256 * i, nq - 1));
+            }
+            float s[TOK];
+#pragma unroll
+            for (int j = 0; j < TOK; ++j) {
                 s[j] = 0.f;
-                if (t0 + j < a.T) {
-                    const uint2* xr = reinterpret_cast<const uint2*>(a.x + size_t(t0 + j) * a.H);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        int q = base + tid + 256 * i;
-                        if (q < nq) {
-                            uint2 u = __ldg(xr + q);
-                            s[j] = fmaf(bf16lo(u.x), w[i].x, s[j]);
-                            s[j] = fmaf(bf16hi(u.x), w[i].y, s[j]);
-                            s[j] = fmaf(bf16lo(u.y), w[i].z, s[j]);
-                            s[j] = fmaf(bf16hi(u.y), w[i].w, s[j]);
-                        }
+                for (int i = 0; i < NI; ++i) {
+                    if (base + tid + 256 * i < nq) {
+                        s[j] = fmaf(bf16lo(u[j][i].x), w[i].x, s[j]);
+                        s[j] = fmaf(bf16hi(u[j][i].x), w[i].y, s[j]);
+                        s[j] = fmaf(bf16lo(u[j][i].y), w[i].z, s[j]);
+                        s[j] = fmaf(bf16hi(u[j][i].y), w[i].w, s[j]);
                     }
                 }
             }
-            tr_step(s, 8, 16, lane);
-            tr_step(s, 4, 8, lane);
-            tr_step(s, 2, 4, lane);
-            s[0] += __shfl_xor_sync(0xffffffffu, s[0], 2);
-            s[0] += __shfl_xor_sync(0xffffffffu, s[0], 1);
-            const int t = t0 + ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-            if ((lane & 3) == 0 && t < a.T) red[t][warp] += s[0];
+            // transpose-reduce: lane l ends with the warp sum of token t0 + (its TOK-slot from
+            // bits 4, 3 (and 2) of l)
+            int t;
+            if (TOK == 1) {
+#pragma unroll
+                for (int o = 16; o; o >>= 1) s[0] += __shfl_xor_sync(0xffffffffu, s[0], o);
+                t = lane == 0 ? t0 : a.T;
+            } else if (TOK == 8) {
+                tr_step(s, 8, 16, lane);
+                tr_step(s, 4, 8, lane);
+                tr_step(s, 2, 4, lane);
+                s[0] += __shfl_xor_sync(0xffffffffu, s[0], 2);
+                s[0] += __shfl_xor_sync(0xffffffffu, s[0], 1);
+                t = (lane & 3) == 0 ? t0 + ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1) : a.T;
+            } else {   // TOK == 4
+                tr_step(s, 4, 16, lane);
+                tr_step(s, 2, 8, lane);
+                s[0] += __shfl_xor_sync(0xffffffffu, s[0], 4);
+                s[0] += __shfl_xor_sync(0xffffffffu, s[0], 2);
+                s[0] += __shfl_xor_sync(0xffffffffu, s[0], 1);
+                t = (lane & 7) == 0 ? t0 + ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1) : a.T;
+            }
+            if (t < a.T) red[t][warp] += s[0];
         }
     }
     __syncthreads();
@@ -95,11 +117,17 @@ __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteArgs a) {
     __syncthreads();
     if (!last) return;
     __threadfence();
-    // ---- last CTA: top-k for every token (+ permutation), a warp per token
+    // ---- last CTA: top-k for every token (+ permutation), a warp per token; the next token's
+    // logits load while this one's are selected
     __shared__ int32_t sidx[kSmallRoute * kMaxTopK];
-    for (int t = warp; t < a.T; t += 8)
-        warp_topk_row(a.logits + size_t(t) * a.E, a.E, a.k, a.topk_idx + size_t(t) * a.k, a.topk_w + size_t(t) * a.k,
-                      sidx + t * a.k);
+    uint32_t key[kTopkPer], nkey[kTopkPer];
+    if (warp < a.T) warp_topk_keys(a.logits + size_t(warp) * a.E, a.E, key);
+    for (int t = warp; t < a.T; t += 8) {
+        if (t + 8 < a.T) warp_topk_keys(a.logits + size_t(t + 8) * a.E, a.E, nkey);
+        warp_topk_select(key, a.k, a.topk_idx + size_t(t) * a.k, a.topk_w + size_t(t) * a.k, sidx + t * a.k);
+#pragma unroll
+        for (int s = 0; s < kTopkPer; ++s) key[s] = nkey[s];
+    }
     if (tid == 0) *a.ticket = 0u;
     __syncthreads();
     if (!a.do_permute) return;
@@ -126,7 +154,13 @@ cudaError_t launch_route(int T, int H, int E, int k, int S, const uint16_t* x, c
         at[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = at;
         cfg.numAttrs = 1;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, route_small_kernel, a);
+        // hidden <= 2048: two row vectors per thread, eight tokens a pass; wider rows: four and
+        // four; a single token: one a pass
+        const bool narrow = H / 4 <= 512;
+        cudaError_t e = T == 1 ? (narrow ? cudaLaunchKernelEx(&cfg, route_small_kernel<1, 2>, a)
+                                         : cudaLaunchKernelEx(&cfg, route_small_kernel<1, 4>, a))
+                               : (narrow ? cudaLaunchKernelEx(&cfg, route_small_kernel<8, 2>, a)
+                                         : cudaLaunchKernelEx(&cfg, route_small_kernel<4, 4>, a));
         if (e != cudaSuccess || !perm) return e;
         return launch_perm_check(topk_idx, T, k, E, S, *perm, st);
     }

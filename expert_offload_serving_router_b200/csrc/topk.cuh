@@ -109,21 +109,25 @@ __device__ __forceinline__ void top_slot(const Top8& t, int k, int j, int32_t* e
     *w_out = expf(key_logit(kk) - l0) / den;
 }
 
-// Warp-wide top-k over the E <= 256 logits of one token, read from global memory `row` (L2:
-// another CTA wrote them) straight into registers.  Lane l holds the keys of experts l, l+32, ...; each of the k rounds takes the warp's largest key
-// (one max-reduction) and, among the lanes holding it, the lowest expert (one min-reduction),
-// then the owning lane drops it.  Same order as Top8 (logit desc, index asc; key 0 never
-// chosen) and the same gates; lanes 0..k-1 write slot = lane.
-__device__ inline void warp_topk_row(const float* row, int E, int k, int32_t* idx_out, float* w_out,
-                                     int32_t* idx_smem) {
-    constexpr int kPer = kMaxExperts / 32;
+// Warp-wide top-k over the E <= 256 logits of one token.  warp_topk_keys reads the row from
+// global memory `row` (L2: other CTAs wrote it) into registers -- lane l holds the keys of
+// experts l, l+32, ... -- so a caller can have the next token's loads in flight while it selects
+// this one.  warp_topk_select takes k rounds: each takes the warp's largest key (one
+// max-reduction) and, among the lanes holding it, the lowest expert (one min-reduction), then
+// the owning lane drops it.  Same order as Top8 (logit desc, index asc; key 0 never chosen) and
+// the same gates; lanes 0..k-1 write slot = lane.
+constexpr int kTopkPer = kMaxExperts / 32;
+__device__ __forceinline__ void warp_topk_keys(const float* row, int E, uint32_t (&key)[kTopkPer]) {
     const int lane = threadIdx.x & 31;
-    uint32_t key[kPer];
 #pragma unroll
-    for (int s = 0; s < kPer; ++s) {
+    for (int s = 0; s < kTopkPer; ++s) {
         const int e = lane + 32 * s;
         key[s] = e < E ? logit_key(__ldcg(row + e)) : 0u;
     }
+}
+__device__ inline void warp_topk_select(uint32_t (&key)[kTopkPer], int k, int32_t* idx_out, float* w_out,
+                                        int32_t* idx_smem) {
+    const int lane = threadIdx.x & 31;
     Top8 t;
     t.init();
 #pragma unroll
@@ -131,7 +135,7 @@ __device__ inline void warp_topk_row(const float* row, int E, int k, int32_t* id
         if (j >= k) break;
         uint32_t bk = 0u, be = 0xffffffffu;        // this lane's best: experts ascend with s
 #pragma unroll
-        for (int s = 0; s < kPer; ++s) {
+        for (int s = 0; s < kTopkPer; ++s) {
             const bool better = key[s] > bk;
             bk = better ? key[s] : bk;
             be = better ? uint32_t(lane + 32 * s) : be;
@@ -140,7 +144,7 @@ __device__ inline void warp_topk_row(const float* row, int E, int k, int32_t* id
         if (mk == 0u) break;                       // only key-0 experts left: slots stay (0, 0)
         const uint32_t me = __reduce_min_sync(0xffffffffu, bk == mk ? be : 0xffffffffu);
 #pragma unroll
-        for (int s = 0; s < kPer; ++s)
+        for (int s = 0; s < kTopkPer; ++s)
             if (uint32_t(lane + 32 * s) == me) key[s] = 0u;
         t.key[j] = mk;
         t.idx[j] = int32_t(me);
