@@ -841,13 +841,24 @@ decode_mx_fused_kernel(const __grid_constant__ CUtensorMap tm_w13, const __grid_
             }
             const uint8_t* wsc = d.down ? p.wsc2 + (size_t(d.g) * p.H + wrow) * nsb
                                         : p.wsc13 + (size_t(d.g) * 2 * p.F + wrow) * nsb;
-            // a row's scales arrive as 16-byte vectors (four K steps each), all loads in flight:
-            // issued unconditionally (vectors past the row's last re-read it) so none waits on a branch
+            // a row's scales arrive as 16-byte vectors (four K steps each), the weight and the
+            // activation vectors all in flight before any is used (vectors past the row's last
+            // re-read it)
             const uint4* ws = reinterpret_cast<const uint4*>(wsc);
             const int nv = nk / 4;
-            uint4 wv[kDxSteps / 4];
+            uint4 wv[kDxSteps / 4], av[kDxSteps / 4];
 #pragma unroll
             for (int c4 = 0; c4 < kDxSteps / 4; ++c4) wv[c4] = __ldg(ws + min(c4, nv - 1));
+            const bool do_act = act_new && act_warp && (et & 31) < p.NB;
+            const int pl = et >> 5, nrow = et & 31, m = pl * p.NB + nrow;   // B row of the merged operand
+            const bool valid = d.down ? nrow < d.n : nrow < p.T;
+            if (do_act) {
+                const uint8_t* bsrc = d.down ? (pl ? p.hsl : p.hsh) : (pl ? p.xsl : p.xsh);
+                const int brow = d.down ? d.r0 + nrow : nrow;
+                const uint4* bs = reinterpret_cast<const uint4*>(bsrc + size_t(valid ? brow : 0) * nsb);
+#pragma unroll
+                for (int c4 = 0; c4 < kDxSteps / 4; ++c4) av[c4] = __ldcg(bs + min(c4, nv - 1));
+            }
 #pragma unroll
             for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
                 if (c4 >= nv) break;
@@ -856,18 +867,11 @@ decode_mx_fused_kernel(const __grid_constant__ CUtensorMap tm_w13, const __grid_
                 for (int cc = 0; cc < 4; ++cc)
                     *reinterpret_cast<uint32_t*>(wdst + (4 * c4 + cc) * 512 + 16 * (et & 31) + 4 * (et >> 5)) = w4[cc];
             }
-            if (act_new && act_warp && (et & 31) < p.NB) {
-                const int pl = et >> 5, nrow = et & 31, m = pl * p.NB + nrow;   // B row of the merged operand
-                const uint8_t* bsrc = d.down ? (pl ? p.hsl : p.hsh) : (pl ? p.xsl : p.xsh);
-                const int brow = d.down ? d.r0 + nrow : nrow;
-                const bool valid = d.down ? nrow < d.n : nrow < p.T;
-                const uint4* bs = reinterpret_cast<const uint4*>(bsrc + size_t(valid ? brow : 0) * nsb);
-#pragma unroll
-                for (int c4 = 0; c4 < kDxSteps / 4; ++c4) wv[c4] = __ldcg(bs + min(c4, nv - 1));
+            if (do_act) {
 #pragma unroll
                 for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
                     if (c4 >= nv) break;
-                    const uint4 b = valid ? wv[c4] : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+                    const uint4 b = valid ? av[c4] : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
                     const uint32_t b4[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc)
