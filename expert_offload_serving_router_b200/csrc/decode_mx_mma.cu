@@ -188,6 +188,78 @@ __device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, volatile
     return r != 0;
 }
 
+// The eight MMAs of one 256-deep stage: two 128-deep sub-tiles of four 32-deep K blocks each
+// (scale byte j of every row's step word selects block j); sfa / sfb advance one step per
+// sub-tile.  acc0: the stage's first MMA accumulates (false only for an item's first stage).
+__device__ __forceinline__ void dx_stage_mmas(uint32_t dacc, uint64_t ad0, uint64_t bd0, int stage,
+                                              const uint32_t (&idm)[4], uint32_t& sfa, uint32_t& sfb, bool acc0) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const uint64_t ad = ad0 + uint64_t((stage * kDxAStage + u * kDxATile) >> 4);
+        const uint64_t bd = bd0 + uint64_t((stage * kDxBStage + u * kDxBSub) >> 4);
+        umma_mx(dacc, ad, bd, idm[0], sfa, sfb, (acc0 || u) ? 1u : 0u);
+        umma_mx(dacc, ad + 2, bd + 2, idm[1], sfa + (1u << 30), sfb + (1u << 30), 1u);
+        umma_mx(dacc, ad + 4, bd + 4, idm[2], sfa + (2u << 30), sfb + (2u << 30), 1u);
+        umma_mx(dacc, ad + 6, bd + 6, idm[3], sfa + (3u << 30), sfb + (3u << 30), 1u);
+        sfa += 4u;
+        sfb += 4u;
+    }
+}
+
+// This thread's accumulator lane at `tacc`: column c of the hi rows plus column NB + c of the lo
+// rows into v[c], c < NB (NB = 16 or 32); waited for.
+__device__ __forceinline__ void dx_acc_load(uint32_t tacc, int NB, float (&v)[32]) {
+    if (NB == 32) {
+        float w[32];
+        tmem_ld32_nowait(tacc, v);
+        tmem_ld32_nowait(tacc + 32u, w);
+        tmem_wait_ld(v, w);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) v[c] += w[c];
+    } else {
+        tmem_ld32_nowait(tacc, v);
+        tmem_wait_16(v);
+        tmem_fence_regs(v + 16);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) v[c] += v[16 + c];
+    }
+}
+
+// One A-tile row's weight scales (`ws`: nv 16-byte vectors of four 128-deep K steps each) and,
+// when do_act, one B row's activation scales (`bs`; the scale 1.0 where !valid) laid out as
+// tcgen05.cp source atoms: the atom of step c at c x 512 bytes, byte 16 (row % 32) + 4 (row / 32)
+// + j = the row's scale of 32-block j (row = et for weights, m for activations).  Every load is in
+// flight before any is used (vectors past the row's last re-read it).
+__device__ __forceinline__ void dx_lay_atoms(const uint4* ws, int nv, int et, uint8_t* wdst, bool do_act,
+                                             const uint4* bs, bool valid, int m, uint8_t* adst) {
+    uint4 wv[kDxSteps / 4], av[kDxSteps / 4];
+#pragma unroll
+    for (int c4 = 0; c4 < kDxSteps / 4; ++c4) wv[c4] = __ldg(ws + min(c4, nv - 1));
+    if (do_act) {
+#pragma unroll
+        for (int c4 = 0; c4 < kDxSteps / 4; ++c4) av[c4] = __ldcg(bs + min(c4, nv - 1));
+    }
+#pragma unroll
+    for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
+        if (c4 >= nv) break;
+        const uint32_t w4[4] = {wv[c4].x, wv[c4].y, wv[c4].z, wv[c4].w};
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+            *reinterpret_cast<uint32_t*>(wdst + (4 * c4 + cc) * 512 + 16 * (et & 31) + 4 * (et >> 5)) = w4[cc];
+    }
+    if (do_act) {
+#pragma unroll
+        for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
+            if (c4 >= nv) break;
+            const uint4 b = valid ? av[c4] : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+            const uint32_t b4[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+                *reinterpret_cast<uint32_t*>(adst + (4 * c4 + cc) * 512 + 16 * (m & 31) + 4 * (m >> 5)) = b4[cc];
+        }
+    }
+}
+
 // Where an item's scale factors live.  TMEM columns: [0, 128) the two accumulator buffers, then
 // nact activation-scale buffers and two weight-scale buffers of 4 columns per 128-deep K step
 // (step c of a buffer at column base + 4 c).  Shared memory (the 32 KB atom area): gate/up --
@@ -338,18 +410,7 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
                     // the stage's operands were all written by TMA (async proxy): its barrier's
                     // completion orders them before these MMAs, no thread-sync fence needed
                     if (!wait_fast(&full[stage], phase, abort_flag, p.wait_ns)) { ok = false; break; }
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const uint64_t ad = ad0 + uint64_t((stage * kDxAStage + u * kDxATile) >> 4);
-                        const uint64_t bd = bd0 + uint64_t((stage * kDxBStage + u * kDxBSub) >> 4);
-                        // the four 32-deep K blocks of the sub-tile (scale byte j of each row's step word)
-                        umma_mx(dacc, ad, bd, idm[0], sfa, sfb, (kb | u) != 0);
-                        umma_mx(dacc, ad + 2, bd + 2, idm[1], sfa + (1u << 30), sfb + (1u << 30), 1u);
-                        umma_mx(dacc, ad + 4, bd + 4, idm[2], sfa + (2u << 30), sfb + (2u << 30), 1u);
-                        umma_mx(dacc, ad + 6, bd + 6, idm[3], sfa + (3u << 30), sfb + (3u << 30), 1u);
-                        sfa += 4u;
-                        sfb += 4u;
-                    }
+                    dx_stage_mmas(dacc, ad0, bd0, stage, idm, sfa, sfb, kb != 0);
                     umma_commit(&empty[stage]);
                     if (++stage == kDxSt) { stage = 0; phase ^= 1u; }
                 }
@@ -418,39 +479,13 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
             } else {
                 wrow = rg2 * 128 + et;
             }
-            // a row's scales arrive as 16-byte vectors (four K steps each), all loads in flight:
-            // issued unconditionally (vectors past the row's last re-read it) so none waits on a branch
-            const uint4* ws = reinterpret_cast<const uint4*>(p.wsc + (size_t(g2) * rows_e + wrow) * nsb);
-            const int nv = nk / 4;
-            uint4 wv[kDxSteps / 4];
-#pragma unroll
-            for (int c4 = 0; c4 < kDxSteps / 4; ++c4) wv[c4] = __ldg(ws + min(c4, nv - 1));
-#pragma unroll
-            for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
-                if (c4 >= nv) break;
-                const uint32_t w4[4] = {wv[c4].x, wv[c4].y, wv[c4].z, wv[c4].w};
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc)
-                    *reinterpret_cast<uint32_t*>(wdst + (4 * c4 + cc) * 512 + 16 * (et & 31) + 4 * (et >> 5)) = w4[cc];
-            }
-            if (act_new && et < 64 && (et & 31) < p.NB) {
-                const int pl = et >> 5, nrow = et & 31, m = pl * p.NB + nrow;   // B row of the merged operand
-                const uint8_t* bsrc = pl ? p.bsc_lo : p.bsc_hi;
-                const int brow = MODE == 0 ? nrow : r02 + nrow;
-                const bool valid = MODE == 0 ? nrow < p.T : nrow < n2;
-                const uint4* bs = reinterpret_cast<const uint4*>(bsrc + size_t(valid ? brow : 0) * nsb);
-#pragma unroll
-                for (int c4 = 0; c4 < kDxSteps / 4; ++c4) wv[c4] = __ldcg(bs + min(c4, nv - 1));
-#pragma unroll
-                for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
-                    if (c4 >= nv) break;
-                    const uint4 b = valid ? wv[c4] : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-                    const uint32_t b4[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
-                        *reinterpret_cast<uint32_t*>(adst + (4 * c4 + cc) * 512 + 16 * (m & 31) + 4 * (m >> 5)) = b4[cc];
-                }
-            }
+            const int pl = et >> 5, nrow = et & 31, m = pl * p.NB + nrow;   // B row of the merged operand
+            const bool do_act = act_new && et < 64 && nrow < p.NB;
+            const bool valid = MODE == 0 ? nrow < p.T : nrow < n2;
+            const int brow = MODE == 0 ? nrow : r02 + nrow;
+            const uint8_t* bsrc = pl ? p.bsc_lo : p.bsc_hi;
+            dx_lay_atoms(reinterpret_cast<const uint4*>(p.wsc + (size_t(g2) * rows_e + wrow) * nsb), nk / 4, et, wdst,
+                         do_act, reinterpret_cast<const uint4*>(bsrc + size_t(valid ? brow : 0) * nsb), valid, m, adst);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&atoms_full[wb]);
@@ -480,22 +515,7 @@ decode_mx_mma_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
             if (!warp_wait(&tfull[buf], uint32_t(j >> 1) & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             float v[32];
-            // column c of the hi rows plus column NB + c of the lo rows
-            const uint32_t tacc = tmem + (uint32_t(q * 32) << 16) + uint32_t(kDxAccCols * buf);
-            if (p.NB == 32) {
-                float w[32];
-                tmem_ld32_nowait(tacc, v);
-                tmem_ld32_nowait(tacc + 32u, w);
-                tmem_wait_ld(v, w);
-#pragma unroll
-                for (int c = 0; c < 32; ++c) v[c] += w[c];
-            } else {
-                tmem_ld32_nowait(tacc, v);
-                tmem_wait_16(v);
-                tmem_fence_regs(v + 16);
-#pragma unroll
-                for (int c = 0; c < 16; ++c) v[c] += v[16 + c];
-            }
+            dx_acc_load(tmem + (uint32_t(q * 32) << 16) + uint32_t(kDxAccCols * buf), p.NB, v);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -746,17 +766,7 @@ decode_mx_fused_kernel(const __grid_constant__ CUtensorMap tm_w13, const __grid_
                 const int nk = d.down ? nk_dn : nk_gu;
                 for (int kb = 0; kb < nk / 2; ++kb) {
                     if (!wait_fast(&full[stage], phase, abort_flag, p.wait_ns)) { ok = false; break; }
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const uint64_t ad = ad0 + uint64_t((stage * kDxAStage + u * kDxATile) >> 4);
-                        const uint64_t bd = bd0 + uint64_t((stage * kDxBStage + u * kDxBSub) >> 4);
-                        umma_mx(dacc, ad, bd, idm[0], sfa, sfb, (kb | u) != 0);
-                        umma_mx(dacc, ad + 2, bd + 2, idm[1], sfa + (1u << 30), sfb + (1u << 30), 1u);
-                        umma_mx(dacc, ad + 4, bd + 4, idm[2], sfa + (2u << 30), sfb + (2u << 30), 1u);
-                        umma_mx(dacc, ad + 6, bd + 6, idm[3], sfa + (3u << 30), sfb + (3u << 30), 1u);
-                        sfa += 4u;
-                        sfb += 4u;
-                    }
+                    dx_stage_mmas(dacc, ad0, bd0, stage, idm, sfa, sfb, kb != 0);
                     umma_commit(&empty[stage]);
                     if (++stage == kDxSt) { stage = 0; phase ^= 1u; }
                 }
@@ -841,43 +851,13 @@ decode_mx_fused_kernel(const __grid_constant__ CUtensorMap tm_w13, const __grid_
             }
             const uint8_t* wsc = d.down ? p.wsc2 + (size_t(d.g) * p.H + wrow) * nsb
                                         : p.wsc13 + (size_t(d.g) * 2 * p.F + wrow) * nsb;
-            // a row's scales arrive as 16-byte vectors (four K steps each), the weight and the
-            // activation vectors all in flight before any is used (vectors past the row's last
-            // re-read it)
-            const uint4* ws = reinterpret_cast<const uint4*>(wsc);
-            const int nv = nk / 4;
-            uint4 wv[kDxSteps / 4], av[kDxSteps / 4];
-#pragma unroll
-            for (int c4 = 0; c4 < kDxSteps / 4; ++c4) wv[c4] = __ldg(ws + min(c4, nv - 1));
-            const bool do_act = act_new && act_warp && (et & 31) < p.NB;
             const int pl = et >> 5, nrow = et & 31, m = pl * p.NB + nrow;   // B row of the merged operand
+            const bool do_act = act_new && act_warp && nrow < p.NB;
             const bool valid = d.down ? nrow < d.n : nrow < p.T;
-            if (do_act) {
-                const uint8_t* bsrc = d.down ? (pl ? p.hsl : p.hsh) : (pl ? p.xsl : p.xsh);
-                const int brow = d.down ? d.r0 + nrow : nrow;
-                const uint4* bs = reinterpret_cast<const uint4*>(bsrc + size_t(valid ? brow : 0) * nsb);
-#pragma unroll
-                for (int c4 = 0; c4 < kDxSteps / 4; ++c4) av[c4] = __ldcg(bs + min(c4, nv - 1));
-            }
-#pragma unroll
-            for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
-                if (c4 >= nv) break;
-                const uint32_t w4[4] = {wv[c4].x, wv[c4].y, wv[c4].z, wv[c4].w};
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc)
-                    *reinterpret_cast<uint32_t*>(wdst + (4 * c4 + cc) * 512 + 16 * (et & 31) + 4 * (et >> 5)) = w4[cc];
-            }
-            if (do_act) {
-#pragma unroll
-                for (int c4 = 0; c4 < kDxSteps / 4; ++c4) {
-                    if (c4 >= nv) break;
-                    const uint4 b = valid ? av[c4] : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-                    const uint32_t b4[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
-                        *reinterpret_cast<uint32_t*>(adst + (4 * c4 + cc) * 512 + 16 * (m & 31) + 4 * (m >> 5)) = b4[cc];
-                }
-            }
+            const int brow = d.down ? d.r0 + nrow : nrow;
+            const uint8_t* bsrc = d.down ? (pl ? p.hsl : p.hsh) : (pl ? p.xsl : p.xsh);
+            dx_lay_atoms(reinterpret_cast<const uint4*>(wsc), nk / 4, et, wdst, do_act,
+                         reinterpret_cast<const uint4*>(bsrc + size_t(valid ? brow : 0) * nsb), valid, m, adst);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&atoms_full[j & 1]);
@@ -905,22 +885,8 @@ decode_mx_fused_kernel(const __grid_constant__ CUtensorMap tm_w13, const __grid_
             tc_fence_after();
             const uint32_t tacc = tmem + (uint32_t(q * 32) << 16) + uint32_t(kDxAccCols * buf);
             if (d.down) {
-                // column c of the hi rows plus column NB + c of the lo rows
                 float v[32];
-                if (p.NB == 32) {
-                    float w[32];
-                    tmem_ld32_nowait(tacc, v);
-                    tmem_ld32_nowait(tacc + 32u, w);
-                    tmem_wait_ld(v, w);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) v[c] += w[c];
-                } else {
-                    tmem_ld32_nowait(tacc, v);
-                    tmem_wait_16(v);
-                    tmem_fence_regs(v + 16);
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) v[c] += v[16 + c];
-                }
+                dx_acc_load(tacc, p.NB, v);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[buf]);
