@@ -190,6 +190,19 @@ int32_t ft_set_block_scaled_decode(int32_t mode) {
     return prev;
 }
 
+int32_t ft_moe_decode_kernels(const ft_moe_shape* shape, int32_t T) {
+    if (check_shape(shape) != FT_OK || T < 0) return -1;
+    if (T == 0 || T > g_decode_max) return 0;
+    DecodeArgs a{};
+    a.T = T; a.k = shape->top_k; a.E = shape->num_experts; a.S = shape->num_shared;
+    a.H = shape->hidden; a.F = shape->ffn; a.wdtype = shape->wdtype;
+    int n = 1 + decode_path_kernels(decode_path(a), true);   // the router, then the experts
+#if FT_DEBUG_BOUNDS
+    n += 1;                                                  // the permutation check
+#endif
+    return n;
+}
+
 uint64_t ft_set_pipeline_wait_limit_ns(uint64_t ns) {
     const unsigned long long prev = g_gemm_wait_ns;
     g_gemm_wait_ns = ns ? ns : kWaitNs;

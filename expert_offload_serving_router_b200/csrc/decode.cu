@@ -268,10 +268,26 @@ constexpr int kDecodeMmaMinTShared = 2;
 // MXFP4 decode batches of 4+ tokens run on the block-scaled tensor cores (ft_set_block_scaled_decode
 // selects never / always / that default); smaller ones on the GEMVs below, faster there
 
+DecodePath decode_path(const DecodeArgs& a) {
+    if (a.T >= (a.S ? kDecodeMmaMinTShared : kDecodeMmaMinT) && decode_mma_eligible(a)) return kDecodeMma;
+    if (block_scaled_decode(a.T) && decode_mx_eligible(a)) return decode_mx_fused(a) ? kDecodeMxFused : kDecodeMxTwo;
+    return kDecodeGemv;
+}
+
+int decode_path_kernels(DecodePath p, bool combine) {
+    switch (p) {
+        case kDecodeMma: return 1 + combine;                 // decode_mma_kernel, combine
+        case kDecodeMxFused: return 2 + combine;             // quant2 (x), decode_mx_fused_kernel, combine
+        case kDecodeMxTwo: return 4 + combine;               // quant2 (x), gate/up, quant2 (h), down, combine
+        default: return 2;                                   // gate/up GEMV, down GEMV (+ combine, fused)
+    }
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
-    if (a.T >= (a.S ? kDecodeMmaMinTShared : kDecodeMmaMinT) && decode_mma_eligible(a)) return launch_decode_mma(a, st);
-    if (block_scaled_decode(a.T) && decode_mx_eligible(a)) return launch_decode_mx(a, st);
+    const DecodePath path = decode_path(a);
+    if (path == kDecodeMma) return launch_decode_mma(a, st);
+    if (path == kDecodeMxFused || path == kDecodeMxTwo) return launch_decode_mx(a, st);
     const int P = a.T * a.k, R = P + (a.S ? a.T : 0);
     const int G = a.E + (a.S ? 1 : 0);
     {

@@ -959,6 +959,8 @@ bool decode_mx_eligible(const DecodeArgs& a) {
            a.H <= kDxMaxK && a.F <= kDxMaxK;
 }
 
+bool decode_mx_fused(const DecodeArgs& a) { return a.F <= kFxMaxKDn && a.T <= kFxMaxT; }
+
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_dep(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t st, Args... args) {
     cudaLaunchConfig_t cfg = {};
@@ -1021,7 +1023,7 @@ cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
     if (!plane_map(&gbh, xh, H, 32, NB) || !plane_map(&gbl, xl, H, 32, NB) || !plane_map(&dbh, hh, F, R, NB) ||
         !plane_map(&dbl, hl, F, R, NB))
         return cudaErrorInvalidValue;
-    if (F <= kFxMaxKDn && T <= kFxMaxT) {
+    if (decode_mx_fused(a)) {
         // x planes, then gate/up and down in one persistent launch (h planes written by its epilogue)
         constexpr size_t fsmem = dec_mx_fused_smem();
         static bool fattr = false;

@@ -86,11 +86,17 @@ cudaError_t launch_permute(int T, int k, int E, int S, int H, const int32_t* idx
                            uint16_t* x_sorted, int32_t* chunk_cnt, int32_t* chunk_base, int32_t* local_rank,
                            const PermOut& out, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+// the kernels launch_decode runs for a batch (decode.cu): one choice, used for the launch and for
+// the kernel count ft_moe_decode_kernels reports
+enum DecodePath { kDecodeGemv, kDecodeMma, kDecodeMxFused, kDecodeMxTwo };
+DecodePath decode_path(const DecodeArgs& a);
+int decode_path_kernels(DecodePath p, bool combine);   // kernels launched (combine: y != NULL)
 // tensor-core decode (BF16, contiguous weights): false when the shape or weights do not qualify
 bool decode_mma_eligible(const DecodeArgs& a);
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st);
 // block-scaled MXFP4 decode on the tensor cores (decode_mx_mma.cu)
 bool decode_mx_eligible(const DecodeArgs& a);
+bool decode_mx_fused(const DecodeArgs& a);   // gate/up and down in one launch (else two)
 cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st);
 bool block_scaled_decode(int T);   // api.cu: ft_set_block_scaled_decode
 int launch_moe_gemm(const GemmLaunch& L, cudaStream_t st);

@@ -59,6 +59,7 @@ _SIGS = {
     "ft_get_decode_max_tokens": (c_i32, []),
     "ft_set_pipeline_wait_limit_ns": (c_u64, [c_u64]),
     "ft_set_block_scaled_decode": (c_i32, [c_i32]),
+    "ft_moe_decode_kernels": (c_i32, [ctypes.POINTER(ft_moe_shape), c_i32]),
     "ft_hbm_read_probe": (c_i32, [c_vp, c_sz, c_vp, c_i32, c_vp]),
     "ft_tma_read_probe": (c_i32, [c_i32, c_vp, c_sz, c_sz, c_vp, c_vp]),
     "ft_moe_workspace_bytes": (c_sz, [ctypes.POINTER(ft_moe_shape), c_i32]),
@@ -180,6 +181,10 @@ def ft_set_pipeline_wait_limit_ns(ns: int) -> int:
 
 def ft_set_block_scaled_decode(mode: int) -> int:
     return lib().ft_set_block_scaled_decode(mode)
+
+
+def ft_moe_decode_kernels(shape: ft_moe_shape, T: int) -> int:
+    return lib().ft_moe_decode_kernels(ctypes.byref(shape), T)
 
 
 def ft_hbm_read_probe(buf, nbytes: int, sink, ctas_per_sm: int, stream=None) -> None:

@@ -147,6 +147,18 @@ int32_t ft_get_decode_max_tokens(void);
  * in f16.  ft_moe_workspace_bytes reserves room for the planes on MXFP4 shapes. */
 int32_t ft_set_block_scaled_decode(int32_t mode);
 
+/* How many kernels one decode-sized ft_moe_layer_forward call (contiguous
+ * weights) launches for this shape and T under the current settings
+ * (ft_set_decode_max_tokens, ft_set_block_scaled_decode): the router (with the
+ * fused top-k and counting sort), then the expert kernels of the path the call
+ * takes -- BF16 tensor-core decode: 1 + the combine; block-scaled MXFP4: the x
+ * planes, 1 (T <= 16, FFN <= 2048) or 3 (two projections and the h planes)
+ * kernels, and the combine; the GEMVs: gate/up and down (combine fused).  The
+ * debug-bounds build adds its permutation check.  Host-only, no CUDA call.
+ * Returns 0 when T is 0 or above the decode threshold (the grouped-GEMM path),
+ * -1 for an invalid shape or T < 0. */
+int32_t ft_moe_decode_kernels(const ft_moe_shape* shape, int32_t T);
+
 /* Bound on every pipeline wait of the grouped-GEMM kernels (steps 3 and 4 when
  * T > decode threshold): the time, in ns, a role waits for a stage without
  * progress before it gives up.  Default 4 s (4000000000); ns = 0 restores the

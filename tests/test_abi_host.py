@@ -259,3 +259,35 @@ def test_tma_probe_rejects_bad_arguments_on_host():
         with pytest.raises(F.FtError) as ei:
             F.ft_tma_read_probe(mode, buf, n, region, status, stream=0)
         assert ei.value.status == F.FT_ERR_INVALID_ARG
+
+
+def test_decode_kernel_count_follows_the_dispatch():
+    """ft_moe_decode_kernels: router + the expert kernels of the path a decode-sized layer call
+    takes (host-only).  BF16: GEMVs (gate/up, down with the combine) or the tensor-core decode
+    (one kernel + combine) -- three either way; MXFP4: GEMVs below 4 tokens, then the x planes +
+    the fused block-scaled kernel + combine up to 16 tokens, then two projection launches and
+    the h planes; nothing above the decode threshold."""
+    if "FTMOE_LIB" in __import__("os").environ:
+        pytest.skip("counts are for the normal build")
+    qwen, gemma, dsv4 = _shape("qwen3_a3b"), _shape("gemma4_26b_a4b"), _shape("dsv4_flash")
+    for T in (1, 3, 4, 16, 32):
+        assert F.ft_moe_decode_kernels(qwen, T) == 3
+        assert F.ft_moe_decode_kernels(gemma, T) == 3
+    assert [F.ft_moe_decode_kernels(dsv4, T) for T in (1, 3, 4, 8, 16, 17, 32)] == [3, 3, 4, 4, 4, 6, 6]
+    wide = F.make_shape(1024, 4096, 24, 4, 0, F.FT_W_MXFP4)        # FFN > 2048: two launches
+    assert F.ft_moe_decode_kernels(wide, 8) == 6
+    assert F.ft_moe_decode_kernels(dsv4, 0) == 0 and F.ft_moe_decode_kernels(dsv4, 33) == 0
+    assert F.ft_moe_decode_kernels(dsv4, -1) == -1
+    assert F.ft_moe_decode_kernels(F.make_shape(1000, 768, 128, 8), 4) == -1   # invalid shape
+    prev = F.ft_set_block_scaled_decode(0)
+    try:
+        assert F.ft_moe_decode_kernels(dsv4, 8) == 3                # GEMVs only
+        F.ft_set_block_scaled_decode(1)
+        assert F.ft_moe_decode_kernels(dsv4, 1) == 4                # block-scaled at every size
+    finally:
+        F.ft_set_block_scaled_decode(prev)
+    prev_max = F.ft_set_decode_max_tokens(8)
+    try:
+        assert F.ft_moe_decode_kernels(qwen, 8) == 3 and F.ft_moe_decode_kernels(qwen, 9) == 0
+    finally:
+        F.ft_set_decode_max_tokens(prev_max)
