@@ -124,11 +124,13 @@ const char* ft_last_error(void);
 /* Library version string. */
 const char* ft_version(void);
 
-/* Token-count threshold of the decode path: T <= this uses the memory-bound
- * GEMV kernels (128-bit weight streaming, fused down-projection + combine);
- * larger T uses the tcgen05 grouped GEMM.  Default 32, or the environment
- * variable FT_DECODE_MAX_TOKENS read at load time.  Process-wide; returns the
- * previous value.  Values < 0 are rejected (returns -1). */
+/* Token-count threshold of the decode path: T <= this uses the weight-streaming
+ * decode kernels (the tcgen05 decode on BF16 or block-scaled MXFP4 weights for
+ * batches that qualify, else the 128-bit GEMVs with the down projection and the
+ * combine fused; ft_moe_decode_kernels tells which); larger T uses the tcgen05
+ * grouped GEMM.  Default 32, or the environment variable FT_DECODE_MAX_TOKENS
+ * read at load time.  Process-wide; returns the previous value.  Values < 0 are
+ * rejected (returns -1). */
 int32_t ft_set_decode_max_tokens(int32_t t);
 int32_t ft_get_decode_max_tokens(void);
 
