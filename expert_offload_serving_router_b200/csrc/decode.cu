@@ -359,13 +359,10 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
         if (rpb && R <= kMaxDecodeRows) {
             DownBulkCfg c{rpb, int(size_t(rpb) * wrow), na_max, R};
             const size_t dsm = need(rpb);
-            static bool attr[2] = {false, false};
+            static PerDeviceOnce attr[2];
             auto kern = mx ? decode_down_bulk_kernel<true> : decode_down_bulk_kernel<false>;
-            if (!attr[mx]) {
-                e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kBulkSmem));
-                if (e != cudaSuccess) return e;
-                attr[mx] = true;
-            }
+            e = attr[mx]([&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kBulkSmem)); });
+            if (e != cudaSuccess) return e;
             e = launch_pdl(kern, dim3(a.H / rpb), dim3(256), dsm, st, a, c);
             if (e != cudaSuccess) return e;
             return cudaGetLastError();

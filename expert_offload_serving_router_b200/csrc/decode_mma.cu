@@ -297,14 +297,16 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st) {
     // within a few microseconds, measured) and never more than the items a batch can have.  Were
     // a CTA ever kept from running by other work, a waiting down item gives up after the bounded
     // wait and the call reports a timeout.
-    static bool attrs_set = false;
-    if (!attrs_set) {
-        cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e == cudaSuccess)   // the whole unified L1 / shared array as shared memory
-            e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                     int(cudaSharedmemCarveoutMaxShared));
+    static PerDeviceOnce attrs;
+    {
+        const cudaError_t e = attrs([&] {
+            cudaError_t r = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            if (r == cudaSuccess)   // the whole unified L1 / shared array as shared memory
+                r = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         int(cudaSharedmemCarveoutMaxShared));
+            return r;
+        });
         if (e != cudaSuccess) return e;
-        attrs_set = true;
     }
     const int cap = 3 * num_sms();
     const int max_items = na_max * (p.gu_blocks + p.dn_blocks);

@@ -1026,12 +1026,12 @@ cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
     if (decode_mx_fused(a)) {
         // x planes, then gate/up and down in one persistent launch (h planes written by its epilogue)
         constexpr size_t fsmem = dec_mx_fused_smem();
-        static bool fattr = false;
-        if (!fattr) {
-            cudaError_t e = cudaFuncSetAttribute(decode_mx_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 int(fsmem));
+        static PerDeviceOnce fattr;
+        {
+            const cudaError_t e = fattr([&] {
+                return cudaFuncSetAttribute(decode_mx_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsmem));
+            });
             if (e != cudaSuccess) return e;
-            fattr = true;
         }
         DecMxFusedParams f{};
         f.T = T; f.k = k; f.E = E; f.H = H; f.F = F; f.G = G; f.NB = NB;
@@ -1059,13 +1059,15 @@ cudaError_t launch_decode_mx(const DecodeArgs& a, cudaStream_t st) {
         return cudaGetLastError();
     }
     constexpr size_t smem = dec_mx_smem();
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(decode_mx_mma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(decode_mx_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    static PerDeviceOnce attr;
+    {
+        const cudaError_t e = attr([&] {
+            cudaError_t r = cudaFuncSetAttribute(decode_mx_mma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(decode_mx_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            return r;
+        });
         if (e != cudaSuccess) return e;
-        attr = true;
     }
     const int cap = num_sms();            // persistent: one CTA per SM (ring and scale atoms fill shared memory)
     cudaError_t e = launch_dep(quant2_kernel, (32 * (H / 32) + 255) / 256, 256, 0, st, a.x, T, 32, H, xh, xl, xsh, xsl);

@@ -407,10 +407,11 @@ int launch_moe_gemm_mx_pair(const GemmLaunch& L, const GemmParams& p0, cudaStrea
     }
     constexpr size_t smem = mx_pair_smem_bytes();
     static int max_clusters = 0;
-    if (!max_clusters) {
-        if (cudaFuncSetAttribute(moe_gemm_mx_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-            cudaSuccess)
-            return 2;
+    static PerDeviceOnce attr;
+    if (attr([&] { return cudaFuncSetAttribute(moe_gemm_mx_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)); }) !=
+        cudaSuccess)
+        return 2;
+    if (!max_clusters) {   // the same on every device of one model: queried once
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3(2 * (num_sms() / 2));
         cfg.blockDim = dim3(kMxThreads);

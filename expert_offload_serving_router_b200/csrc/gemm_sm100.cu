@@ -504,12 +504,10 @@ template <bool MX, int HV>
 static int launch_variant(int grid, cudaStream_t st, const CUtensorMap& tw, const CUtensorMap& tsw, const CUtensorMap* tb,
                           const GemmParams& p) {
     const size_t smem = gemm_smem_bytes(HV);
-    static bool set = false;
-    if (!set) {
-        if (cudaFuncSetAttribute(moe_gemm_kernel<MX, HV>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-            return 2;
-        set = true;
-    }
+    static PerDeviceOnce attr;
+    if (attr([&] { return cudaFuncSetAttribute(moe_gemm_kernel<MX, HV>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)); }) !=
+        cudaSuccess)
+        return 2;
     moe_gemm_kernel<MX, HV><<<grid, 320, smem, st>>>(tw, tsw, tb[0], tb[1], tb[2], tb[3], tb[4], p);
     return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
@@ -533,10 +531,11 @@ static int launch_pair(const GemmLaunch& L, const GemmParams& p, const CUtensorM
     }
     static int max_clusters = 0;
     constexpr size_t smem = C::smem();
-    if (!max_clusters) {
-        if (cudaFuncSetAttribute(moe_gemm_pair_kernel<HPC>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-            cudaSuccess)
-            return 2;
+    static PerDeviceOnce attr;
+    if (attr([&] { return cudaFuncSetAttribute(moe_gemm_pair_kernel<HPC>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)); }) !=
+        cudaSuccess)
+        return 2;
+    if (!max_clusters) {   // the same on every device of one model: queried once
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3(2 * (num_sms() / 2));
         cfg.blockDim = dim3(320);

@@ -115,11 +115,10 @@ extern "C" ft_status ft_tma_read_probe(int32_t mode, const void* buf, size_t byt
         return fail(FT_ERR_INVALID_ARG, "ft_tma_read_probe: tensor map");
     const int tiles = int(rows / 128 / size_t(nsm));    // every CTA's rows lie inside the buffer
     const int smem = kTpSt * kTpSlot + 1024;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(tma_read_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    static PerDeviceOnce attr;
+    {
+        const cudaError_t e = attr([&] { return cudaFuncSetAttribute(tma_read_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); });
         if (e != cudaSuccess) return cuda_ok(e, "tma probe attribute");
-        attr = true;
     }
     tma_read_probe_kernel<<<nsm, 64, smem, static_cast<cudaStream_t>(stream)>>>(tm, tiles, mode, int(grows ? grows : 4), status);
     return cuda_ok(cudaGetLastError(), "tma probe launch");

@@ -280,12 +280,9 @@ cudaError_t launch_route_tc(int T, int H, int E, int k, const uint16_t* x, const
     while (stages > 1 && rc_smem(stages, NP) > size_t(kRcSmemCap)) --stages;
     const size_t smem = rc_smem(stages, NP);
     if (smem > size_t(kRcSmemCap)) return cudaErrorInvalidConfiguration;
-    static bool attr = false;
-    if (!attr) {
-        e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRcSmemCap);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static PerDeviceOnce attr;
+    e = attr([&] { return cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRcSmemCap); });
+    if (e != cudaSuccess) return e;
     const int tiles = (T + kRcTok - 1) / kRcTok;
     RcParams p{};
     p.T = T; p.Tpad = tiles * kRcTok; p.H = H; p.NP = NP; p.stages = stages;

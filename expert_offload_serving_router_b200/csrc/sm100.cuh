@@ -222,4 +222,22 @@ inline bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
 }
 int num_sms();
 
+// One-time setup per device: a kernel's cudaFuncSetAttribute values belong to the current
+// device's copy of it, so the flag is per device ordinal (devices past the table repeat the
+// setup on every call, which is correct, only slower).
+struct PerDeviceOnce {
+    static constexpr int kDevices = 64;
+    bool done[kDevices] = {};
+    template <typename Fn>
+    cudaError_t operator()(Fn&& fn) {
+        int d = -1;
+        if (cudaGetDevice(&d) != cudaSuccess) d = -1;
+        const bool slot = d >= 0 && d < kDevices;
+        if (slot && done[d]) return cudaSuccess;
+        const cudaError_t e = fn();
+        if (e == cudaSuccess && slot) done[d] = true;
+        return e;
+    }
+};
+
 }  // namespace ftmoe
