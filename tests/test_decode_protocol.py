@@ -15,7 +15,8 @@ sequences (gate/up items, then down items of one or more groups), and the checke
   and accumulators in TMEM -- is written while a reader may still use it (write after read);
 * every reader finds the data of the item it is for (read after write).
 
-Planted mistakes (one wait dropped from one role) must each be caught.  The cross-CTA readiness
+The two-launch form (`decode_mx_mma_kernel<0/1>`) is checked the same way at each of its buffer
+plans.  Planted mistakes (one wait dropped from one role) must each be caught.  The cross-CTA readiness
 counters lie outside one CTA's protocol (their bounded waits are covered by the GPU tests):
 here every group's h is ready from the start.
 """
@@ -200,9 +201,9 @@ def build_protocol(items, nk, drop=None):
     return roles, bars, R
 
 
-def run(items, nk, seed, drop=None):
+def run(items, nk, seed, drop=None, protocol=None):
     rng = random.Random(seed)
-    roles, bars, _ = build_protocol(items, nk, drop)
+    roles, bars, _ = (protocol or build_protocol)(items, nk, drop)
     cur = {name: next(g, None) for name, g in roles.items()}
     inflight = {"mma": [], "cp": []}          # per issuing thread: commit effects, in issue order
 
@@ -243,6 +244,170 @@ def run(items, nk, seed, drop=None):
     stuck = {name: act for name, act in cur.items() if act is not None}
     if stuck:
         raise Violation(f"deadlock: {stuck}")
+
+
+def build_protocol_two(mode, nact, nwb):
+    """Roles of one CTA of `decode_mx_mma_kernel<mode>` (the two-launch form): a contiguous run
+    of items; the epilogue warps also lay out the next item's atoms (before the current item's
+    epilogue); nwb weight-atom buffers in shared memory and nact activation-scale buffers in
+    TMEM (1 of each when the contraction is too long for two).  Gate/up (mode 0): every item
+    multiplies x, whose atoms sit in weight buffer 1's place until item 0's copies are done;
+    down (mode 1): the group's activation atoms have a region of their own."""
+    def protocol(items, nk, drop=None):
+        n = len(items)
+        keys = [(g if mode else -1) for _, g in items]
+        act_new = [j == 0 or keys[j] != keys[j - 1] for j in range(n)]
+        run_of, r = [], -1
+        for j in range(n):
+            r += act_new[j]
+            run_of.append(r)
+        act_of = [None] * n
+        for j in range(n):
+            act_of[j] = j if act_new[j] else act_of[j - 1]
+        bars = {}
+        for s in range(ST):
+            bars[("full", s)] = Bar(1)
+            bars[("empty", s)] = Bar(1)
+        for b in range(2):
+            for nm in ("tfull", "tempty", "atoms_full", "atoms_free", "sf_ready"):
+                bars[(nm, b)] = Bar(1)
+        R = Regions()
+
+        def smem_w(j):
+            return [("smem_w", j % nwb)]
+
+        def smem_act(j):
+            return [("smem_w", 1)] if mode == 0 else [("smem_act",)]
+
+        def tmem_act(j):
+            return [("tmem_act", run_of[j] % nact)]
+
+        def W(role, bar, parity, means):
+            return None if drop == (role, bar[0]) else ("wait", bar, parity, means)
+
+        def A(bar):
+            return ("arrive", bar)
+
+        def F(fn):
+            return ("fn", fn)
+
+        def producer():
+            step = 0
+            for j in range(n):
+                for kb in range(nk(mode == 1)):
+                    s, ph = step % ST, (step // ST) & 1
+                    yield W("producer", ("empty", s), ph ^ 1, step // ST - 1)
+                    yield F(lambda s=s, j=j: R.write(("stage", s), f"TMA of item {j}"))
+                    yield F(lambda s=s, j=j, kb=kb: R.fill(("stage", s), (j, kb)))
+                    yield A(("full", s))
+                    step += 1
+
+        def mma():
+            step = 0
+            for j in range(n):
+                b = j & 1
+                yield W("mma", ("sf_ready", b), (j >> 1) & 1, j >> 1)
+                yield W("mma", ("tempty", b), ((j >> 1) & 1) ^ 1, (j >> 1) - 1)
+                yield F(lambda j=j, b=b: R.write(("acc", b), f"MMAs of item {j}"))
+                yield F(lambda j=j, b=b: R.read(("tmem_w", b), ("mma", j), j))
+                for t in tmem_act(j):
+                    yield F(lambda t=t, j=j: R.read(t, ("mma", j), act_of[j]))
+                for kb in range(nk(mode == 1)):
+                    s, ph = step % ST, (step // ST) & 1
+                    yield W("mma", ("full", s), ph, step // ST)
+                    yield F(lambda s=s, j=j, kb=kb: R.read(("stage", s), ("mma", j, kb), (j, kb)))
+                    yield ("commit", "mma", [F(lambda s=s, j=j, kb=kb: R.done(("stage", s), ("mma", j, kb))),
+                                             A(("empty", s))])
+                    step += 1
+                yield ("commit", "mma", [F(lambda j=j, b=b: [R.done(t, ("mma", j)) for t in [("tmem_w", b)] + tmem_act(j)]),
+                                         F(lambda j=j, b=b: R.fill(("acc", b), j)),
+                                         F(lambda j=j, b=b: R.readers.setdefault(("acc", b), set()).add(("epi", j))),
+                                         A(("tfull", b))])
+
+        def copier():
+            for j in range(n):
+                b, wb = j & 1, j % nwb
+                yield W("copier", ("atoms_full", wb), (j // nwb) & 1, j // nwb)
+                if j >= 2:
+                    yield W("copier", ("tfull", b), ((j - 2) >> 1) & 1, (j - 2) >> 1)
+                if act_new[j] and nact == 1 and j >= 1:
+                    yield W("copier", ("tfull", (j - 1) & 1), ((j - 1) >> 1) & 1, (j - 1) >> 1)
+                src = [(x, j) for x in smem_w(j)] + ([(x, act_of[j]) for x in smem_act(j)] if act_new[j] else [])
+                dst = [(("tmem_w", b), j)] + ([(t, act_of[j]) for t in tmem_act(j)] if act_new[j] else [])
+                for t, _ in dst:
+                    yield F(lambda t=t, j=j: R.write(t, f"scale copies of item {j}"))
+                for x, want in src:
+                    yield F(lambda x=x, want=want, j=j: R.read(x, ("cp", j), want))
+                yield ("commit", "cp", [F(lambda src=src, j=j: [R.done(x, ("cp", j)) for x, _ in src]),
+                                        F(lambda dst=dst: [R.fill(t, tag) for t, tag in dst]),
+                                        A(("sf_ready", b)), A(("atoms_free", wb))])
+
+        def epilogue_builders():
+            def copied(x):
+                return W("epilogue", ("atoms_free", x % nwb), (x // nwb) & 1, x // nwb)
+
+            def build(j):
+                regions = smem_w(j) + (smem_act(j) if act_new[j] else [])
+                for x in regions:
+                    yield F(lambda x=x, j=j: R.write(x, f"atoms of item {j}"))
+                yield F(lambda j=j, regions=regions: [R.fill(x, j) for x in regions])
+                yield A(("atoms_full", j % nwb))
+            yield from build(0)
+            for j in range(n):
+                if j + 1 < n:
+                    if j + 1 >= nwb:
+                        yield copied(j + 1 - nwb)
+                    if act_new[j + 1] or (mode == 0 and j == 0):
+                        yield copied(j)
+                    yield from build(j + 1)
+                b = j & 1
+                yield W("epilogue", ("tfull", b), (j >> 1) & 1, j >> 1)
+                yield F(lambda j=j, b=b: R.read(("acc", b), ("epi", j), j))
+                yield F(lambda j=j, b=b: R.done(("acc", b), ("epi", j)))
+                yield A(("tempty", b))
+
+        def strip(gen):
+            return (a for a in gen if a is not None)
+
+        roles = {"producer": strip(producer()), "mma": strip(mma()), "copier": strip(copier()),
+                 "epilogue": strip(epilogue_builders())}
+        return roles, bars, R
+    return protocol
+
+
+@pytest.mark.parametrize("mode,nact,nwb", [(0, 1, 2), (1, 2, 2), (1, 1, 1), (1, 2, 1), (1, 1, 2)])
+def test_two_launch_decode_protocol_random_interleavings(mode, nact, nwb):
+    """The two-launch kernel at every buffer plan its host side can pick: gate/up (one x scale
+    buffer, two weight-atom buffers), down with K <= 3072 (two and two) and longer K (one
+    activation-scale buffer in TMEM, one weight-atom buffer), plus the mixed plans."""
+    rng = random.Random(mode * 7 + nact * 3 + nwb)
+    proto = build_protocol_two(mode, nact, nwb)
+    for _ in range(40):
+        n = rng.choice([1, 2, 3, 5, 9, 14])
+        g, groups = rng.randrange(4), []
+        for _ in range(n):
+            if rng.random() < 0.3:
+                g += 1
+            groups.append(g)
+        items = [(mode == 1, gg) for gg in groups]
+        for seed in range(10):
+            run(items, lambda down: 3 if down else 5, seed, protocol=proto)
+
+
+# (In this form the MMA thread's wait for the epilogue to hand an accumulator back is implied:
+# item j + 2's scale atoms are laid out by the same warps only after item j's epilogue, so the
+# model finds no race without it; the waits below are the ones whose absence is one.)
+@pytest.mark.parametrize("drop", [("copier", "tfull"), ("epilogue", "atoms_free"), ("mma", "sf_ready"),
+                                  ("copier", "atoms_full"), ("producer", "empty")])
+def test_two_launch_checker_catches_a_dropped_wait(drop):
+    proto = build_protocol_two(1, 1, 1)
+    items = [(True, 0), (True, 0), (True, 1), (True, 1), (True, 2), (True, 3)]
+    for seed in range(400):
+        try:
+            run(items, lambda down: 3, seed, drop=drop, protocol=proto)
+        except Violation:
+            return
+    raise AssertionError(f"dropping the {drop[0]}'s wait on {drop[1]} went unnoticed")
 
 
 def item_lists(rng, count=60):
