@@ -16,9 +16,10 @@ sequences (gate/up items, then down items of one or more groups), and the checke
 * every reader finds the data of the item it is for (read after write).
 
 The two-launch form (`decode_mx_mma_kernel<0/1>`) is checked the same way at each of its buffer
-plans.  Planted mistakes (one wait dropped from one role) must each be caught.  The cross-CTA readiness
-counters lie outside one CTA's protocol (their bounded waits are covered by the GPU tests):
-here every group's h is ready from the start.
+plans.  Planted mistakes (one wait dropped from one role) must each be caught.  The single-CTA
+checks take every group's h as written; a multi-CTA check runs whole launches with the
+cross-CTA counters (waits for all of a group's gate/up epilogues, two counted reads per down
+item, reset by the last).
 """
 import random
 
@@ -63,10 +64,35 @@ class Regions:
         self.readers.setdefault(r, set()).discard(tag)
 
 
-def build_protocol(items, nk, drop=None):
+class Groups:
+    """The cross-CTA counters of a launch: per group, the gate/up epilogue arrivals (ready once
+    all of the group's gate/up items have written their h planes) and the reads of down items
+    (two per down item: its producer after the wait, its copier once the item's atoms exist);
+    the last read resets both."""
+
+    def __init__(self, n_groups, gu_blocks, dn_blocks):
+        self.h, self.reads = [0] * n_groups, [0] * n_groups
+        self.gu, self.dn = gu_blocks, dn_blocks
+
+    def ready(self, g):
+        return self.h[g] >= self.gu
+
+    def h_done(self, g):
+        self.h[g] += 1
+
+    def read_done(self, g):
+        if not self.ready(g):
+            raise Violation(f"a read of group {g} counted before all its h was written")
+        self.reads[g] += 1
+        if self.reads[g] == 2 * self.dn:
+            self.h[g], self.reads[g] = 0, 0
+
+
+def build_protocol(items, nk, drop=None, glob=None):
     """Roles of one CTA for `items` = [(down, group)] (its items in order) and nk(down) = the
     item's 256-deep stages.  drop = (role, barrier name): leave that role's waits on that barrier
-    out (a planted mistake).  Returns (roles, barriers, regions)."""
+    out (a planted mistake).  glob: the launch's Groups when several CTAs are modelled (without
+    it every group's h counts as written).  Returns (roles, barriers, regions)."""
     n = len(items)
     keys = [(g if d else -1) for d, g in items]
     act_new = [j == 0 or keys[j] != keys[j - 1] for j in range(n)]
@@ -119,6 +145,11 @@ def build_protocol(items, nk, drop=None):
     def producer():
         step = 0
         for j in range(n):
+            if glob and items[j][0]:
+                g = items[j][1]
+                if drop != ("producer", "group"):
+                    yield ("spin", lambda g=g: glob.ready(g))
+                yield F(lambda g=g: glob.read_done(g))
             for kb in range(nk(items[j][0])):
                 s, ph = step % ST, (step // ST) & 1
                 yield W("producer", ("empty", s), ph ^ 1, step // ST - 1)
@@ -155,6 +186,8 @@ def build_protocol(items, nk, drop=None):
         for j in range(n):
             b = j & 1
             yield W("copier", ("atoms_full", b), (j >> 1) & 1, j >> 1)
+            if glob and items[j][0]:
+                yield F(lambda g=items[j][1]: glob.read_done(g))
             if j >= 2:
                 yield W("copier", ("tfull", b), ((j - 2) >> 1) & 1, (j - 2) >> 1)
             if first_down[j]:
@@ -179,6 +212,8 @@ def build_protocol(items, nk, drop=None):
                 yield copied(0)
             if j >= 1 and act_new[j] and items[j][0]:
                 yield copied(j - 1)
+            if glob and act_new[j] and items[j][0] and drop != ("builders", "group"):   # h scales are read
+                yield ("spin", lambda g=items[j][1]: glob.ready(g))
             regions = smem_w(j) + (smem_act(j) if act_new[j] else [])
             for x in regions:
                 yield F(lambda x=x, j=j: R.write(x, f"builders of item {j}"))
@@ -192,6 +227,8 @@ def build_protocol(items, nk, drop=None):
             yield F(lambda j=j, b=b: R.read(("acc", b), ("epi", j), j))
             yield F(lambda j=j, b=b: R.done(("acc", b), ("epi", j)))
             yield A(("tempty", b))
+            if glob and not items[j][0]:                    # h planes stored, then the count
+                yield F(lambda g=items[j][1]: glob.h_done(g))
 
     def strip(gen):
         return (a for a in gen if a is not None)
@@ -496,3 +533,102 @@ def test_checker_catches_the_missing_first_down_wait():
     finally:
         g["build_protocol"] = orig
     assert caught
+
+
+def run_launch(ctas, nk, glob, seed, drop=None):
+    """Several CTAs' roles under one random schedule (CTA roles and commit streams with random
+    speeds); the launch must finish and leave every group's counters at zero."""
+    rng = random.Random(seed)
+    roles, bars, inflight, cur, speed = {}, {}, {}, {}, {}
+    for c, items in enumerate(ctas):
+        r, b, _ = build_protocol(items, nk, drop=drop, glob=glob)
+        for name, gen in r.items():
+            roles[(c, name)] = gen
+            cur[(c, name)] = next(gen, None)
+            speed[(c, name)] = rng.choice([0.02, 0.3, 1.0, 1.0, 3.0])
+        bars[c] = b
+        for t in ("mma", "cp"):                      # commit streams, keyed apart from the roles
+            inflight[(c, t, "q")] = []
+            speed[(c, t, "q")] = rng.choice([0.05, 1.0, 3.0])
+
+    def ok(key, act):
+        if act[0] == "spin":
+            return act[1]()
+        if act[0] != "wait":
+            return True
+        bar, parity, means = act[1:]
+        b = bars[key[0]][bar]
+        if (b.done & 1) == parity:
+            return False
+        if b.done != means + 1:
+            raise Violation(f"CTA {key[0]}: wait on {bar} for phase {means} passed after {b.done}")
+        return True
+
+    for _ in range(10 ** 7):
+        runnable = [k for k, a in cur.items() if a is not None and ok(k, a)]
+        runnable += [k for k, q in inflight.items() if q]
+        if not runnable:
+            break
+        k = rng.choices(runnable, weights=[speed[x] for x in runnable])[0]
+        if k in inflight:
+            for act in inflight[k].pop(0):
+                if act[0] == "arrive":
+                    bars[k[0]][act[1]].arrive()
+                else:
+                    act[1]()
+            continue
+        act = cur[k]
+        if act[0] == "commit":
+            inflight[(k[0], act[1], "q")].append(act[2])
+        elif act[0] == "arrive":
+            bars[k[0]][act[1]].arrive()
+        elif act[0] == "fn":
+            act[1]()
+        cur[k] = next(roles[k], None)
+    stuck = {k: a for k, a in cur.items() if a is not None}
+    if stuck:
+        raise Violation(f"deadlock: {stuck}")
+    if any(glob.h) or any(glob.reads):
+        raise Violation(f"counters left at h={glob.h} reads={glob.reads}")
+
+
+@pytest.mark.parametrize("n_act,gu_blocks,dn_blocks,grid", [(3, 2, 3, 4), (2, 4, 2, 3), (5, 1, 1, 7),
+                                                             (1, 3, 5, 9), (4, 3, 2, 5)])
+def test_fused_decode_launch_cross_cta(n_act, gu_blocks, dn_blocks, grid):
+    """The whole launch: items b, b + grid, ... of [gate/up items | down items] per CTA (some
+    CTAs start on down items), down items waiting for their group's gate/up epilogues in other
+    CTAs and their own; every schedule finishes with the counters back at zero."""
+    gu = [(False, g) for g in range(n_act) for _ in range(gu_blocks)]
+    dn = [(True, g) for g in range(n_act) for _ in range(dn_blocks)]
+    lst = gu + dn
+    ctas = [lst[b::grid] for b in range(min(grid, len(lst)))]
+    for seed in range(40):
+        run_launch(ctas, lambda down: 2, Groups(n_act, gu_blocks, dn_blocks), seed)
+
+
+class EarlyReset(Groups):
+    """A planted counting mistake: the counters reset after the producers' reads alone."""
+
+    def read_done(self, g):
+        if not self.ready(g):
+            raise Violation(f"a read of group {g} counted before all its h was written")
+        self.reads[g] += 1
+        if self.reads[g] == self.dn:
+            self.h[g], self.reads[g] = 0, 0
+
+
+@pytest.mark.parametrize("mistake", ["producer-wait", "builders-wait", "early-reset"])
+def test_cross_cta_checker_catches_mistakes(mistake):
+    n_act, gu_blocks, dn_blocks, grid = 3, 2, 3, 4
+    gu = [(False, g) for g in range(n_act) for _ in range(gu_blocks)]
+    dn = [(True, g) for g in range(n_act) for _ in range(dn_blocks)]
+    lst = gu + dn
+    ctas = [lst[b::grid] for b in range(grid)]
+    drop = {"producer-wait": ("producer", "group"), "builders-wait": ("builders", "group")}.get(mistake)
+    kind = EarlyReset if mistake == "early-reset" else Groups
+    for seed in range(300):
+        try:
+            run_launch(ctas, lambda down: 2, kind(n_act, gu_blocks, dn_blocks), seed, drop=drop)
+        except Violation:
+            return
+    raise AssertionError(f"{mistake} went unnoticed")
