@@ -1,5 +1,6 @@
-"""Model check of the mbarrier protocol of one CTA of the fused block-scaled decode kernel
-(`decode_mx_fused_kernel`, csrc/decode_mx_mma.cu), on the CPU.
+"""Model check, on the CPU, of the mbarrier and cross-CTA protocols of the tensor-core decode
+kernels: the fused block-scaled decode (`decode_mx_fused_kernel`, csrc/decode_mx_mma.cu), its
+two-launch form, and the BF16 tensor-core decode (`decode_mma_kernel`, csrc/decode_mma.cu).
 
 Each role of the CTA -- TMA producer, MMA issuer, scale copier, atom builders, epilogue -- is a
 sequence of steps written from the kernel: waits (mbarrier parity waits with the hardware's
@@ -535,13 +536,13 @@ def test_checker_catches_the_missing_first_down_wait():
     assert caught
 
 
-def run_launch(ctas, nk, glob, seed, drop=None):
+def run_launch(ctas, nk, glob, seed, drop=None, protocol=None):
     """Several CTAs' roles under one random schedule (CTA roles and commit streams with random
     speeds); the launch must finish and leave every group's counters at zero."""
     rng = random.Random(seed)
     roles, bars, inflight, cur, speed = {}, {}, {}, {}, {}
     for c, items in enumerate(ctas):
-        r, b, _ = build_protocol(items, nk, drop=drop, glob=glob)
+        r, b, _ = (protocol or build_protocol)(items, nk, drop=drop, glob=glob)
         for name, gen in r.items():
             roles[(c, name)] = gen
             cur[(c, name)] = next(gen, None)
@@ -632,3 +633,114 @@ def test_cross_cta_checker_catches_mistakes(mistake):
         except Violation:
             return
     raise AssertionError(f"{mistake} went unnoticed")
+
+
+class GroupsBF16(Groups):
+    """The BF16 tensor-core decode counts one read per down item (its producer's): the last of
+    dn_blocks resets the group."""
+
+    def read_done(self, g):
+        if not self.ready(g):
+            raise Violation(f"a read of group {g} counted before all its h was written")
+        self.reads[g] += 1
+        if self.reads[g] == self.dn:
+            self.h[g], self.reads[g] = 0, 0
+
+
+def build_protocol_bf16(items, nk, drop=None, glob=None, stages=3):
+    """Roles of one CTA of the BF16 tensor-core decode (`decode_mma_kernel`, csrc/decode_mma.cu):
+    a 3-stage ring, two accumulators, no scale factors; items b, b + grid, ... of [gate/up |
+    down]; the producer waits for a down item's group before its first load and counts the read;
+    the gate/up epilogue hands the accumulator back, stores h and counts itself."""
+    n = len(items)
+    bars = {}
+    for s_ in range(stages):
+        bars[("full", s_)] = Bar(1)
+        bars[("empty", s_)] = Bar(1)
+    for b in range(2):
+        bars[("tfull", b)] = Bar(1)
+        bars[("tempty", b)] = Bar(1)
+    R = Regions()
+
+    def W(role, bar, parity, means):
+        return None if drop == (role, bar[0]) else ("wait", bar, parity, means)
+
+    def producer():
+        step = 0
+        for j in range(n):
+            if glob and items[j][0]:
+                g = items[j][1]
+                if drop != ("producer", "group"):
+                    yield ("spin", lambda g=g: glob.ready(g))
+                yield ("fn", lambda g=g: glob.read_done(g))
+            for kb in range(nk(items[j][0])):
+                s_, ph = step % stages, (step // stages) & 1
+                yield W("producer", ("empty", s_), ph ^ 1, step // stages - 1)
+                yield ("fn", lambda s_=s_, j=j: R.write(("stage", s_), f"TMA of item {j}"))
+                yield ("fn", lambda s_=s_, j=j, kb=kb: R.fill(("stage", s_), (j, kb)))
+                yield ("arrive", ("full", s_))
+                step += 1
+
+    def mma():
+        step = 0
+        for j in range(n):
+            b = j & 1
+            yield W("mma", ("tempty", b), ((j >> 1) & 1) ^ 1, (j >> 1) - 1)
+            yield ("fn", lambda j=j, b=b: R.write(("acc", b), f"MMAs of item {j}"))
+            for kb in range(nk(items[j][0])):
+                s_, ph = step % stages, (step // stages) & 1
+                yield W("mma", ("full", s_), ph, step // stages)
+                yield ("fn", lambda s_=s_, j=j, kb=kb: R.read(("stage", s_), ("mma", j, kb), (j, kb)))
+                yield ("commit", "mma", [("fn", lambda s_=s_, j=j, kb=kb: R.done(("stage", s_), ("mma", j, kb))),
+                                         ("arrive", ("empty", s_))])
+                step += 1
+            yield ("commit", "mma", [("fn", lambda j=j, b=b: R.fill(("acc", b), j)),
+                                     ("fn", lambda j=j, b=b: R.readers.setdefault(("acc", b), set()).add(("epi", j))),
+                                     ("arrive", ("tfull", b))])
+
+    def epilogue():
+        for j in range(n):
+            b = j & 1
+            yield W("epilogue", ("tfull", b), (j >> 1) & 1, j >> 1)
+            yield ("fn", lambda j=j, b=b: R.read(("acc", b), ("epi", j), j))
+            yield ("fn", lambda j=j, b=b: R.done(("acc", b), ("epi", j)))
+            yield ("arrive", ("tempty", b))
+            if glob and not items[j][0]:
+                yield ("fn", lambda g=items[j][1]: glob.h_done(g))
+
+    def strip(gen):
+        return (a for a in gen if a is not None)
+
+    roles = {"producer": strip(producer()), "mma": strip(mma()), "epilogue": strip(epilogue())}
+    return roles, bars, R
+
+
+@pytest.mark.parametrize("n_act,gu_blocks,dn_blocks,grid", [(3, 2, 3, 4), (2, 4, 2, 3), (5, 1, 1, 7),
+                                                             (1, 3, 5, 9), (6, 2, 4, 12)])
+def test_bf16_decode_launch_cross_cta(n_act, gu_blocks, dn_blocks, grid):
+    """The BF16 tensor-core decode's whole launch (several CTAs per SM in the kernel: here as
+    many independent CTAs), with its producer-only read count."""
+    gu = [(False, g) for g in range(n_act) for _ in range(gu_blocks)]
+    dn = [(True, g) for g in range(n_act) for _ in range(dn_blocks)]
+    lst = gu + dn
+    ctas = [lst[b::grid] for b in range(min(grid, len(lst)))]
+    for seed in range(40):
+        run_launch(ctas, lambda down: 2 if down else 3, GroupsBF16(n_act, gu_blocks, dn_blocks), seed,
+                   protocol=build_protocol_bf16)
+
+
+@pytest.mark.parametrize("drop", [("producer", "group"), ("mma", "tempty"), ("producer", "empty"),
+                                  ("epilogue", "tfull"), ("mma", "full")])
+def test_bf16_checker_catches_mistakes(drop):
+    n_act, gu_blocks, dn_blocks, grid = 3, 2, 3, 4
+    gu = [(False, g) for g in range(n_act) for _ in range(gu_blocks)]
+    dn = [(True, g) for g in range(n_act) for _ in range(dn_blocks)]
+    lst = gu + dn
+    ctas = [lst[b::grid] for b in range(grid)]
+    for seed in range(300):
+        try:
+            run_launch(ctas, lambda down: 2, GroupsBF16(n_act, gu_blocks, dn_blocks), seed, drop=drop,
+                       protocol=build_protocol_bf16)
+        except Violation:
+            return
+    raise AssertionError(f"dropping the {drop[0]}'s wait on {drop[1]} went unnoticed")
