@@ -48,6 +48,9 @@ def lib():
         L.oracle_e8m0_to_f64.restype = dbl
         L.oracle_e8m0_to_f64.argtypes = [ctypes.c_uint8]
         L.oracle_decode_matrix.argtypes = [i32, P, P, i64, i64, P]
+        L.oracle_e4m3_to_f64.restype = dbl
+        L.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        L.oracle_decode_nvfp4.argtypes = [P, P, ctypes.c_float, i64, i64, P]
         L.oracle_router_logits.argtypes = [i32, i32, i32, P, P, P, P, P]
         L.oracle_topk.argtypes = [i32, i32, i32, P, P, P]
         L.oracle_permute.argtypes = [i32, i32, i32, i32, P, P, P, P]
@@ -86,6 +89,18 @@ def e2m1_to_f64(code) -> float:
 
 def e8m0_to_f64(b) -> float:
     return lib().oracle_e8m0_to_f64(int(b))
+
+
+def e4m3_to_f64(b) -> float:
+    return lib().oracle_e4m3_to_f64(int(b))
+
+
+def decode_nvfp4(codes, scales, tensor_scale: float, rows: int, cols: int) -> np.ndarray:
+    """NVFP4 [rows, cols] to fp64: E2M1 codes (two per byte), E4M3 scale per 16, fp32 tensor scale."""
+    codes, scales = _c(codes, np.uint8), _c(scales, np.uint8)
+    out = np.empty((rows, cols), dtype=np.float64)
+    lib().oracle_decode_nvfp4(_p(codes), _p(scales), float(tensor_scale), rows, cols, _p(out))
+    return out
 
 
 def decode_matrix(wdtype: int, w, scale, rows: int, cols: int) -> np.ndarray:

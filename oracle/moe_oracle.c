@@ -73,6 +73,34 @@ double oracle_e8m0_to_f64(uint8_t b)
     return ldexp(1.0, (int)b - 127);
 }
 
+/* OCP 8-bit float E4M3 (the MXFP8 element format, and NVFP4's block-scale format): bits
+ * (s, e3 e2 e1 e0, m2 m1 m0), exponent bias 7, no infinities.  Normal (e != 0):
+ * (-1)^s * 2^(e-7) * (1 + m/8); subnormal (e == 0): (-1)^s * 2^-6 * (m/8); S.1111.111 is NaN. */
+double oracle_e4m3_to_f64(uint8_t b)
+{
+    int s = (b >> 7) & 1, e = (b >> 3) & 15, m = b & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = e ? ldexp(1.0 + m / 8.0, e - 7) : ldexp(m / 8.0, -6);
+    return s ? -mag : mag;
+}
+
+/* NVFP4 matrix [rows, cols] to fp64, exact (NVIDIA's 4-bit block format, named on the pages
+ * only as the laptop build's: FreeToken article, dothoosh.com, editorial analysis; the layout
+ * follows its public definition): E2M1 codes packed as for MXFP4 (codes[r][c/2], low nibble =
+ * even c), one E4M3 scale per 16 consecutive elements of a row (scales[r][c/16]), one fp32
+ * scale for the whole tensor; value = E2M1 * E4M3 * tensor_scale.  cols % 16 == 0. */
+void oracle_decode_nvfp4(const uint8_t* codes, const uint8_t* scales, float tensor_scale, long rows, long cols,
+                         double* out)
+{
+    for (long r = 0; r < rows; ++r)
+        for (long c = 0; c < cols; ++c) {
+            uint8_t byte = codes[r * (cols / 2) + c / 2];
+            uint8_t code = (c & 1) ? (byte >> 4) : (byte & 15);
+            out[r * cols + c] = oracle_e2m1_to_f64(code) * oracle_e4m3_to_f64(scales[r * (cols / 16) + c / 16]) *
+                                (double)tensor_scale;
+        }
+}
+
 /* element (r, c) of an MXFP4 matrix with `cols` columns:
  * codes[r][c/2] (low nibble = even c), scales[r][c/32]. */
 static double mx_elem(const uint8_t* codes, const uint8_t* scales, long cols, long r, long c)

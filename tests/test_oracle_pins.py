@@ -402,3 +402,56 @@ def test_lru_resize_worked_example():
 def test_lru_resize_rejects_a_step_larger_than_the_new_budget():
     with pytest.raises(ValueError):
         oracle.lru_sim_resizable(16, 4, [[1, 2], [1, 3, 4], [4]], {1: 2})
+
+
+# ---------------------------------------------------------------- NVFP4 weights (decode only)
+def _e2m1_golden():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "e2m1_ocp_mx_v1.txt")) if l.strip() and not l.startswith("#")]
+    return np.array([float(v) for _, v in sorted((int(c, 2), v) for c, v in rows)])
+
+
+def test_e4m3_decode_matches_torch_float8_for_every_byte():
+    """The oracle's E4M3 byte decode against torch's float8_e4m3fn conversion (an independent
+    implementation of the OCP FP8 E4M3 format), all 256 bytes, NaN included."""
+    import torch
+    ref = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_to_f64(b) for b in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref)) and np.isnan(got).sum() == 2      # 0x7F, 0xFF
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert got[0x7E] == 448.0 and got[0x08] == 2.0 ** -6 and got[0x01] == 2.0 ** -9 and got[0x38] == 1.0
+
+
+def test_e4m3_decode_values_are_the_rounding_grid():
+    """Every finite E4M3 value is a fixed point of the oracle's E4M3 rounding (written apart from
+    the decode, for the MXFP8 study), and the values between consecutive positive codes round
+    to one of the two."""
+    vals = sorted({oracle.e4m3_to_f64(b) for b in range(128) if b != 0x7F})
+    for v in vals:
+        assert oracle.e4m3_round(v) == v and oracle.e4m3_round(-v) == -v
+    for a, b in zip(vals, vals[1:]):
+        assert oracle.e4m3_round((a + b) / 2) in (a, b)
+        assert oracle.e4m3_round(a + (b - a) / 4) == a and oracle.e4m3_round(b - (b - a) / 4) == b
+
+
+def test_nvfp4_decode_matches_tables():
+    """NVFP4 decode = E2M1 value (the OCP table) x E4M3 block scale (torch's conversion) x tensor
+    scale, per element with the block of 16 along the row and the low nibble first; plus one
+    hand-worked row."""
+    import torch
+    rng = np.random.default_rng(3)
+    rows, cols = 5, 64
+    codes = rng.integers(0, 256, size=(rows, cols // 2), dtype=np.uint8)
+    scales = rng.integers(0, 0x7F, size=(rows, cols // 16), dtype=np.uint8)      # positive, not NaN
+    ts = np.float32(0.0625)
+    e2m1 = _e2m1_golden()
+    sc = torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nib = np.stack([codes & 15, codes >> 4], axis=-1).reshape(rows, cols)
+    want = e2m1[nib] * np.repeat(sc, 16, axis=1) * float(ts)
+    assert np.array_equal(oracle.decode_nvfp4(codes, scales, ts, rows, cols), want)
+    # row by hand: codes 0x7 (6.0) and 0xF (-6.0) alternating, block scales 1.0 (0x38) and 2^-6 (0x08)
+    c1 = np.full((1, 16), 0xF7, dtype=np.uint8)
+    s1 = np.array([[0x38, 0x08]], dtype=np.uint8)
+    got = oracle.decode_nvfp4(c1, s1, np.float32(0.5), 1, 32)[0]
+    assert np.array_equal(got[:16], np.tile([3.0, -3.0], 8))
+    assert np.array_equal(got[16:], np.tile([6.0 * 2 ** -7, -6.0 * 2 ** -7], 8))
