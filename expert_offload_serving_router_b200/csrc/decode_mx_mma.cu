@@ -6,8 +6,9 @@
 // copy of the activations loses too much (the error study: 5.6e-2 of max|y| on the
 // DeepSeek-V4-Flash-shaped layer, over the 3e-2 tolerance), so each activation row is carried as
 // two planes -- hi = the OCP MX conversion of v, lo = the same conversion of v - hi, each with its
-// own E8M0 scale per 32 (1.2e-3 of max|y| in the study) -- and every K step issues one MMA per
-// plane into the same fp32 accumulator.
+// own E8M0 scale per 32 (1.2e-3 of max|y| in the study).  Both planes form one B operand of
+// 2 NB rows (hi rows, then lo rows), so each 32-deep K block is one MMA, and the epilogue adds
+// accumulator column c and column NB + c.
 //
 //   quant2_kernel:  bf16 rows -> E4M3 planes hi, lo [rows, K] + E8M0 scales [rows, K/32] each.
 //   decode_mx_mma_kernel<MODE>: items (active group, 128 weight rows), a contiguous run of them per
