@@ -387,6 +387,16 @@ def measure_decode(torch, F, L, tokens, rank, hbm_gbs, nrot=4):
     return out
 
 
+def guarded(name, fn):
+    """Run one auxiliary measurement (rank-local: no collectives inside) so that a failure is
+    reported in the line, as {"error": ...}, instead of ending the run before the headline prints."""
+    try:
+        return fn()
+    except Exception as ex:  # the headline line must still be printed
+        print(f"bench: {name} failed: {ex!r}", file=sys.stderr, flush=True)
+        return {"error": f"{type(ex).__name__}: {ex}"}
+
+
 def measure_e2e(torch, dist, F, L, ctx, T, steps, warmup, world):
     """Same metric through the public whole-layer call with pinned host buffers: every step
     copies x host->device, runs ft_moe_layer_forward and copies y device->host.  The copies
@@ -776,7 +786,8 @@ def main():
     tc_peak = tc_sus if pre["total_ms"] > 1000.0 else tc_burst
     traffic = recorded_traffic(*ROOFLINE_SUMMARY)
     e2e = None if args.no_e2e else measure_e2e(torch, dist, F, L, pre["ctx"], T, args.steps, args.warmup, world)
-    decode = None if args.no_decode else measure_decode(torch, F, L, dec_tokens or HEADLINE_DECODE, rank, hbm_gbs)
+    decode = None if args.no_decode else guarded(
+        "decode", lambda: measure_decode(torch, F, L, dec_tokens or HEADLINE_DECODE, rank, hbm_gbs))
     headline_ms = pre["ms_step"]
     del L, pre["ctx"]
     torch.cuda.empty_cache()
@@ -784,16 +795,17 @@ def main():
     if not args.no_extra:
         extra = {}
         for name, Tds in EXTRA_WORKLOADS:
-            Tp = PREFILL_SIZES[name]
-            c = inputs.CONFIGS[name]
-            Lx = Layer(torch, F, c, inputs.make_layer(c, seed=0))
-            px = measure_prefill(torch, F, Lx, Tp, 10, 3, torch.cuda.current_stream(), rank)
-            extra[name] = {"prefill": summarize_prefill(px, hbm_gbs, tc_burst)}
-            if Tds and not args.no_decode:
-                extra[name]["decode"] = measure_decode(torch, F, Lx, Tds, rank, hbm_gbs)
-            del Lx, px
+            def one(name=name, Tds=Tds):
+                c = inputs.CONFIGS[name]
+                Lx = Layer(torch, F, c, inputs.make_layer(c, seed=0))
+                px = measure_prefill(torch, F, Lx, PREFILL_SIZES[name], 10, 3, torch.cuda.current_stream(), rank)
+                out = {"prefill": summarize_prefill(px, hbm_gbs, tc_burst)}
+                if Tds and not args.no_decode:
+                    out["decode"] = measure_decode(torch, F, Lx, Tds, rank, hbm_gbs)
+                return out
+            extra[name] = guarded(name, one)
             torch.cuda.empty_cache()
-    stack = None if args.no_stack else measure_stack(torch, F, rank, hbm_gbs)
+    stack = None if args.no_stack else guarded("offload stack", lambda: measure_stack(torch, F, rank, hbm_gbs))
     if stack and "prefill" in stack:
         # copy time per layer from the pinned-copy probe, compute time per layer from the same
         # layer shape measured resident (the headline DSV4-Flash-shaped prefill at the stack's T)

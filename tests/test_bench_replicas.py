@@ -67,3 +67,17 @@ def test_overlap_efficiency_formula():
     assert bench.overlap_efficiency(60.0, 5.0, 8, 2 * (60 * 8 + 5)) == pytest.approx(0.5)
     # compute-bound layers: ideal = copy + 7 * compute + compute
     assert bench.overlap_efficiency(2.0, 10.0, 8, 2.0 + 80.0) == pytest.approx(1.0)
+
+
+def test_failed_auxiliary_measurement_is_reported_not_fatal(capsys):
+    """A decode / other-workload / stack measurement that raises leaves an error entry in the
+    line; the headline still prints."""
+    import bench
+
+    def boom():
+        raise RuntimeError("device check failed")
+
+    assert bench.guarded("decode", lambda: {"T1": 1.0}) == {"T1": 1.0}
+    out = bench.guarded("decode", boom)
+    assert out == {"error": "RuntimeError: device check failed"}
+    assert "decode failed" in capsys.readouterr().err
